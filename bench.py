@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Throughput of the BitLinear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the "square" workload
+(one BitLinear 2048 -> 2048, 4096 tokens per GPU, bf16 X / dY, fp32 latent W):
+weight quantisation (absmean + ternary round + 2-bit pack), RMSNorm + int8 activation
+quantisation, the int8 x ternary contraction, the straight-through backward (grad
+input GEMM, RMSNorm backward, grad weight GEMM), and a 16-token decode GEMV over the
+freshly packed weights.  With N > 1 GPUs each rank holds its own 4096 tokens (weak
+scaling) and the weight gradient is summed over ranks with an NCCL all-reduce.
+
+Prints one JSON line (rank 0).  Inputs are synthetic and seeded (bit_ternary_qat_b200.synth).
+L2 is flushed (a 512 MB write) before every timed step; each step is timed with CUDA
+events on the launching stream, the per-rank sum is max-reduced over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+T_TOK, D_IN, D_OUT = 4096, 2048, 2048
+DECODE_B = 16
+METRIC = "BitLinear fwd+bwd tokens/s & % of TC peak; packed-ternary GEMV HBM GB/s"
+WORKLOAD = "square: BitLinear 2048->2048, 4096 tokens/GPU, bf16 X/dY, fp32 W; quant+fwd+bwd+16-token decode GEMV"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "bit_ternary_qat_b200", "csrc")
+    for f in sorted(os.listdir(cdir)):
+        with open(os.path.join(cdir, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        if d.get("src_sha") != kernel_src_hash():
+            return None
+        v = d.get("kernels", {}).get(kernel_key, {}).get("dram_bytes_per_launch")
+        return None if v is None else float(v)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ------------------------------------------------------------------------------------
+
+def oracle_step(ora, li, t_s: int):
+    """The oracle's pass over the hot path on the first t_s tokens (weight quantisation
+    over the full W).  Returns seconds."""
+    X = li.X[:t_s].float().numpy()
+    dY = li.dY[:t_s].float().numpy()
+    W = li.W.numpy()
+    t0 = time.perf_counter()
+    gamma, wq = ora.quant_weight(W)
+    packed = ora.pack(wq)
+    r = ora.rmsnorm_rinv(X, 1e-6)
+    xq, s, xdq = ora.act_quant(X, r, None)
+    acc = ora.int_gemm(xq, wq)
+    ora.linear_epilogue(acc, gamma, s)
+    xdq_b = ora.bf16_bits_to_f32(ora.round_bf16(xdq))
+    dxh = ora.grad_input_hat(dY, wq, gamma)
+    ora.rmsnorm_backward(X, r, None, dxh)
+    ora.grad_weight(dY, xdq_b)
+    b = min(DECODE_B, t_s)
+    ora.gemv(packed, gamma, W.shape[1], xq[:b], s[:b])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(target_s: float = 15.0):
+    import oracle as ora
+    from bit_ternary_qat_b200 import synth
+    ora.build()
+    li = synth.workload_inputs("square")[0]
+    t_s = 64
+    dt = oracle_step(ora, li, t_s)
+    while dt < target_s / 4 and t_s < T_TOK:
+        t_s = min(T_TOK, t_s * 4)
+        dt = oracle_step(ora, li, t_s)
+    return {"value": t_s / dt, "unit": "tokens/s", "cores": ora.num_threads(), "kind": "oracle",
+            "sample": f"one oracle step on {t_s} of the {T_TOK} tokens of the square workload "
+                      f"(weight quantisation over the full 2048x2048 W included), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle as ora
+    from bit_ternary_qat_b200 import synth
+    ora.build()
+    li = synth.workload_inputs("square")[0]
+    t_s = 256
+    for _ in range(args.warmup):
+        oracle_step(ora, li, t_s)
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += oracle_step(ora, li, t_s)
+    value = t_s * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens_per_step": t_s},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": ora.num_threads(),
+                         "sample": f"each step: the oracle on {t_s} of {T_TOK} tokens (full weight quantisation)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------
+# the CUDA path
+# ------------------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import bit_ternary_qat_b200 as bl
+    from bit_ternary_qat_b200 import build as blbuild, synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    if rank == 0:
+        blbuild.build()
+    if world > 1:
+        dist.barrier()
+    bl.load()
+
+    # ---------------------------------------------------------------- inputs (HBM resident)
+    wl = synth.WORKLOADS["square"]
+    gen = synth.generator(wl.seed)
+    W_h = synth.normal((D_OUT, D_IN), synth.W_STD, gen)                  # same W on every rank
+    gen_r = synth.generator(wl.seed * 1000 + rank)                       # rank's own tokens
+    X_h = synth.normal((T_TOK, D_IN), 1.0, gen_r).to(torch.bfloat16)
+    dY_h = synth.normal((T_TOK, D_OUT), synth.DY_STD_BF16, gen_r).to(torch.bfloat16)
+    W, X, dY = W_h.to(dev), X_h.to(dev), dY_h.to(dev)
+
+    f32, bf16, i8, u8 = torch.float32, torch.bfloat16, torch.int8, torch.uint8
+    bufs = dict(
+        gamma=torch.empty(1, dtype=f32, device=dev), wq_i8=torch.empty(D_OUT, D_IN, dtype=i8, device=dev),
+        wq_bf16=torch.empty(D_OUT, D_IN, dtype=bf16, device=dev),
+        packed=torch.empty(D_OUT, D_IN // 4, dtype=u8, device=dev),
+        xq=torch.empty(T_TOK, D_IN, dtype=i8, device=dev), sx=torch.empty(T_TOK, dtype=f32, device=dev),
+        rinv=torch.empty(T_TOK, dtype=f32, device=dev), xdq=torch.empty(T_TOK, D_IN, dtype=bf16, device=dev),
+        y=torch.empty(T_TOK, D_OUT, dtype=bf16, device=dev), dX=torch.empty(T_TOK, D_IN, dtype=f32, device=dev),
+        dW=torch.empty(D_OUT, D_IN, dtype=f32, device=dev), dg=torch.empty(D_IN, dtype=f32, device=dev),
+        ydec=torch.empty(DECODE_B, D_OUT, dtype=f32, device=dev),
+        ws=bl.workspace(T_TOK, D_OUT, D_IN, dev))
+    flush = torch.empty(512 * 1024 * 1024, dtype=u8, device=dev)        # > 126 MB L2
+
+    # names of the timed pieces, in step order (each is one public call)
+    PIECES = ["quant_weight", "act_quant", "linear_i8", "grad_input", "rmsnorm_bwd", "grad_weight",
+              "allreduce_dW", "decode_gemv"]
+
+    def step(ev=None, inputs=None):
+        b = bufs
+        Wi, Xi, dYi = inputs if inputs is not None else (W, X, dY)
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        bl.bitlinear_quant_weight(Wi, ws=b["ws"], out=b)
+        rec(1)
+        bl.bitlinear_act_quant(Xi, apply_rmsnorm=True, out=b)
+        rec(2)
+        bl.bitlinear_linear(b["xq"], b["sx"], b["wq_i8"], b["gamma"], y=b["y"])
+        rec(3)
+        bl.bitlinear_grad_input(dYi, b["wq_bf16"], b["gamma"], dXhat=b["dX"])
+        rec(4)
+        bl.bitlinear_rmsnorm_backward(Xi, b["rinv"], b["dX"], ws=b["ws"], dg=b["dg"])
+        rec(5)
+        bl.bitlinear_backward_weight(dYi, b["xdq"], dW=b["dW"])
+        rec(6)
+        if world > 1:
+            dist.all_reduce(b["dW"])
+        rec(7)
+        bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B], y=b["ydec"])
+        rec(8)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+            torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- warm-up
+    for _ in range(max(3, args.warmup)):
+        step()
+    sync_all()
+    assert bl.check_device_status() == 0
+
+    # ---------------------------------------------------------------- timed region
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(K)]
+    gpu_uuid = None
+    try:
+        gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_uuid = str(local)
+    clk = ClockSampler(gpu_uuid) if rank == 0 else None
+    launches0 = bl.launch_count()
+    sync_all()
+    if clk:
+        clk.start()
+        time.sleep(0.3)
+    for i in range(K):
+        flush.zero_()                       # evict L2 (outside the timed events)
+        step(evs[i])
+    sync_all()
+    clocks = clk.stop() if clk else None
+    launches = bl.launch_count() - launches0
+    per_step = [e[0].elapsed_time(e[8]) for e in evs]
+    piece_ms = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, p in enumerate(PIECES)}
+    tot_ms = sum(per_step)
+    t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    tot_ms = float(t.item())
+    assert bl.check_device_status() == 0
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        W_p, X_p, dY_p = W_h.pin_memory(), X_h.pin_memory(), dY_h.pin_memory()
+        W_d, X_d, dY_d = torch.empty_like(W), torch.empty_like(X), torch.empty_like(dY)
+        dW_p = torch.empty(D_OUT, D_IN, dtype=f32).pin_memory()
+        g_p = torch.empty(1, dtype=f32).pin_memory()
+        h2d = W_p.numel() * 4 + X_p.numel() * 2 + dY_p.numel() * 2
+        d2h = dW_p.numel() * 4 + 4
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(2):
+            W_d.copy_(W_p, non_blocking=True); X_d.copy_(X_p, non_blocking=True); dY_d.copy_(dY_p, non_blocking=True)
+            step(inputs=(W_d, X_d, dY_d))
+            dW_p.copy_(bufs["dW"], non_blocking=True); g_p.copy_(bufs["gamma"], non_blocking=True)
+        sync_all()
+        for i in range(K):
+            flush.zero_()
+            es[i][0].record()
+            W_d.copy_(W_p, non_blocking=True); X_d.copy_(X_p, non_blocking=True); dY_d.copy_(dY_p, non_blocking=True)
+            step(inputs=(W_d, X_d, dY_d))
+            dW_p.copy_(bufs["dW"], non_blocking=True); g_p.copy_(bufs["gamma"], non_blocking=True)
+            es[i][1].record()
+        sync_all()
+        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in es)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": T_TOK * world * K / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---------------------------------------------------------------- decode GEMV (28672 x 8192)
+    gemv = None
+    if not args.no_gemv and rank == 0:
+        gemv = gemv_measure(bl, torch, dev, flush, peaks())
+
+    if world > 1:
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # ---------------------------------------------------------------- roofline of the dominant kernel
+    pk = peaks()
+    gemm_flops = 2.0 * T_TOK * D_OUT * D_IN
+    gemm_pieces = {"linear_i8": "int8", "grad_input": "bf16", "grad_weight": "bf16"}
+    dom = max(gemm_pieces, key=lambda p: piece_ms[p])
+    dom_ms = piece_ms[dom]
+    achieved = gemm_flops / (dom_ms * 1e-3) / 1e12
+    if gemm_pieces[dom] == "bf16":
+        peak, peak_note = pk["bf16_sust"], f"bf16 sustained ({pk['src']})"
+    else:
+        peak, peak_note = 2.0 * pk["bf16_sust"], f"int8 = 2 x bf16 sustained ({pk['src']}; nominal 4.5/2.25 ratio)"
+    kernel_names = {"linear_i8": "tc_gemm_kernel<int8,K,K,256,linear>",
+                    "grad_input": "tc_gemm_kernel<bf16,K,MN,256,scale_f32>",
+                    "grad_weight": "tc_gemm_kernel<bf16,MN,MN,256,f32>"}
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": ncu_traffic(dom), "kernel": kernel_names[dom], "peak_kind": peak_note,
+                "launch_ms": dom_ms}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline()
+
+    value = T_TOK * world * K / (tot_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": tot_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s8+bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": T_TOK, "d_in": D_IN, "d_out": D_OUT,
+                   "decode_batch": DECODE_B, "parallelism": f"dp{world}",
+                   "l2": "flushed before every timed step (512 MB write)"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "pieces_ms": {k: round(v, 5) for k, v in piece_ms.items()},
+        "gemm_tflops": {p: gemm_flops / (piece_ms[p] * 1e-3) / 1e12 for p in gemm_pieces},
+        "decode_gemv": gemv,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def gemv_measure(bl, torch, dev, flush, pk):
+    """Decode GEMV on the 28672 x 8192 packed weight at batch 1, 4, 16 (L2 flushed)."""
+    from bit_ternary_qat_b200 import synth
+    N, K = 28672, 8192
+    W, _ = synth.decode_inputs(1, N, K)
+    q = bl.bitlinear_quant_weight(W.to(dev), want_i8=False, want_bf16=False)
+    del W
+    out = {}
+    for B in (1, 4, 16):
+        _, x = synth.decode_inputs(B, 16, K, seed=40 + B)
+        aq = bl.bitlinear_act_quant(x.to(dev), apply_rmsnorm=False, want_xdq=False)
+        y = torch.empty(B, N, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            bl.ternary_gemv(q["packed"], q["gamma"], K, aq["xq"], aq["sx"], y=y)
+        reps = 20
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in es:
+            flush.zero_()
+            a.record()
+            bl.ternary_gemv(q["packed"], q["gamma"], K, aq["xq"], aq["sx"], y=y)
+            b.record()
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in es)
+        nbytes = N * K // 4 + B * K + 4 * B + 4 * B * N + 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[f"B{B}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / pk["hbm"],
+                        "int_ops_T": 2.0 * B * N * K / (ms * 1e-3) / 1e12}
+    out["hbm_peak_GBs"] = pk["hbm"]
+    out["workload"] = "decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192], L2 flushed"
+    return out
+
+
+if __name__ == "__main__":
+    main()

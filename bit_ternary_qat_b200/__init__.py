@@ -1,22 +1,21 @@
 """B200-native BitNet b1.58 BitLinear hot path.
 
-The compute lives in ``libbitlinear.so`` (hand-written sm_100a CUDA kernels behind a
-C ABI declared in ``include/bitlinear.h``).  This package only marshals arguments
-into that library: it loads it lazily on first use and raises if it is missing --
-there is no CPU fallback.
+The compute lives in ``libbitlinear.so`` (hand-written sm_100a CUDA kernels behind the
+C ABI declared in ``include/bitlinear.h``).  This package only marshals arguments into
+that library (``ops``): the library is loaded on the first call and every call raises
+if it is missing -- there is no CPU fallback.
 """
-from . import synth  # noqa: F401  (seeded inputs; no layer arithmetic)
+from . import synth  # noqa: F401  (seeded inputs; none of the layer's arithmetic)
+from . import ops  # noqa: F401
+from .ops import (  # noqa: F401
+    bitlinear_act_quant, bitlinear_backward, bitlinear_backward_input, bitlinear_backward_weight,
+    bitlinear_grad_input, bitlinear_rmsnorm_backward,
+    bitlinear_forward, bitlinear_linear, bitlinear_quant_weight, check_device_status, launch_count,
+    selftest_bounded_wait, set_wait_limit_ns, ternary_gemv, ternary_pack, workspace, workspace_bytes,
+)
 
 
 def load():
-    """Load the CUDA library (raises if it is not built)."""
+    """Load the CUDA library now (raises if it is not built)."""
     from . import _lib
     return _lib.lib()
-
-
-def __getattr__(name):
-    from . import ops
-    try:
-        return getattr(ops, name)
-    except AttributeError:
-        raise AttributeError(name) from None

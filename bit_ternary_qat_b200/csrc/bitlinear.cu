@@ -1,0 +1,530 @@
+// bitlinear.cu -- C ABI of the BitLinear hot path (declared in include/bitlinear.h).
+//
+// Host side only: argument validation (before any CUDA call, so a bad call launches
+// nothing), TMA tensor-map encoding, grid sizing and kernel launches.  All arithmetic
+// of the path happens in the kernels included below; nothing here touches the data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/bitlinear.h"
+#include "common.cuh"
+#include "act_quant.cuh"
+#include "weight_quant.cuh"
+#include "gemm_tc.cuh"
+#include "gemm_simt.cuh"
+#include "rmsnorm_bwd.cuh"
+#include "gemv.cuh"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+
+bl_status fail(bl_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+#define BL_REQUIRE(cond, status, ...)                  \
+    do {                                               \
+        if (!(cond)) return fail(status, __VA_ARGS__); \
+    } while (0)
+
+#define BL_TRY(expr)                     \
+    do {                                 \
+        bl_status _s = (expr);           \
+        if (_s != BL_OK) return _s;      \
+    } while (0)
+
+bl_status check_dims(int64_t T, int64_t N, int64_t K) {
+    BL_REQUIRE(T >= 1 && N >= 1 && K >= 1, BL_ERR_INVALID_ARG, "sizes must be positive (T=%lld N=%lld K=%lld)",
+               (long long)T, (long long)N, (long long)K);
+    BL_REQUIRE(T <= kMaxDim && N <= kMaxDim && K <= kMaxDim, BL_ERR_UNSUPPORTED_SHAPE, "sizes must be < 2^31");
+    BL_REQUIRE(K % 32 == 0, BL_ERR_UNSUPPORTED_SHAPE, "K (d_in) must be a multiple of 32, got %lld", (long long)K);
+    BL_REQUIRE(N % 16 == 0, BL_ERR_UNSUPPORTED_SHAPE, "N (d_out) must be a multiple of 16, got %lld", (long long)N);
+    return BL_OK;
+}
+
+bl_status check_ptr(const void* p, const char* name, bool required) {
+    if (p == nullptr) {
+        BL_REQUIRE(!required, BL_ERR_INVALID_ARG, "%s must not be NULL", name);
+        return BL_OK;
+    }
+    BL_REQUIRE(aligned16(p), BL_ERR_MISALIGNED, "%s must be 16-byte aligned", name);
+    return BL_OK;
+}
+
+bl_status check_dtype(bl_dtype dt) {
+    BL_REQUIRE(dt == BL_F32 || dt == BL_BF16, BL_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    return BL_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// device checks
+// ------------------------------------------------------------------------------------
+struct DeviceInfo {
+    int sms = 0;
+    int major = 0;
+    int max_smem_optin = 0;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+bool g_dev_ok[64] = {};
+
+bl_status current_device(DeviceInfo* out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    BL_REQUIRE(dev >= 0 && dev < 64, BL_ERR_DEVICE, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev_ok[dev]) {
+        DeviceInfo d;
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
+        if (d.major != 10) return fail(BL_ERR_DEVICE, "device %d is sm_%d0; this library is built for sm_100a", dev, d.major);
+        g_dev[dev] = d;
+        g_dev_ok[dev] = true;
+    }
+    *out = g_dev[dev];
+    return BL_OK;
+}
+
+bl_status launched(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return BL_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// TMA tensor maps
+// ------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer x inner] with 128-byte swizzled boxes [box_outer x box_inner].
+bl_status make_tmap(CUtensorMap* tm, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+                    uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    BL_REQUIRE(fn != nullptr, BL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const uint64_t esize = bf16 ? 2 : 1;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * esize};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    BL_REQUIRE(r == CUDA_SUCCESS, BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return BL_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// tcgen05 GEMM launcher
+// ------------------------------------------------------------------------------------
+constexpr int kBN = 256;
+
+template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
+bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, bl::TcGemmArgs a, cudaStream_t st,
+                    const DeviceInfo& dev) {
+    auto kern = bl::tc_gemm_kernel<kInt8, kAMN, kBMN, kBN, kEpi>;
+    const size_t smem = bl::tc_smem_bytes<kBN>();
+    BL_REQUIRE((int)smem <= dev.max_smem_optin, BL_ERR_DEVICE, "GEMM needs %zu bytes of shared memory", smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    a.m_tiles = (a.M + bl::kTcBM - 1) / bl::kTcBM;
+    a.n_tiles = (a.N + kBN - 1) / kBN;
+    const int kb_elems = kInt8 ? 128 : 64;
+    a.k_blocks = (a.K + kb_elems - 1) / kb_elems;
+    a.wait_ns = g_wait_ns.load();
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = tiles < dev.sms ? tiles : dev.sms;
+    kern<<<grid, bl::kTcThreads, smem, st>>>(ta, tb, a);
+    return launched("tc_gemm");
+}
+
+// ------------------------------------------------------------------------------------
+// pieces shared by the entry points (validation already done by the caller)
+// ------------------------------------------------------------------------------------
+bl_status run_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int apply_norm, const float* g,
+                        float eps, int8_t* Xq, float* sx, float* rinv, void* Xdq, cudaStream_t st) {
+    if (x_dt == BL_BF16)
+        bl::act_quant_kernel<true><<<(unsigned)T, bl::kActThreads, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx,
+                                                                            rinv, Xdq);
+    else
+        bl::act_quant_kernel<false><<<(unsigned)T, bl::kActThreads, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx,
+                                                                             rinv, Xdq);
+    return launched("act_quant");
+}
+
+bl_status run_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq, const float* gamma,
+                     int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
+    CUtensorMap ta, tb;
+    BL_TRY(make_tmap(&ta, Xq, false, (uint64_t)K, (uint64_t)T, 128, 128));
+    BL_TRY(make_tmap(&tb, Wq, false, (uint64_t)K, (uint64_t)N, 128, kBN));
+    bl::TcGemmArgs a{};
+    a.M = (int)T; a.N = (int)N; a.K = (int)K;
+    a.out = Y; a.ldo = N; a.out_bf16 = y_dt == BL_BF16 ? 1 : 0;
+    a.acc_out = acc; a.row_scale = sx; a.gamma = gamma;
+    return launch_tc<true, false, false, bl::kEpiLinear>(ta, tb, a, st, dev);
+}
+
+bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf16, const float* gamma, int64_t T,
+                              int64_t K, int64_t N, float* dXhat, cudaStream_t st, const DeviceInfo& dev) {
+    if (dt == BL_BF16) {
+        CUtensorMap ta, tb;
+        BL_TRY(make_tmap(&ta, dY, true, (uint64_t)N, (uint64_t)T, 64, 128));      // dY, K-major (contraction N)
+        BL_TRY(make_tmap(&tb, Wq_bf16, true, (uint64_t)K, (uint64_t)N, 64, 64));  // W_q, MN-major (rows = N)
+        bl::TcGemmArgs a{};
+        a.M = (int)T; a.N = (int)K; a.K = (int)N;
+        a.out = dXhat; a.ldo = K; a.gamma = gamma;
+        return launch_tc<false, false, true, bl::kEpiScaleF32>(ta, tb, a, st, dev);
+    }
+    // fp32 layer: CUDA-core fp32 contraction, C[t,k] = gamma * sum_n dY[t,n] W_q[n,k]
+    dim3 grid((unsigned)((K + 63) / 64), (unsigned)((T + 63) / 64));
+    bl::simt_gemm_kernel<float, uint16_t><<<grid, 256, 0, st>>>((int)T, (int)K, (int)N,
+                                                               static_cast<const float*>(dY), N, 1, Wq_bf16, 1, K,
+                                                               gamma, dXhat, K);
+    return launched("simt_gemm(grad_input)");
+}
+
+bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int64_t T, int64_t K, int64_t N,
+                               float* dW, cudaStream_t st, const DeviceInfo& dev) {
+    if (dt == BL_BF16) {
+        CUtensorMap ta, tb;
+        BL_TRY(make_tmap(&ta, dY, true, (uint64_t)N, (uint64_t)T, 64, 64));    // dY^T: MN-major (n contiguous)
+        BL_TRY(make_tmap(&tb, Xdq, true, (uint64_t)K, (uint64_t)T, 64, 64));   // X_dq: MN-major (k contiguous)
+        bl::TcGemmArgs a{};
+        a.M = (int)N; a.N = (int)K; a.K = (int)T;
+        a.out = dW; a.ldo = K;
+        return launch_tc<false, true, true, bl::kEpiF32>(ta, tb, a, st, dev);
+    }
+    dim3 grid((unsigned)((K + 63) / 64), (unsigned)((N + 63) / 64));
+    bl::simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>((int)N, (int)K, (int)T, static_cast<const float*>(dY),
+                                                            1, N, static_cast<const float*>(Xdq), 1, K, nullptr, dW,
+                                                            K);
+    return launched("simt_gemm(grad_weight)");
+}
+
+size_t quant_ws_bytes() { return sizeof(double) * bl::kWqMaxPartials; }
+size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdBlocks * (size_t)K; }
+
+bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const float* g, float* dX, int64_t T,
+                          int64_t K, float* dg, void* ws, cudaStream_t st) {
+    const int grid = (int)(T < bl::kBwdBlocks ? T : bl::kBwdBlocks);
+    float* partial = dg != nullptr ? static_cast<float*>(ws) : nullptr;
+    const size_t smem = dg != nullptr ? sizeof(float) * (size_t)K : 0;
+    if (smem > 48 * 1024) {
+        cudaError_t e = dt == BL_BF16
+                            ? cudaFuncSetAttribute(bl::rmsnorm_bwd_kernel<true>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                            : cudaFuncSetAttribute(bl::rmsnorm_bwd_kernel<false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    }
+    if (dt == BL_BF16)
+        bl::rmsnorm_bwd_kernel<true><<<grid, bl::kBwdThreads, smem, st>>>(X, rinv, g, dX, (int)T, (int)K, partial);
+    else
+        bl::rmsnorm_bwd_kernel<false><<<grid, bl::kBwdThreads, smem, st>>>(X, rinv, g, dX, (int)T, (int)K, partial);
+    BL_TRY(launched("rmsnorm_bwd"));
+    if (dg != nullptr) {
+        bl::dg_reduce_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(partial, grid, (int)K, dg);
+        BL_TRY(launched("dg_reduce"));
+    }
+    return BL_OK;
+}
+
+}  // namespace
+
+// ====================================================================================
+// exported C ABI
+// ====================================================================================
+extern "C" {
+
+int bl_abi_version(void) { return BITLINEAR_ABI_VERSION; }
+
+const char* bl_last_error(void) { return g_last_error.c_str(); }
+
+size_t bitlinear_workspace_bytes(int64_t T, int64_t N, int64_t K) {
+    (void)T;
+    (void)N;
+    if (K < 0) K = 0;
+    size_t a = quant_ws_bytes();
+    size_t b = dg_ws_bytes(K);
+    size_t m = a > b ? a : b;
+    return (m + 255) & ~size_t(255);
+}
+
+void bl_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? 2000000000ull : ns); }
+
+uint64_t bl_launch_count(void) { return g_launches.load(); }
+
+bl_status bl_check_device_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+    int v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, bl::g_bl_status, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(bl::g_bl_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "status word: %s", cudaGetErrorString(e));
+    if (v != 0) return fail((bl_status)v, "a kernel reported status %d (bounded wait expired)", v);
+    return BL_OK;
+}
+
+bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
+                                 uint8_t* Wpacked, float* gamma, void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", false));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_ptr(ws, "ws", true));
+    BL_TRY(check_dims(1, N, K));
+    BL_REQUIRE(ws_bytes >= quant_ws_bytes(), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu",
+               quant_ws_bytes(), ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = N * K;
+    const int parts = bl::wq_num_partials(n);
+    double* partials = static_cast<double*>(ws);
+    bl::absmean_partial_kernel<<<parts, bl::kWqThreads, 0, st>>>(W, n, partials);
+    BL_TRY(launched("absmean_partial"));
+    const int64_t groups = n / 16;
+    int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
+    const int64_t cap = (int64_t)dev.sms * 8;
+    if (blocks > cap) blocks = cap;
+    bl::ternary_quant_kernel<<<(unsigned)blocks, bl::kWqThreads, 0, st>>>(W, n, partials, parts, Wq_i8, Wq_bf16,
+                                                                          Wpacked, gamma);
+    return launched("ternary_quant");
+}
+
+bl_status bitlinear_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int apply_rmsnorm, const float* g,
+                              float eps, int8_t* Xq, float* sx, float* rinv, void* Xdq, void* stream) {
+    BL_TRY(check_dtype(x_dt));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(rinv, "rinv", apply_rmsnorm != 0));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(Xdq, "Xdq", false));
+    BL_TRY(check_dims(T, 16, K));
+    BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_act_quant(X, x_dt, T, K, apply_rmsnorm, g, eps, Xq, sx, rinv, Xdq, static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq_i8,
+                           const float* gamma, int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, void* stream) {
+    BL_TRY(check_dtype(y_dt));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Y, "Y", true));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_dims(T, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, y_dt, acc, static_cast<cudaStream_t>(stream), dev);
+}
+
+bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int64_t K, const float* g, float eps,
+                            const int8_t* Wq_i8, const float* gamma, int64_t N, void* Y, int8_t* Xq, float* sx,
+                            float* rinv, void* Xdq, int32_t* acc, void* stream) {
+    BL_TRY(check_dtype(x_dt));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Y, "Y", true));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(rinv, "rinv", true));
+    BL_TRY(check_ptr(Xdq, "Xdq", false));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_dims(T, N, K));
+    BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
+    return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, x_dt, acc, st, dev);
+}
+
+bl_status bitlinear_backward_input(const void* dY, const void* X, bl_dtype dt, int64_t T, int64_t K, int64_t N,
+                                   const float* g, const float* rinv, const uint16_t* Wq_bf16, const float* gamma,
+                                   float* dX, float* dg, void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_dtype(dt));
+    BL_TRY(check_ptr(dY, "dY", true));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(rinv, "rinv", true));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(dX, "dX", true));
+    BL_TRY(check_ptr(dg, "dg", false));
+    BL_TRY(check_ptr(ws, "ws", dg != nullptr));
+    BL_TRY(check_dims(T, N, K));
+    if (dg != nullptr)
+        BL_REQUIRE(ws_bytes >= dg_ws_bytes(K), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", dg_ws_bytes(K),
+                   ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    BL_TRY(run_grad_input_gemm(dY, dt, Wq_bf16, gamma, T, K, N, dX, st, dev));
+    return run_rmsnorm_bwd(X, dt, rinv, g, dX, T, K, dg, ws, st);
+}
+
+bl_status bitlinear_grad_input(const void* dY, bl_dtype dt, int64_t T, int64_t K, int64_t N, const uint16_t* Wq_bf16,
+                               const float* gamma, float* dXhat, void* stream) {
+    BL_TRY(check_dtype(dt));
+    BL_TRY(check_ptr(dY, "dY", true));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(dXhat, "dXhat", true));
+    BL_TRY(check_dims(T, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_grad_input_gemm(dY, dt, Wq_bf16, gamma, T, K, N, dXhat, static_cast<cudaStream_t>(stream), dev);
+}
+
+bl_status bitlinear_rmsnorm_backward(const void* X, bl_dtype dt, int64_t T, int64_t K, const float* g,
+                                     const float* rinv, float* dX_inout, float* dg, void* ws, size_t ws_bytes,
+                                     void* stream) {
+    BL_TRY(check_dtype(dt));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(rinv, "rinv", true));
+    BL_TRY(check_ptr(dX_inout, "dX", true));
+    BL_TRY(check_ptr(dg, "dg", false));
+    BL_TRY(check_ptr(ws, "ws", dg != nullptr));
+    BL_TRY(check_dims(T, 16, K));
+    if (dg != nullptr)
+        BL_REQUIRE(ws_bytes >= dg_ws_bytes(K), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", dg_ws_bytes(K),
+                   ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_rmsnorm_bwd(X, dt, rinv, g, dX_inout, T, K, dg, ws, static_cast<cudaStream_t>(stream));
+}
+
+bl_status bitlinear_backward_weight(const void* dY, const void* Xdq, bl_dtype dt, int64_t T, int64_t K, int64_t N,
+                                    float* dW, void* stream) {
+    BL_TRY(check_dtype(dt));
+    BL_TRY(check_ptr(dY, "dY", true));
+    BL_TRY(check_ptr(Xdq, "Xdq", true));
+    BL_TRY(check_ptr(dW, "dW", true));
+    BL_TRY(check_dims(T, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_grad_weight_gemm(dY, Xdq, dt, T, K, N, dW, static_cast<cudaStream_t>(stream), dev);
+}
+
+bl_status bitlinear_backward(const void* dY, const void* X, const void* Xdq, bl_dtype dt, int64_t T, int64_t K,
+                             int64_t N, const float* g, const float* rinv, const uint16_t* Wq_bf16, const float* gamma,
+                             float* dX, float* dW, float* dg, void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_ptr(Xdq, "Xdq", true));
+    BL_TRY(check_ptr(dW, "dW", true));
+    BL_TRY(bitlinear_backward_input(dY, X, dt, T, K, N, g, rinv, Wq_bf16, gamma, dX, dg, ws, ws_bytes, stream));
+    return bitlinear_backward_weight(dY, Xdq, dt, T, K, N, dW, stream);
+}
+
+bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t* Wpacked, void* stream) {
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", true));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", true));
+    BL_TRY(check_dims(1, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    const int64_t groups = N * K / 16;
+    int64_t blocks = (groups + 255) / 256;
+    if (blocks > (int64_t)dev.sms * 8) blocks = (int64_t)dev.sms * 8;
+    bl::ternary_pack_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(Wq_i8, N * K, Wpacked);
+    return launched("ternary_pack");
+}
+
+bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
+                       const float* sx, int64_t B, float* y, int32_t* acc, void* stream) {
+    BL_TRY(check_ptr(Wpacked, "Wpacked", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(xq, "xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(y, "y", true));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_dims(1, N, K));
+    BL_REQUIRE(B >= 1 && B <= 16, BL_ERR_UNSUPPORTED_SHAPE, "batch must be in [1, 16], got %lld", (long long)B);
+    BL_REQUIRE(K <= 65536, BL_ERR_UNSUPPORTED_SHAPE, "K must be <= 65536 for the GEMV, got %lld", (long long)K);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t smem = (size_t)B * (size_t)K;   // B x K/16 groups x 16 bytes
+    BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
+               "GEMV stages B*K = %zu activation bytes in shared memory; at most %d fit", smem, dev.max_smem_optin);
+    const int rows_per_block = bl::kGemvWarps;
+    int64_t need = (N + rows_per_block - 1) / rows_per_block;
+#define BL_GEMV_CASE(NBV)                                                                                          \
+    {                                                                                                              \
+        auto kern = bl::ternary_gemv_kernel<NBV>;                                                                  \
+        if (smem > 48 * 1024) {                                                                                    \
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
+            if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));     \
+        }                                                                                                          \
+        int per_sm = 0;                                                                                            \
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kGemvThreads, smem);                      \
+        if (per_sm < 1) per_sm = 1;                                                                                \
+        int64_t grid = (int64_t)dev.sms * per_sm;                                                                  \
+        if (grid > need) grid = need;                                                                              \
+        kern<<<(unsigned)grid, bl::kGemvThreads, smem, st>>>(Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, y,   \
+                                                             acc);                                                 \
+    }
+    if (B == 1) BL_GEMV_CASE(1)
+    else if (B <= 4) BL_GEMV_CASE(4)
+    else BL_GEMV_CASE(16)
+#undef BL_GEMV_CASE
+    return launched("ternary_gemv");
+}
+
+bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+    BL_REQUIRE(limit_ns > 0 && limit_ns <= 10000000000ull, BL_ERR_INVALID_ARG, "limit must be in (0, 10 s]");
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    bl::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return launched("selftest_wait");
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// gemv.cuh -- K7: decode GEMV over 2-bit packed ternary weights.
+//
+// P5 ("1.58-bit量化技术…") §3.1: a ternary weight turns the multiply-accumulate into
+// add (W = +1), subtract (W = -1) or skip (W = 0); §4.1: codes 00 -> 0, 01 -> +1,
+// 10 -> -1, 11 reserved (decodes to 0 here).  Output y = (acc * gamma) / s_b.
+//
+// The weights are streamed from HBM exactly once (N x K/4 bytes, one warp per output row,
+// lanes on consecutive 8-byte chunks so any K % 32 == 0 row is aligned).  No code is ever decoded to a
+// value: for each 32-bit word of 16 codes, the bit-planes lo_j = (w >> 2j) & 0x01010101
+// and hi_j = (w >> 2j+1) & 0x01010101 (j = 0..3) are 0/1 bytes, and
+//   sum_k dec(c_k) x_k = sum_j dp4a(lo_j, x_j) - dp4a(hi_j, x_j),
+// which also maps the reserved 11 to 0.  Byte i of lo_j holds the code of element
+// 16g + 4i + j, so the activation words are staged once per block in shared memory in
+// that interleaved order: x_j = (x[16g+j], x[16g+4+j], x[16g+8+j], x[16g+12+j]).
+#pragma once
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+
+// Shared-memory activation layout: element (b, h, c) = the 4 interleaved words of
+// group g = 2c + h (c = 8-byte chunk index of a packed row, h = word within the chunk),
+// so consecutive lanes read consecutive 16-byte entries (no bank conflicts).
+// sum_i a.u8[i] * b.s8[i] + c
+__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ int gemv_xs_index(int b, int h, int c, int nchunk) {
+    return (b * 2 + h) * nchunk + c;
+}
+
+// NB <= 4: the bit-planes are masked in place (w & (0x01010101 << 2j)), which needs no
+// shifts but leaves plane j scaled by 2^(2j) (lo) or 2^(2j+1) (hi); one accumulator per
+// plane, unscaled exactly at the end.  NB > 4: planes are shifted down first so a batch
+// row needs only two accumulators.
+template <int NB>
+__global__ void __launch_bounds__(kGemvThreads) ternary_gemv_kernel(const uint8_t* __restrict__ packed,
+                                                                    const float* __restrict__ gamma, int N, int K,
+                                                                    const int8_t* __restrict__ xq,
+                                                                    const float* __restrict__ sx, int B,
+                                                                    float* __restrict__ y,
+                                                                    int32_t* __restrict__ acc_out) {
+    extern __shared__ int4 xs[];       // [B][2][K/32]
+    const int G = K / 16;
+    const int nchunk = K / 32;          // 8-byte chunks (32 codes) per packed row
+    for (int idx = threadIdx.x; idx < B * G; idx += kGemvThreads) {
+        const int b = idx / G, g = idx - b * G;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(b) * K) + g);
+        int4 o;
+        int* ov = reinterpret_cast<int*>(&o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t t01 = __byte_perm(raw.x, raw.y, j | ((4 + j) << 4));
+            const uint32_t t23 = __byte_perm(raw.z, raw.w, j | ((4 + j) << 4));
+            ov[j] = static_cast<int>(__byte_perm(t01, t23, 0x5410));
+        }
+        xs[gemv_xs_index(b, g & 1, g >> 1, nchunk)] = o;
+    }
+    __syncthreads();
+
+    const float gm = __ldg(gamma);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr bool kInPlace = NB <= 4;
+    constexpr int kAcc = kInPlace ? 8 : 2;
+    for (int n = blockIdx.x * kGemvWarps + warp; n < N; n += gridDim.x * kGemvWarps) {
+        int acc[NB][kAcc];
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int a = 0; a < kAcc; ++a) acc[b][a] = 0;
+        const uint2* row = reinterpret_cast<const uint2*>(packed + static_cast<int64_t>(n) * (K / 4));
+#pragma unroll 2
+        for (int c = lane; c < nchunk; c += 32) {
+            const uint2 pw = __ldcs(row + c);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t w = h == 0 ? pw.x : pw.y;
+                int lo[4], hi[4];
+                if constexpr (kInPlace) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        lo[j] = static_cast<int>(w & (0x01010101u << (2 * j)));
+                        hi[j] = static_cast<int>(w & (0x02020202u << (2 * j)));
+                    }
+                } else {
+                    const uint32_t w1 = w >> 1;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        lo[j] = static_cast<int>((w >> (2 * j)) & 0x01010101u);
+                        hi[j] = static_cast<int>((w1 >> (2 * j)) & 0x01010101u);
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    if (b < B) {
+                        const int4 xv = xs[gemv_xs_index(b, h, c, nchunk)];
+                        const int xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if constexpr (kInPlace) {
+                                // bytes of lo[j]/hi[j] are 0 or 2^(2j) / 2^(2j+1): read them as
+                                // unsigned (2^7 does not fit a signed byte)
+                                acc[b][2 * j] = dp4a_us(static_cast<uint32_t>(lo[j]), xw[j], acc[b][2 * j]);
+                                acc[b][2 * j + 1] = dp4a_us(static_cast<uint32_t>(hi[j]), xw[j], acc[b][2 * j + 1]);
+                            } else {
+                                acc[b][0] = __dp4a(lo[j], xw[j], acc[b][0]);
+                                acc[b][1] = __dp4a(hi[j], xw[j], acc[b][1]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            if (b < B) {
+                int part;
+                if constexpr (kInPlace) {
+                    part = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) part += (acc[b][2 * j] >> (2 * j)) - (acc[b][2 * j + 1] >> (2 * j + 1));
+                } else {
+                    part = acc[b][0] - acc[b][1];
+                }
+                const int tot = warp_sum(part);
+                if (lane == 0) {
+                    const int64_t o = static_cast<int64_t>(b) * N + n;
+                    y[o] = __fdiv_rn(__fmul_rn(static_cast<float>(tot), gm), __ldg(sx + b));
+                    if (acc_out != nullptr) acc_out[o] = tot;
+                }
+            }
+        }
+    }
+}
+
+// Bounded-wait self test: one thread waits on an mbarrier that nothing arrives on.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, limit_ns, &abort_flag);
+}
+
+}  // namespace bl

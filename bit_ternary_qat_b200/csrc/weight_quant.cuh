@@ -1,0 +1,156 @@
+// weight_quant.cuh -- K2: per-tensor absmean ternary weight quantiser + 2-bit packing.
+//
+// Restates P3 ("BitNet 1.5技术解析…") §2.1 weight_quant and P5 ("1.58-bit量化技术…")
+// §2.2 ternary_quantize:  gamma = max(mean|W|, 1e-5),  W_q = clamp(round(W/gamma), -1, 1),
+// and P5 §4.1 (2-bit codes 00 -> 0, 01 -> +1, 10 -> -1) / §5.1 (64-bit aligned packing).
+//
+// Two launches, both memory-bound:
+//   pass 1  each block sums |W| over a fixed slice in fp64 -> one partial per block;
+//   pass 2  every block re-derives gamma from the partials in a fixed order (so no third
+//           launch and no atomics: the result is bit-identical run to run), then streams W
+//           again (an L2 hit when W fits in L2) and writes int8 codes, bf16 codes and the
+//           packed 2-bit codes in one go.
+//
+// The ternary decision needs no per-element division.  fl32(w / gamma) is monotone in w,
+// so {w > 0 : fl32(w/gamma) > 0.5} = {w >= w*} for one fp32 threshold w*, found by a
+// 31-step bisection over fp32 bit patterns that evaluates the IEEE division itself.
+// Because the division is sign-symmetric, W_q = sign(w) * [|w| >= w*] reproduces
+// clamp(round_half_even(fl32(w/gamma)), -1, 1) exactly for every finite w.
+#pragma once
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kWqThreads = 256;
+constexpr int kWqMaxPartials = 1184;   // 8 blocks per SM on 148 SMs
+
+// Number of pass-1 blocks for n elements: depends on n only, so gamma is the same on
+// every device.
+__host__ __device__ inline int wq_num_partials(int64_t n) {
+    int64_t vecs = n / 4;
+    int64_t p = (vecs + kWqThreads * 16 - 1) / (kWqThreads * 16);
+    if (p < 1) p = 1;
+    if (p > kWqMaxPartials) p = kWqMaxPartials;
+    return static_cast<int>(p);
+}
+
+__global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float* __restrict__ W, int64_t n,
+                                                                     double* __restrict__ partials) {
+    __shared__ double red[kWqThreads / 32];
+    const int64_t nvec = n / 4;
+    const float4* w4 = reinterpret_cast<const float4*>(W);
+    double acc = 0.0;
+    for (int64_t i = blockIdx.x * (int64_t)kWqThreads + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * kWqThreads) {
+        float4 v = __ldg(w4 + i);
+        acc += (double)fabsf(v.x);
+        acc += (double)fabsf(v.y);
+        acc += (double)fabsf(v.z);
+        acc += (double)fabsf(v.w);
+    }
+    acc = warp_sum(acc);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double s = 0.0;
+        for (int w = 0; w < kWqThreads / 32; ++w) s += red[w];
+        partials[blockIdx.x] = s;
+    }
+}
+
+// Smallest positive fp32 w with fl32(w / gamma) > 0.5 (gamma >= 1e-5 > 0).
+__device__ __forceinline__ float ternary_threshold(float gamma) {
+    uint32_t lo = 0u;            // 0 / gamma = 0      -> not above 0.5
+    uint32_t hi = 0x7f7fffffu;   // FLT_MAX / gamma   -> above 0.5
+    while (hi - lo > 1u) {
+        uint32_t mid = lo + ((hi - lo) >> 1);
+        if (__fdiv_rn(__uint_as_float(mid), gamma) > 0.5f) hi = mid; else lo = mid;
+    }
+    return __uint_as_float(hi);
+}
+
+// grid-stride over 16-element groups; n % 32 == 0.
+__global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
+    const float* __restrict__ W, int64_t n, const double* __restrict__ partials, int nparts,
+    int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
+    float* __restrict__ gamma_out) {
+    __shared__ float s_thr;
+    if (threadIdx.x < 32) {
+        // fixed-order sum of the partials: lane-strided, then a fixed butterfly
+        double s = 0.0;
+        for (int i = threadIdx.x; i < nparts; i += 32) s += partials[i];
+        s = warp_sum(s);
+        if (threadIdx.x == 0) {
+            float mean = static_cast<float>(s / static_cast<double>(n));
+            float gamma = fmaxf(mean, 1e-5f);
+            s_thr = ternary_threshold(gamma);
+            if (blockIdx.x == 0) *gamma_out = gamma;
+        }
+    }
+    __syncthreads();
+    const float thr = s_thr;
+    const int64_t ngroups = n / 16;
+    const float4* w4 = reinterpret_cast<const float4*>(W);
+    for (int64_t gi = blockIdx.x * (int64_t)kWqThreads + threadIdx.x; gi < ngroups;
+         gi += (int64_t)gridDim.x * kWqThreads) {
+        float w[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float4 v = __ldg(w4 + gi * 4 + j);
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        }
+        int q[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) q[e] = (w[e] >= thr) ? 1 : ((w[e] <= -thr) ? -1 : 0);
+        if (wq_i8 != nullptr) {
+            uint32_t b[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                b[j] = (uint32_t)(uint8_t)(int8_t)q[4 * j] | ((uint32_t)(uint8_t)(int8_t)q[4 * j + 1] << 8) |
+                       ((uint32_t)(uint8_t)(int8_t)q[4 * j + 2] << 16) | ((uint32_t)(uint8_t)(int8_t)q[4 * j + 3] << 24);
+            reinterpret_cast<uint4*>(wq_i8)[gi] = make_uint4(b[0], b[1], b[2], b[3]);
+        }
+        if (wq_bf16 != nullptr) {
+            // bf16 bits of -1, 0, +1
+            uint32_t h[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t lo = q[2 * j] == 0 ? 0u : (q[2 * j] > 0 ? 0x3F80u : 0xBF80u);
+                uint32_t hi = q[2 * j + 1] == 0 ? 0u : (q[2 * j + 1] > 0 ? 0x3F80u : 0xBF80u);
+                h[j] = lo | (hi << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(wq_bf16) + gi * 2;
+            dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        if (packed != nullptr) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                uint32_t code = q[e] > 0 ? 1u : (q[e] < 0 ? 2u : 0u);
+                word |= code << (2 * e);
+            }
+            reinterpret_cast<uint32_t*>(packed)[gi] = word;
+        }
+    }
+}
+
+// Standalone packing of int8 codes (ternary_pack): one thread per 16 codes.
+__global__ void __launch_bounds__(256) ternary_pack_kernel(const int8_t* __restrict__ wq, int64_t n,
+                                                           uint8_t* __restrict__ packed) {
+    const int64_t ngroups = n / 16;
+    for (int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; gi < ngroups;
+         gi += (int64_t)gridDim.x * blockDim.x) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(wq) + gi);
+        const uint32_t b[4] = {v.x, v.y, v.z, v.w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            int8_t q = static_cast<int8_t>((b[e >> 2] >> (8 * (e & 3))) & 0xFFu);
+            uint32_t code = q == 1 ? 1u : (q == -1 ? 2u : 0u);
+            word |= code << (2 * e);
+        }
+        reinterpret_cast<uint32_t*>(packed)[gi] = word;
+    }
+}
+
+}  // namespace bl

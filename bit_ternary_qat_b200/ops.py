@@ -1,0 +1,257 @@
+"""Tensor-level binding of the C ABI: same names as the C entry points.
+
+Argument marshalling only: check that tensors are contiguous CUDA tensors of the
+expected dtype, allocate outputs that the caller did not pass (torch is used for
+device memory and streams), pass ``data_ptr()`` values and the current CUDA stream
+to libbitlinear.so.  Every step of the computation runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float32: _lib.BL_F32, torch.bfloat16: _lib.BL_BF16}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return _DT[t.dtype]
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def workspace_bytes(T: int, N: int, K: int) -> int:
+    return int(_lib.lib().bitlinear_workspace_bytes(T, N, K))
+
+
+def workspace(T: int, N: int, K: int, device) -> torch.Tensor:
+    return torch.empty(workspace_bytes(T, N, K), dtype=torch.uint8, device=device)
+
+
+def bitlinear_quant_weight(W: torch.Tensor, want_i8: bool = True, want_bf16: bool = True,
+                           want_packed: bool = True, ws: Optional[torch.Tensor] = None, out=None):
+    """Returns dict(gamma [1] f32, wq_i8 [N,K] i8, wq_bf16 [N,K] bf16, packed [N,K/4] u8)."""
+    _cuda(W, "W", torch.float32)
+    N, K = W.shape
+    dev = W.device
+    o = dict(out or {})
+    o.setdefault("gamma", torch.empty(1, dtype=torch.float32, device=dev))
+    if want_i8:
+        o.setdefault("wq_i8", torch.empty(N, K, dtype=torch.int8, device=dev))
+    if want_bf16:
+        o.setdefault("wq_bf16", torch.empty(N, K, dtype=torch.bfloat16, device=dev))
+    if want_packed:
+        o.setdefault("packed", torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    if ws is None:
+        ws = workspace(1, N, K, dev)
+    _lib.call("bitlinear_quant_weight", W.data_ptr(), N, K, _ptr(o.get("wq_i8")), _ptr(o.get("wq_bf16")),
+              _ptr(o.get("packed")), o["gamma"].data_ptr(), ws.data_ptr(), ws.numel(), _stream(dev))
+    return o
+
+
+def bitlinear_act_quant(X: torch.Tensor, apply_rmsnorm: bool = True, g: Optional[torch.Tensor] = None,
+                        eps: float = 1e-6, want_xdq: bool = True, out=None):
+    """Returns dict(xq [T,K] i8, sx [T] f32, rinv [T] f32 or None, xdq [T,K] X.dtype or None)."""
+    _cuda(X, "X")
+    T, K = X.shape
+    dev = X.device
+    if g is not None:
+        _cuda(g, "g", torch.float32)
+    o = dict(out or {})
+    o.setdefault("xq", torch.empty(T, K, dtype=torch.int8, device=dev))
+    o.setdefault("sx", torch.empty(T, dtype=torch.float32, device=dev))
+    if apply_rmsnorm:
+        o.setdefault("rinv", torch.empty(T, dtype=torch.float32, device=dev))
+    if want_xdq:
+        o.setdefault("xdq", torch.empty(T, K, dtype=X.dtype, device=dev))
+    _lib.call("bitlinear_act_quant", X.data_ptr(), _dt(X), T, K, 1 if apply_rmsnorm else 0, _ptr(g), float(eps),
+              o["xq"].data_ptr(), o["sx"].data_ptr(), _ptr(o.get("rinv")), _ptr(o.get("xdq")), _stream(dev))
+    return o
+
+
+def bitlinear_linear(xq: torch.Tensor, sx: torch.Tensor, wq_i8: torch.Tensor, gamma: torch.Tensor,
+                     out_dtype=torch.bfloat16, want_acc: bool = False, y: Optional[torch.Tensor] = None,
+                     acc: Optional[torch.Tensor] = None):
+    _cuda(xq, "xq", torch.int8)
+    _cuda(wq_i8, "wq_i8", torch.int8)
+    T, K = xq.shape
+    N = wq_i8.shape[0]
+    dev = xq.device
+    if y is None:
+        y = torch.empty(T, N, dtype=out_dtype, device=dev)
+    if want_acc and acc is None:
+        acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    _lib.call("bitlinear_linear", xq.data_ptr(), sx.data_ptr(), T, K, wq_i8.data_ptr(), gamma.data_ptr(), N,
+              y.data_ptr(), _dt(y), _ptr(acc), _stream(dev))
+    return y, acc
+
+
+def bitlinear_forward(X: torch.Tensor, wq_i8: torch.Tensor, gamma: torch.Tensor, g: Optional[torch.Tensor] = None,
+                      eps: float = 1e-6, want_acc: bool = False, want_xdq: bool = True, out=None):
+    """Returns dict(y, xq, sx, rinv, xdq, acc)."""
+    _cuda(X, "X")
+    _cuda(wq_i8, "wq_i8", torch.int8)
+    T, K = X.shape
+    N = wq_i8.shape[0]
+    dev = X.device
+    o = dict(out or {})
+    o.setdefault("y", torch.empty(T, N, dtype=X.dtype, device=dev))
+    o.setdefault("xq", torch.empty(T, K, dtype=torch.int8, device=dev))
+    o.setdefault("sx", torch.empty(T, dtype=torch.float32, device=dev))
+    o.setdefault("rinv", torch.empty(T, dtype=torch.float32, device=dev))
+    if want_xdq:
+        o.setdefault("xdq", torch.empty(T, K, dtype=X.dtype, device=dev))
+    if want_acc:
+        o.setdefault("acc", torch.empty(T, N, dtype=torch.int32, device=dev))
+    _lib.call("bitlinear_forward", X.data_ptr(), _dt(X), T, K, _ptr(g), float(eps), wq_i8.data_ptr(),
+              gamma.data_ptr(), N, o["y"].data_ptr(), o["xq"].data_ptr(), o["sx"].data_ptr(), o["rinv"].data_ptr(),
+              _ptr(o.get("xdq")), _ptr(o.get("acc")), _stream(dev))
+    return o
+
+
+def bitlinear_backward_input(dY: torch.Tensor, X: torch.Tensor, rinv: torch.Tensor, wq_bf16: torch.Tensor,
+                             gamma: torch.Tensor, g: Optional[torch.Tensor] = None, want_dg: bool = True,
+                             ws: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,
+                             dg: Optional[torch.Tensor] = None):
+    _cuda(dY, "dY")
+    _cuda(X, "X", dY.dtype)
+    _cuda(wq_bf16, "wq_bf16", torch.bfloat16)
+    T, N = dY.shape
+    K = X.shape[1]
+    dev = dY.device
+    if dX is None:
+        dX = torch.empty(T, K, dtype=torch.float32, device=dev)
+    if want_dg and dg is None:
+        dg = torch.empty(K, dtype=torch.float32, device=dev)
+    if ws is None and dg is not None:
+        ws = workspace(T, N, K, dev)
+    _lib.call("bitlinear_backward_input", dY.data_ptr(), X.data_ptr(), _dt(dY), T, K, N, _ptr(g), rinv.data_ptr(),
+              wq_bf16.data_ptr(), gamma.data_ptr(), dX.data_ptr(), _ptr(dg), _ptr(ws),
+              0 if ws is None else ws.numel(), _stream(dev))
+    return dX, dg
+
+
+def bitlinear_grad_input(dY: torch.Tensor, wq_bf16: torch.Tensor, gamma: torch.Tensor,
+                         dXhat: Optional[torch.Tensor] = None):
+    """dX_hat = gamma * dY . W_q  (fp32 [T, K])."""
+    _cuda(dY, "dY")
+    _cuda(wq_bf16, "wq_bf16", torch.bfloat16)
+    T, N = dY.shape
+    K = wq_bf16.shape[1]
+    if dXhat is None:
+        dXhat = torch.empty(T, K, dtype=torch.float32, device=dY.device)
+    _lib.call("bitlinear_grad_input", dY.data_ptr(), _dt(dY), T, K, N, wq_bf16.data_ptr(), gamma.data_ptr(),
+              dXhat.data_ptr(), _stream(dY.device))
+    return dXhat
+
+
+def bitlinear_rmsnorm_backward(X: torch.Tensor, rinv: torch.Tensor, dX_inout: torch.Tensor,
+                               g: Optional[torch.Tensor] = None, want_dg: bool = True,
+                               ws: Optional[torch.Tensor] = None, dg: Optional[torch.Tensor] = None):
+    """In place: dX_inout holds dX_hat on entry and dX on return."""
+    _cuda(X, "X")
+    _cuda(dX_inout, "dX_inout", torch.float32)
+    T, K = X.shape
+    dev = X.device
+    if want_dg and dg is None:
+        dg = torch.empty(K, dtype=torch.float32, device=dev)
+    if ws is None and dg is not None:
+        ws = workspace(T, 16, K, dev)
+    _lib.call("bitlinear_rmsnorm_backward", X.data_ptr(), _dt(X), T, K, _ptr(g), rinv.data_ptr(),
+              dX_inout.data_ptr(), _ptr(dg), _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
+    return dX_inout, dg
+
+
+def bitlinear_backward_weight(dY: torch.Tensor, xdq: torch.Tensor, dW: Optional[torch.Tensor] = None):
+    _cuda(dY, "dY")
+    _cuda(xdq, "xdq", dY.dtype)
+    T, N = dY.shape
+    K = xdq.shape[1]
+    if dW is None:
+        dW = torch.empty(N, K, dtype=torch.float32, device=dY.device)
+    _lib.call("bitlinear_backward_weight", dY.data_ptr(), xdq.data_ptr(), _dt(dY), T, K, N, dW.data_ptr(),
+              _stream(dY.device))
+    return dW
+
+
+def bitlinear_backward(dY, X, xdq, rinv, wq_bf16, gamma, g=None, want_dg=True, ws=None, dX=None, dW=None, dg=None):
+    _cuda(dY, "dY")
+    T, N = dY.shape
+    K = X.shape[1]
+    dev = dY.device
+    if dX is None:
+        dX = torch.empty(T, K, dtype=torch.float32, device=dev)
+    if dW is None:
+        dW = torch.empty(N, K, dtype=torch.float32, device=dev)
+    if want_dg and dg is None:
+        dg = torch.empty(K, dtype=torch.float32, device=dev)
+    if ws is None and dg is not None:
+        ws = workspace(T, N, K, dev)
+    _lib.call("bitlinear_backward", dY.data_ptr(), X.data_ptr(), xdq.data_ptr(), _dt(dY), T, K, N, _ptr(g),
+              rinv.data_ptr(), wq_bf16.data_ptr(), gamma.data_ptr(), dX.data_ptr(), dW.data_ptr(), _ptr(dg),
+              _ptr(ws), 0 if ws is None else ws.numel(), _stream(dev))
+    return dX, dW, dg
+
+
+def ternary_pack(wq_i8: torch.Tensor, packed: Optional[torch.Tensor] = None):
+    _cuda(wq_i8, "wq_i8", torch.int8)
+    N, K = wq_i8.shape
+    if packed is None:
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=wq_i8.device)
+    _lib.call("ternary_pack", wq_i8.data_ptr(), N, K, packed.data_ptr(), _stream(wq_i8.device))
+    return packed
+
+
+def ternary_gemv(packed: torch.Tensor, gamma: torch.Tensor, K: int, xq: torch.Tensor, sx: torch.Tensor,
+                 want_acc: bool = False, y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None):
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(xq, "xq", torch.int8)
+    N = packed.shape[0]
+    B = xq.shape[0]
+    dev = packed.device
+    if y is None:
+        y = torch.empty(B, N, dtype=torch.float32, device=dev)
+    if want_acc and acc is None:
+        acc = torch.empty(B, N, dtype=torch.int32, device=dev)
+    _lib.call("ternary_gemv", packed.data_ptr(), gamma.data_ptr(), N, K, xq.data_ptr(), sx.data_ptr(), B,
+              y.data_ptr(), _ptr(acc), _stream(dev))
+    return y, acc
+
+
+def check_device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return int(_lib.lib().bl_check_device_status(_stream(dev)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _lib.lib().bl_set_wait_limit_ns(int(ns))
+
+
+def launch_count() -> int:
+    return int(_lib.lib().bl_launch_count())
+
+
+def selftest_bounded_wait(limit_ns: int, device=None) -> None:
+    dev = device if device is not None else torch.cuda.current_device()
+    _lib.call("bl_selftest_bounded_wait", int(limit_ns), _stream(dev))

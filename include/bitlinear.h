@@ -1,0 +1,215 @@
+/*
+ * bitlinear.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear hot path.
+ *
+ * Source pages (titles), cited per entry point below:
+ *   P2 = "BitNet 三元权重量化训练工程：直通估计器与梯度裁剪实践" (blog.hotdry.top)
+ *   P3 = "BitNet 1.5技术解析：2比特量化在神经网络中的应用与挑战" (intelliparadigm.com)
+ *   P4 = "BitNet b1.58：三元权重下的STE设计与优化" (zyxy.net)
+ *   P5 = "1.58-bit量化技术突破AI算力与内存墙限制" (intelliparadigm.com)
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * Shapes follow nn.Linear (P3 §3.1): the latent weight W is [N x K] row-major
+ * (N = d_out, K = d_in), activations X are [T x K] row-major (T tokens), the output
+ * Y is [T x N].  All matrices are dense row-major with no padding.
+ *
+ * Memory and ownership: every pointer is DEVICE memory owned by the caller and must
+ * stay valid until the work queued on `stream` has finished.  The library allocates
+ * no device or host memory.  Entry points that need scratch take a caller workspace
+ * (`ws`, `ws_bytes`); `bitlinear_workspace_bytes()` gives a size that suffices.
+ * gamma, s_x and r live on the device so a training step never syncs to the host.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * Every entry point is asynchronous on that stream.
+ *
+ * Sizes and alignment (validated on the host before anything is launched):
+ *   - T >= 1, N >= 1, K >= 1; K % 32 == 0 (whole 64-bit words of 2-bit codes per row,
+ *     P5 §5.1); N % 16 == 0 (16-byte aligned rows of Y and dY for TMA and vector
+ *     stores); every pointer 16-byte aligned; T, N, K < 2^31.
+ * Numerics: fp32 quantiser arithmetic with round-half-to-even (torch.round in the
+ * pages' snippets), fp64 reductions, exact int32 accumulation for the int8 x ternary
+ * contraction.  Inputs must be finite.
+ *
+ * Errors: every entry point returns a bl_status.  A non-OK status from validation
+ * means nothing was launched.  BL_ERR_CUDA reports a launch error (the message,
+ * retrievable with bl_last_error(), names the CUDA error).  Kernels never trap:
+ * every wait inside a kernel is bounded, and a wait that runs out records
+ * BL_ERR_TIMEOUT in a device status word that bl_check_device_status() reads.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BL_API __attribute__((visibility("default")))
+#else
+#define BL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_INVALID_ARG = 1,        /* null required pointer, non-positive size, bad dtype */
+    BL_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 32, N % 16, or a size beyond the limits above  */
+    BL_ERR_MISALIGNED = 3,         /* a pointer not 16-byte aligned                       */
+    BL_ERR_WORKSPACE = 4,          /* ws too small (or NULL with ws_bytes needed)          */
+    BL_ERR_CUDA = 5,               /* CUDA runtime / driver error                          */
+    BL_ERR_TIMEOUT = 6,            /* a bounded device wait expired                        */
+    BL_ERR_DEVICE = 7              /* the current device is not an sm_100 (B200) GPU        */
+} bl_status;
+
+typedef enum { BL_F32 = 0, BL_BF16 = 1 } bl_dtype;
+
+/* ABI version of this header (bumped on any signature change). */
+#define BITLINEAR_ABI_VERSION 1
+BL_API int bl_abi_version(void);
+
+/* Message of the last non-OK status returned on this host thread (never NULL). */
+BL_API const char* bl_last_error(void);
+
+/* Bytes of workspace that suffice for every entry point on a layer of this size. */
+BL_API size_t bitlinear_workspace_bytes(int64_t T, int64_t N, int64_t K);
+
+/* Synchronises `stream`, then reads and clears the device status word written by
+ * bounded waits on the current device.  Returns BL_OK, BL_ERR_TIMEOUT or BL_ERR_CUDA. */
+BL_API bl_status bl_check_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, of any single wait inside a kernel launched after this
+ * call (default 2e9).  0 restores the default. */
+BL_API void bl_set_wait_limit_ns(uint64_t ns);
+
+/* Number of kernels this library has launched in this process (all devices). */
+BL_API uint64_t bl_launch_count(void);
+
+/* ------------------------------------------------------------------------------
+ * Weight quantiser: per-tensor absmean ternary (P3 §2.1 weight_quant; P5 §2.2
+ * ternary_quantize; P2 "直通估计器在三元权重量化中的作用").
+ *   gamma = max( mean_{n,k} |W[n,k]|, 1e-5 )        (mean accumulated in fp64)
+ *   W_q   = clamp( round( W / gamma ), -1, 1 )        (fp32 division, half-to-even)
+ * Outputs (each optional, may be NULL):
+ *   Wq_i8    int8  [N x K]   codes -1/0/+1 (operand of the forward GEMM)
+ *   Wq_bf16  bf16  [N x K]   the same codes as bf16 bits (operand of the backward)
+ *   Wpacked  uint8 [N x K/4] 2-bit codes 00->0, 01->+1, 10->-1 (P5 §4.1); element k
+ *            of row n at byte n*K/4 + k/4, bits 2*(k%4)+{0,1}
+ *   gamma    fp32  [1]       required
+ * W: fp32 [N x K].  ws: at least bitlinear_workspace_bytes(1, N, K) bytes.
+ * Deterministic: the same W gives bit-identical outputs on every call. */
+BL_API bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K,
+                                 int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                 float* gamma, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Activation quantiser with optional RMSNorm in front (P3 §3.1 RMSNorm before
+ * activation_quant; P3 §2.2 activation_quant; P2 per-token absmax 8-bit).
+ *   r_t   = 1 / sqrt( mean_k X[t,k]^2 + eps )        (fp64 sum; only if apply_rmsnorm)
+ *   x_hat = X * r_t * g_k                            (x_hat = X if !apply_rmsnorm)
+ *   s_t   = 127 / max( max_k |x_hat[t,k]|, 1e-5 )
+ *   X_q   = clamp( round( x_hat * s_t ), -128, 127 )
+ *   X_dq  = X_q / s_t   (rounded to x_dt; the value the straight-through estimator
+ *                        forwards, saved for the weight gradient)
+ * X: [T x K] of x_dt.  g: fp32 [K] or NULL (gain 1).  Outputs: Xq int8 [T x K],
+ * sx fp32 [T] (required); rinv fp32 [T] (required iff apply_rmsnorm); Xdq [T x K]
+ * of x_dt (optional). */
+BL_API bl_status bitlinear_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K,
+                              int apply_rmsnorm, const float* g, float eps,
+                              int8_t* Xq, float* sx, float* rinv, void* Xdq, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * The int8 x ternary contraction with its rescale (P3 §3.1 F.linear(x_quant, w_quant)
+ * * scale; P5 §3.1 add / subtract / skip):
+ *   acc[t,n] = sum_k X_q[t,k] * W_q[n,k]          exact int32 (tcgen05 kind::i8)
+ *   Y[t,n]   = (acc[t,n] * gamma) / s_t            fp32, then rounded to y_dt
+ * Xq int8 [T x K], sx fp32 [T], Wq_i8 int8 [N x K], gamma fp32 [1] (device).
+ * Y [T x N] of y_dt.  acc int32 [T x N] optional (debug / parity). */
+BL_API bl_status bitlinear_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
+                           const int8_t* Wq_i8, const float* gamma, int64_t N,
+                           void* Y, bl_dtype y_dt, int32_t* acc, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * BitLinear forward (P3 §3.1): bitlinear_act_quant(apply_rmsnorm = 1) followed by
+ * bitlinear_linear with y_dt = x_dt.  Saves Xq, sx, rinv (required) and Xdq
+ * (optional, needed by bitlinear_backward_weight) for the backward. */
+BL_API bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int64_t K,
+                            const float* g, float eps,
+                            const int8_t* Wq_i8, const float* gamma, int64_t N,
+                            void* Y, int8_t* Xq, float* sx, float* rinv, void* Xdq,
+                            int32_t* acc, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Straight-through backward, input side (P3 §3.2; P5 §3.2 TernarySTE returns
+ * grad_output unchanged; P4 §3.2 grad_w = grad_output), then the RMSNorm backward:
+ *   dX_hat[t,k] = gamma * sum_n dY[t,n] * W_q[n,k]            (fp32 accumulation)
+ *   u = X * r,  h = g * dX_hat,  c_t = (1/K) sum_k h u
+ *   dX[t,k]     = r_t * ( h - u * c_t )
+ *   dg[k]       = sum_t dX_hat[t,k] * u[t,k]                  (optional)
+ * dY [T x N] and X [T x K] of dt; g fp32 [K] or NULL; rinv fp32 [T] from the forward;
+ * Wq_bf16 bf16 [N x K] codes; gamma fp32 [1].  dX fp32 [T x K] (gradients in fp32,
+ * P2 "bf16 for forward, fp32 for gradients"); dg fp32 [K] or NULL.
+ * ws: at least bitlinear_workspace_bytes(T, N, K) bytes when dg != NULL. */
+BL_API bl_status bitlinear_backward_input(const void* dY, const void* X, bl_dtype dt,
+                                   int64_t T, int64_t K, int64_t N,
+                                   const float* g, const float* rinv,
+                                   const uint16_t* Wq_bf16, const float* gamma,
+                                   float* dX, float* dg, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* The two halves of bitlinear_backward_input, callable on their own:
+ *   bitlinear_grad_input:       dX_hat = gamma * dY . W_q   -> fp32 [T x K]
+ *   bitlinear_rmsnorm_backward: dX = RMSNorm backward of dX_hat, computed IN PLACE over
+ *                               the fp32 buffer that holds dX_hat; dg optional. */
+BL_API bl_status bitlinear_grad_input(const void* dY, bl_dtype dt, int64_t T, int64_t K, int64_t N,
+                               const uint16_t* Wq_bf16, const float* gamma, float* dXhat,
+                               void* stream);
+BL_API bl_status bitlinear_rmsnorm_backward(const void* X, bl_dtype dt, int64_t T, int64_t K,
+                                     const float* g, const float* rinv, float* dX_inout,
+                                     float* dg, void* ws, size_t ws_bytes, void* stream);
+
+/* Straight-through backward, weight side (P3 §3.2: the gradient reaches the fp32
+ * latent weight):  dW[n,k] = sum_t dY[t,n] * X_dq[t,k]   (fp32 accumulation).
+ * dY [T x N] and Xdq [T x K] of dt; dW fp32 [N x K]. */
+BL_API bl_status bitlinear_backward_weight(const void* dY, const void* Xdq, bl_dtype dt,
+                                    int64_t T, int64_t K, int64_t N, float* dW,
+                                    void* stream);
+
+/* Both halves of the backward on one stream. */
+BL_API bl_status bitlinear_backward(const void* dY, const void* X, const void* Xdq, bl_dtype dt,
+                             int64_t T, int64_t K, int64_t N,
+                             const float* g, const float* rinv,
+                             const uint16_t* Wq_bf16, const float* gamma,
+                             float* dX, float* dW, float* dg,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * 2-bit packing of ternary codes (P5 §4.1; P5 §5.1 64-bit boundaries): Wq_i8 int8
+ * [N x K] with values in {-1,0,1} -> Wpacked uint8 [N x K/4], layout as in
+ * bitlinear_quant_weight.  Values outside {-1,0,1} are packed as 0. */
+BL_API bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t* Wpacked,
+                       void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Decode GEMV over packed ternary weights (P5 §3.1 W=+1 -> y += x, W=-1 -> y -= x,
+ * W=0 -> skip; P5 §4.1 codes, reserved 11 decodes to 0):
+ *   acc[b,n] = sum_k decode(Wpacked[n,k]) * xq[b,k]   exact int32
+ *   y[b,n]   = (acc[b,n] * gamma) / sx[b]              fp32
+ * Wpacked uint8 [N x K/4]; gamma fp32 [1]; xq int8 [B x K]; sx fp32 [B];
+ * y fp32 [B x N]; acc int32 [B x N] optional.  1 <= B <= 16, K <= 65536. */
+BL_API bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K,
+                       const int8_t* xq, const float* sx, int64_t B,
+                       float* y, int32_t* acc, void* stream);
+
+/* ------------------------------------------------------------------------------
+ * Self-test of the bounded-wait machinery: launches one block that waits on an
+ * mbarrier nothing arrives on, with the given limit (ns), and returns.  Afterwards
+ * bl_check_device_status() must report BL_ERR_TIMEOUT.  No counterpart on the pages. */
+BL_API bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

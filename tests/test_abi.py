@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library builds for sm_100a, exports every symbol
+include/bitlinear.h declares, and rejects invalid calls on the host before launching
+anything (so these calls never reach the device)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from bit_ternary_qat_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitlinear.h")
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^BL_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def test_header_declares_expected_entry_points():
+    syms = header_symbols()
+    for name in ["bitlinear_quant_weight", "bitlinear_forward", "bitlinear_backward", "ternary_pack",
+                 "ternary_gemv", "bitlinear_act_quant", "bitlinear_linear", "bitlinear_backward_input",
+                 "bitlinear_backward_weight", "bl_last_error", "bitlinear_workspace_bytes"]:
+        assert name in syms, name
+
+
+def test_library_exports_every_header_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    missing = [s for s in header_symbols() if s not in exported]
+    assert not missing, missing
+    # the binding knows every symbol too
+    assert set(header_symbols()) == set(_lib.SIGNATURES)
+    # and nothing else of ours leaks out of the library (hidden visibility)
+    ours = {s for s in exported if s.startswith(("bl_", "bitlinear_", "ternary_"))}
+    assert ours == set(header_symbols())
+
+
+def test_abi_version_and_workspace(L):
+    assert L.bl_abi_version() == 1
+    assert L.bitlinear_workspace_bytes(4096, 2048, 2048) >= 296 * 2048 * 4
+    assert L.bitlinear_workspace_bytes(1, 16, 32) % 256 == 0
+
+
+FAKE = 1 << 20          # a 16-byte aligned fake device address: never dereferenced on the host
+ODD = FAKE + 4          # misaligned
+
+
+@pytest.mark.parametrize("args,expected", [
+    # (W, N, K, Wq_i8, Wq_bf16, packed, gamma, ws, ws_bytes, stream)
+    ((None, 16, 32, None, None, None, FAKE, FAKE, 1 << 20, None), 1),          # null W
+    ((FAKE, 16, 32, None, None, None, None, FAKE, 1 << 20, None), 1),          # null gamma
+    ((FAKE, 16, 48, None, None, None, FAKE, FAKE, 1 << 20, None), 2),          # K % 32
+    ((FAKE, 24, 32, None, None, None, FAKE, FAKE, 1 << 20, None), 2),          # N % 16
+    ((FAKE, 0, 32, None, None, None, FAKE, FAKE, 1 << 20, None), 1),           # N = 0
+    ((ODD, 16, 32, None, None, None, FAKE, FAKE, 1 << 20, None), 3),           # misaligned
+    ((FAKE, 16, 32, None, None, None, FAKE, FAKE, 8, None), 4),                # workspace too small
+])
+def test_quant_weight_validation(L, args, expected):
+    assert _lib.status("bitlinear_quant_weight", *args) == expected
+    assert len(_lib.last_error()) > 0
+
+
+def test_forward_validation(L):
+    ok = dict(X=FAKE, dt=1, T=8, K=64, g=None, eps=1e-6, wq=FAKE, gamma=FAKE, N=32, Y=FAKE, xq=FAKE, sx=FAKE,
+              rinv=FAKE, xdq=None, acc=None, st=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return _lib.status("bitlinear_forward", *a.values())
+    assert call(dt=7) == 1
+    assert call(X=None) == 1
+    assert call(rinv=None) == 1
+    assert call(T=0) == 1
+    assert call(K=40) == 2
+    assert call(N=8) == 2
+    assert call(Y=ODD) == 3
+    assert call(eps=-1.0) == 1
+
+
+def test_backward_and_gemv_validation(L):
+    # bitlinear_backward_input with dg requested but no workspace
+    st = _lib.status("bitlinear_backward_input", FAKE, FAKE, 1, 8, 64, 32, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                     None, 0, None)
+    assert st == 1
+    st = _lib.status("bitlinear_backward_input", FAKE, FAKE, 1, 8, 64, 32, None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                     FAKE, 16, None)
+    assert st == 4
+    # GEMV batch limits
+    assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 64, FAKE, FAKE, 0, FAKE, None, None) == 2
+    assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 64, FAKE, FAKE, 17, FAKE, None, None) == 2
+    assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 1 << 17, FAKE, FAKE, 1, FAKE, None, None) == 2
+    assert _lib.status("ternary_pack", FAKE, 16, 33, FAKE, None) == 2
+    assert _lib.status("bl_selftest_bounded_wait", 0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "lib_path", lambda: str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.lib()
