@@ -216,7 +216,7 @@ def main():
     import torch
     import torch.distributed as dist
     import bit_ternary_qat_b200 as bl
-    from bit_ternary_qat_b200 import build as blbuild, synth
+    from bit_ternary_qat_b200 import build as blbuild, dp, synth
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -271,8 +271,7 @@ def main():
         rec(5)
         bl.bitlinear_backward_weight(dYi, b["xdq"], dW=b["dW"])
         rec(6)
-        if world > 1:
-            dist.all_reduce(b["dW"])
+        dp.allreduce_weight_grad(b["dW"])
         rec(7)
         bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B], y=b["ydec"])
         rec(8)
