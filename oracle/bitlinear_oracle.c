@@ -204,17 +204,20 @@ void ora_int_gemm(const int8_t* xq, const int8_t* wq, int64_t T, int64_t N, int6
     }
 }
 
-/* Output rescale (P3 §3.1 output * scale with the dequantised operands; the forward
- * equals (x_q/s_t) . (W_q*gamma) = acc * gamma / s_t):
- *   y[t, n] = fl32( fl32((float)acc * gamma) / s_t ).  s_rows[r] is s of output row r. */
+/* Output rescale (P3 §3.1: the linear of the dequantised operands times the weight scale;
+ * with X_dq = x_q / s_t and W_dq = W_q * gamma the forward is acc * (gamma / s_t), i.e. the
+ * integer contraction rescaled by one factor per token):
+ *   c_t     = fl32( gamma / s_t )
+ *   y[t, n] = fl32( (float)acc[t, n] * c_t ).      s_rows[r] is s of output row r. */
 void ora_linear_epilogue(const int32_t* acc, int64_t R, int64_t N, float gamma,
                          const float* s_rows, float* y) {
-    for (int64_t r = 0; r < R; ++r)
+    for (int64_t r = 0; r < R; ++r) {
+        float c = gamma / s_rows[r];
         for (int64_t n = 0; n < N; ++n) {
             float a = (float)acc[r * N + n];
-            float p = a * gamma;
-            y[r * N + n] = p / s_rows[r];
+            y[r * N + n] = a * c;
         }
+    }
 }
 
 /* ---------------------------------------------------------------------------------
@@ -318,7 +321,7 @@ void ora_rmsnorm_backward(const float* X, const float* rinv, const float* g, con
  * Decode GEMV over the 2-bit packed weights (P5 §3.1 add / subtract / skip; P5 §4.1
  * codes).  For each of B activation rows:
  *   acc[b, n] = sum_k decode(packed[n, k]) * x_q[b, k]      exact int32
- *   y[b, n]   = fl32( fl32((float)acc * gamma) / s_b )
+ *   y[b, n]   = fl32( (float)acc * fl32(gamma / s_b) )
  * The loop literally adds, subtracts or skips, as the page describes.
  * --------------------------------------------------------------------------------- */
 void ora_gemv(const uint8_t* packed, float gamma, int64_t N, int64_t K, const int8_t* xq,
@@ -335,8 +338,8 @@ void ora_gemv(const uint8_t* packed, float gamma, int64_t N, int64_t K, const in
                 else if (w == -1) a -= xq[b * K + k];
             }
             acc[b * N + n] = a;
-            float p = (float)a * gamma;
-            y[b * N + n] = p / s[b];
+            float c = gamma / s[b];
+            y[b * N + n] = (float)a * c;
         }
     }
 }
