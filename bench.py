@@ -288,34 +288,92 @@ def main():
     sync_all()
     assert bl.check_device_status() == 0
 
+    # ---------------------------------------------------------------- CUDA graph of one step
+    # The step is 9 library calls; replaying it as a captured graph removes the Python /
+    # ctypes launch overhead from the device timeline.  Events recorded inside the capture
+    # (external event nodes) time every piece of every replay.
+    launches_before_capture = bl.launch_count()
+    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(9)]
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    sync_all()
+    launches_before_capture = bl.launch_count()
+    graphs = []
+    if world == 1:
+        g_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_all):
+            step(gev)
+        graphs.append(g_all)
+
+        def replay():
+            g_all.replay()
+    else:
+        # the NCCL all-reduce stays outside the graphs
+        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1):
+            b = bufs
+            gev[0].record()
+            bl.bitlinear_quant_weight(W, ws=b["ws"], out=b); gev[1].record()
+            bl.bitlinear_act_quant(X, apply_rmsnorm=True, out=b); gev[2].record()
+            bl.bitlinear_linear(b["xq"], b["sx"], b["wq_i8"], b["gamma"], y=b["y"]); gev[3].record()
+            bl.bitlinear_grad_input(dY, b["wq_bf16"], b["gamma"], dXhat=b["dX"]); gev[4].record()
+            bl.bitlinear_rmsnorm_backward(X, b["rinv"], b["dX"], ws=b["ws"], dg=b["dg"]); gev[5].record()
+            bl.bitlinear_backward_weight(dY, b["xdq"], dW=b["dW"]); gev[6].record()
+        with torch.cuda.graph(g2):
+            gev[7].record()
+            bl.ternary_gemv(bufs["packed"], bufs["gamma"], D_IN, bufs["xq"][:DECODE_B], bufs["sx"][:DECODE_B],
+                            y=bufs["ydec"])
+            gev[8].record()
+        graphs += [g1, g2]
+
+        def replay():
+            g1.replay()
+            dp.allreduce_weight_grad(bufs["dW"])
+            g2.replay()
+    kernels_per_step = bl.launch_count() - launches_before_capture
+    for _ in range(max(3, args.warmup)):
+        replay()
+    sync_all()
+    assert bl.check_device_status() == 0
+
     # ---------------------------------------------------------------- timed region
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(K)]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     gpu_uuid = None
     try:
         gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         gpu_uuid = str(local)
     clk = ClockSampler(gpu_uuid) if rank == 0 else None
-    launches0 = bl.launch_count()
+    pieces = {p: [] for p in PIECES}
     sync_all()
     if clk:
         clk.start()
         time.sleep(0.3)
     for i in range(K):
         flush.zero_()                       # evict L2 (outside the timed events)
-        step(evs[i])
+        ev_s[i].record()
+        replay()
+        ev_e[i].record()
+        torch.cuda.synchronize()            # read this replay's piece times
+        for j, p in enumerate(PIECES):
+            pieces[p].append(gev[j].elapsed_time(gev[j + 1]))
     sync_all()
     clocks = clk.stop() if clk else None
-    launches = bl.launch_count() - launches0
-    per_step = [e[0].elapsed_time(e[8]) for e in evs]
-    piece_ms = {p: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, p in enumerate(PIECES)}
+    launches = kernels_per_step * K
+    per_step = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
+    piece_ms = {p: statistics.mean(v) for p, v in pieces.items()}
     tot_ms = sum(per_step)
     t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     tot_ms = float(t.item())
     assert bl.check_device_status() == 0
+    del graphs
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -392,6 +450,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": int(launches),
+        "timing": "each step replays a CUDA graph of the step's library calls; gpu_launches = kernels per step x steps",
         "clocks": clocks,
         "pieces_ms": {k: round(v, 5) for k, v in piece_ms.items()},
         "gemm_tflops": {p: gemm_flops / (piece_ms[p] * 1e-3) / 1e12 for p in gemm_pieces},

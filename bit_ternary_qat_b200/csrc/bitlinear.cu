@@ -137,18 +137,22 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D row-major tensor [outer x inner] with 128-byte swizzled boxes [box_outer x box_inner].
-bl_status make_tmap(CUtensorMap* tm, const void* base, bool bf16, uint64_t inner, uint64_t outer,
+enum TmType { kTmU8 = 0, kTmBf16 = 1, kTmF32 = 2 };
+
+// 2-D row-major tensor [outer x inner] with 128-byte swizzled boxes [box_outer x box_inner]
+// (box_inner * element size == 128 bytes).
+bl_status make_tmap(CUtensorMap* tm, const void* base, TmType t, uint64_t inner, uint64_t outer,
                     uint32_t box_inner, uint32_t box_outer) {
     EncodeTiledFn fn = encode_fn();
     BL_REQUIRE(fn != nullptr, BL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    const uint64_t esize = bf16 ? 2 : 1;
+    const uint64_t esize = t == kTmU8 ? 1 : (t == kTmBf16 ? 2 : 4);
+    const CUtensorMapDataType dt = t == kTmU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : (t == kTmBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {inner * esize};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     BL_REQUIRE(r == CUDA_SUCCESS, BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return BL_OK;
@@ -160,13 +164,19 @@ bl_status make_tmap(CUtensorMap* tm, const void* base, bool bf16, uint64_t inner
 constexpr int kBN = 256;
 
 template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
-bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, bl::TcGemmArgs a, cudaStream_t st,
-                    const DeviceInfo& dev) {
+bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, bl::TcGemmArgs a,
+                    cudaStream_t st, const DeviceInfo& dev) {
     auto kern = bl::tc_gemm_kernel<kInt8, kAMN, kBMN, kBN, kEpi>;
     const size_t smem = bl::tc_smem_bytes<kBN>();
     BL_REQUIRE((int)smem <= dev.max_smem_optin, BL_ERR_DEVICE, "GEMM needs %zu bytes of shared memory", smem);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    static std::atomic<uint64_t> attr_set{0};   // bit d: attribute set on device d
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (!(attr_set.load() & (1ull << dev_id))) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_set.fetch_or(1ull << dev_id);
+    }
     a.m_tiles = (a.M + bl::kTcBM - 1) / bl::kTcBM;
     a.n_tiles = (a.N + kBN - 1) / kBN;
     const int kb_elems = kInt8 ? 128 : 64;
@@ -174,46 +184,71 @@ bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, bl::TcGemmArgs
     a.wait_ns = g_wait_ns.load();
     const int tiles = a.m_tiles * a.n_tiles;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    kern<<<grid, bl::kTcThreads, smem, st>>>(ta, tb, a);
+    kern<<<grid, bl::kTcThreads, smem, st>>>(ta, tb, td, a);
     return launched("tc_gemm");
 }
 
 // ------------------------------------------------------------------------------------
 // pieces shared by the entry points (validation already done by the caller)
 // ------------------------------------------------------------------------------------
+template <bool kBf16, int VPT>
+void launch_act_quant_v(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
+                        float* sx, float* rinv, void* Xdq, cudaStream_t st) {
+    constexpr int NT = bl::act_threads<kBf16>();
+    bl::act_quant_kernel<kBf16, NT, VPT><<<(unsigned)T, NT, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx, rinv,
+                                                                     Xdq);
+}
+
+template <bool kBf16>
+void launch_act_quant(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
+                      float* sx, float* rinv, void* Xdq, cudaStream_t st) {
+    constexpr int NT = bl::act_threads<kBf16>();
+    const int64_t nvec = K / (kBf16 ? 8 : 4);
+    const int64_t vpt = (nvec + NT - 1) / NT;
+    if (vpt <= 1) launch_act_quant_v<kBf16, 1>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    else if (vpt <= 2) launch_act_quant_v<kBf16, 2>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    else if (vpt <= 4) launch_act_quant_v<kBf16, 4>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    else if (vpt <= 8) launch_act_quant_v<kBf16, 8>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    else if (vpt <= 12) launch_act_quant_v<kBf16, 12>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    else launch_act_quant_v<kBf16, 16>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+}
+
 bl_status run_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int apply_norm, const float* g,
                         float eps, int8_t* Xq, float* sx, float* rinv, void* Xdq, cudaStream_t st) {
     if (x_dt == BL_BF16)
-        bl::act_quant_kernel<true><<<(unsigned)T, bl::kActThreads, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx,
-                                                                            rinv, Xdq);
+        launch_act_quant<true>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     else
-        bl::act_quant_kernel<false><<<(unsigned)T, bl::kActThreads, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx,
-                                                                             rinv, Xdq);
+        launch_act_quant<false>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     return launched("act_quant");
 }
 
 bl_status run_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq, const float* gamma,
                      int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
-    CUtensorMap ta, tb;
-    BL_TRY(make_tmap(&ta, Xq, false, (uint64_t)K, (uint64_t)T, 128, 128));
-    BL_TRY(make_tmap(&tb, Wq, false, (uint64_t)K, (uint64_t)N, 128, kBN));
+    CUtensorMap ta, tb, td;
+    BL_TRY(make_tmap(&ta, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, 128));
+    BL_TRY(make_tmap(&tb, Wq, kTmU8, (uint64_t)K, (uint64_t)N, 128, kBN));
     bl::TcGemmArgs a{};
     a.M = (int)T; a.N = (int)N; a.K = (int)K;
-    a.out = Y; a.ldo = N; a.out_bf16 = y_dt == BL_BF16 ? 1 : 0;
     a.acc_out = acc; a.row_scale = sx; a.gamma = gamma;
-    return launch_tc<true, false, false, bl::kEpiLinear>(ta, tb, a, st, dev);
+    if (y_dt == BL_BF16) {
+        BL_TRY(make_tmap(&td, Y, kTmBf16, (uint64_t)N, (uint64_t)T, 64, 32));
+        return launch_tc<true, false, false, bl::kEpiLinearBf16>(ta, tb, td, a, st, dev);
+    }
+    BL_TRY(make_tmap(&td, Y, kTmF32, (uint64_t)N, (uint64_t)T, 32, 32));
+    return launch_tc<true, false, false, bl::kEpiLinearF32>(ta, tb, td, a, st, dev);
 }
 
 bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf16, const float* gamma, int64_t T,
                               int64_t K, int64_t N, float* dXhat, cudaStream_t st, const DeviceInfo& dev) {
     if (dt == BL_BF16) {
-        CUtensorMap ta, tb;
-        BL_TRY(make_tmap(&ta, dY, true, (uint64_t)N, (uint64_t)T, 64, 128));      // dY, K-major (contraction N)
-        BL_TRY(make_tmap(&tb, Wq_bf16, true, (uint64_t)K, (uint64_t)N, 64, 64));  // W_q, MN-major (rows = N)
+        CUtensorMap ta, tb, td;
+        BL_TRY(make_tmap(&ta, dY, kTmBf16, (uint64_t)N, (uint64_t)T, 64, 128));      // dY, K-major (contraction N)
+        BL_TRY(make_tmap(&tb, Wq_bf16, kTmBf16, (uint64_t)K, (uint64_t)N, 64, 64));  // W_q, MN-major (rows = N)
+        BL_TRY(make_tmap(&td, dXhat, kTmF32, (uint64_t)K, (uint64_t)T, 32, 32));
         bl::TcGemmArgs a{};
         a.M = (int)T; a.N = (int)K; a.K = (int)N;
-        a.out = dXhat; a.ldo = K; a.gamma = gamma;
-        return launch_tc<false, false, true, bl::kEpiScaleF32>(ta, tb, a, st, dev);
+        a.gamma = gamma;
+        return launch_tc<false, false, true, bl::kEpiScaleF32>(ta, tb, td, a, st, dev);
     }
     // fp32 layer: CUDA-core fp32 contraction, C[t,k] = gamma * sum_n dY[t,n] W_q[n,k]
     dim3 grid((unsigned)((K + 63) / 64), (unsigned)((T + 63) / 64));
@@ -226,13 +261,13 @@ bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf
 bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int64_t T, int64_t K, int64_t N,
                                float* dW, cudaStream_t st, const DeviceInfo& dev) {
     if (dt == BL_BF16) {
-        CUtensorMap ta, tb;
-        BL_TRY(make_tmap(&ta, dY, true, (uint64_t)N, (uint64_t)T, 64, 64));    // dY^T: MN-major (n contiguous)
-        BL_TRY(make_tmap(&tb, Xdq, true, (uint64_t)K, (uint64_t)T, 64, 64));   // X_dq: MN-major (k contiguous)
+        CUtensorMap ta, tb, td;
+        BL_TRY(make_tmap(&ta, dY, kTmBf16, (uint64_t)N, (uint64_t)T, 64, 64));    // dY^T: MN-major (n contiguous)
+        BL_TRY(make_tmap(&tb, Xdq, kTmBf16, (uint64_t)K, (uint64_t)T, 64, 64));   // X_dq: MN-major (k contiguous)
+        BL_TRY(make_tmap(&td, dW, kTmF32, (uint64_t)K, (uint64_t)N, 32, 32));
         bl::TcGemmArgs a{};
         a.M = (int)N; a.N = (int)K; a.K = (int)T;
-        a.out = dW; a.ldo = K;
-        return launch_tc<false, true, true, bl::kEpiF32>(ta, tb, a, st, dev);
+        return launch_tc<false, true, true, bl::kEpiF32>(ta, tb, td, a, st, dev);
     }
     dim3 grid((unsigned)((K + 63) / 64), (unsigned)((N + 63) / 64));
     bl::simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>((int)N, (int)K, (int)T, static_cast<const float*>(dY),
@@ -242,32 +277,48 @@ bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int
 }
 
 size_t quant_ws_bytes() { return sizeof(double) * bl::kWqMaxPartials; }
-size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdBlocks * (size_t)K; }
+size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
+
+template <bool kBf16X, int VPT>
+int launch_rmsnorm_bwd_v(const void* X, const float* rinv, const float* g, float* dX, int64_t T, int64_t K,
+                         float* partial, int sms, cudaStream_t st) {
+    constexpr int R = VPT == 1 ? 4 : (VPT == 2 ? 2 : 1);
+    int64_t grid = (T + R - 1) / R;
+    const int64_t cap = sms * 4 < bl::kBwdMaxBlocks ? sms * 4 : bl::kBwdMaxBlocks;
+    if (grid > cap) grid = cap;
+    bl::rmsnorm_bwd_kernel<kBf16X, VPT, R><<<(unsigned)grid, bl::kBwdThreads, 0, st>>>(X, rinv, g, dX, (int)T, (int)K,
+                                                                                       partial);
+    return (int)grid;
+}
+
+template <bool kBf16X>
+int launch_rmsnorm_bwd(const void* X, const float* rinv, const float* g, float* dX, int64_t T, int64_t K,
+                       float* partial, int sms, cudaStream_t st) {
+    const int64_t nvec = K / 4;
+    const int64_t vpt = (nvec + bl::kBwdThreads - 1) / bl::kBwdThreads;
+    if (vpt <= 1) return launch_rmsnorm_bwd_v<kBf16X, 1>(X, rinv, g, dX, T, K, partial, sms, st);
+    if (vpt <= 2) return launch_rmsnorm_bwd_v<kBf16X, 2>(X, rinv, g, dX, T, K, partial, sms, st);
+    if (vpt <= 4) return launch_rmsnorm_bwd_v<kBf16X, 4>(X, rinv, g, dX, T, K, partial, sms, st);
+    if (vpt <= 8) return launch_rmsnorm_bwd_v<kBf16X, 8>(X, rinv, g, dX, T, K, partial, sms, st);
+    if (vpt <= 12) return launch_rmsnorm_bwd_v<kBf16X, 12>(X, rinv, g, dX, T, K, partial, sms, st);
+    return launch_rmsnorm_bwd_v<kBf16X, 16>(X, rinv, g, dX, T, K, partial, sms, st);
+}
 
 bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const float* g, float* dX, int64_t T,
-                          int64_t K, float* dg, void* ws, cudaStream_t st) {
-    const int grid = (int)(T < bl::kBwdBlocks ? T : bl::kBwdBlocks);
+                          int64_t K, float* dg, void* ws, int sms, cudaStream_t st) {
     float* partial = dg != nullptr ? static_cast<float*>(ws) : nullptr;
-    const size_t smem = dg != nullptr ? sizeof(float) * (size_t)K : 0;
-    if (smem > 48 * 1024) {
-        cudaError_t e = dt == BL_BF16
-                            ? cudaFuncSetAttribute(bl::rmsnorm_bwd_kernel<true>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                            : cudaFuncSetAttribute(bl::rmsnorm_bwd_kernel<false>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    }
-    if (dt == BL_BF16)
-        bl::rmsnorm_bwd_kernel<true><<<grid, bl::kBwdThreads, smem, st>>>(X, rinv, g, dX, (int)T, (int)K, partial);
-    else
-        bl::rmsnorm_bwd_kernel<false><<<grid, bl::kBwdThreads, smem, st>>>(X, rinv, g, dX, (int)T, (int)K, partial);
+    const int grid = dt == BL_BF16 ? launch_rmsnorm_bwd<true>(X, rinv, g, dX, T, K, partial, sms, st)
+                                   : launch_rmsnorm_bwd<false>(X, rinv, g, dX, T, K, partial, sms, st);
     BL_TRY(launched("rmsnorm_bwd"));
     if (dg != nullptr) {
-        bl::dg_reduce_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(partial, grid, (int)K, dg);
+        bl::dg_reduce_kernel<<<(unsigned)((K + 31) / 32), 1024, 0, st>>>(partial, grid, (int)K, dg);
         BL_TRY(launched("dg_reduce"));
     }
     return BL_OK;
 }
+
+// Row kernels keep a whole row in registers: d_in is limited to 16384.
+constexpr int64_t kMaxRowK = 16384;
 
 }  // namespace
 
@@ -344,6 +395,8 @@ bl_status bitlinear_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K
     BL_TRY(check_ptr(g, "g", false));
     BL_TRY(check_ptr(Xdq, "Xdq", false));
     BL_TRY(check_dims(T, 16, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
     BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
@@ -380,6 +433,8 @@ bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int64_t K, 
     BL_TRY(check_ptr(Xdq, "Xdq", false));
     BL_TRY(check_ptr(acc, "acc", false));
     BL_TRY(check_dims(T, N, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
     BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
@@ -402,6 +457,8 @@ bl_status bitlinear_backward_input(const void* dY, const void* X, bl_dtype dt, i
     BL_TRY(check_ptr(dg, "dg", false));
     BL_TRY(check_ptr(ws, "ws", dg != nullptr));
     BL_TRY(check_dims(T, N, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
     if (dg != nullptr)
         BL_REQUIRE(ws_bytes >= dg_ws_bytes(K), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", dg_ws_bytes(K),
                    ws_bytes);
@@ -409,7 +466,7 @@ bl_status bitlinear_backward_input(const void* dY, const void* X, bl_dtype dt, i
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     BL_TRY(run_grad_input_gemm(dY, dt, Wq_bf16, gamma, T, K, N, dX, st, dev));
-    return run_rmsnorm_bwd(X, dt, rinv, g, dX, T, K, dg, ws, st);
+    return run_rmsnorm_bwd(X, dt, rinv, g, dX, T, K, dg, ws, dev.sms, st);
 }
 
 bl_status bitlinear_grad_input(const void* dY, bl_dtype dt, int64_t T, int64_t K, int64_t N, const uint16_t* Wq_bf16,
@@ -436,12 +493,14 @@ bl_status bitlinear_rmsnorm_backward(const void* X, bl_dtype dt, int64_t T, int6
     BL_TRY(check_ptr(dg, "dg", false));
     BL_TRY(check_ptr(ws, "ws", dg != nullptr));
     BL_TRY(check_dims(T, 16, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
     if (dg != nullptr)
         BL_REQUIRE(ws_bytes >= dg_ws_bytes(K), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", dg_ws_bytes(K),
                    ws_bytes);
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
-    return run_rmsnorm_bwd(X, dt, rinv, g, dX_inout, T, K, dg, ws, static_cast<cudaStream_t>(stream));
+    return run_rmsnorm_bwd(X, dt, rinv, g, dX_inout, T, K, dg, ws, dev.sms, static_cast<cudaStream_t>(stream));
 }
 
 bl_status bitlinear_backward_weight(const void* dY, const void* Xdq, bl_dtype dt, int64_t T, int64_t K, int64_t N,

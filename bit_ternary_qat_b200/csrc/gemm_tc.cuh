@@ -4,22 +4,28 @@
 //
 // Three uses, one kernel template:
 //   forward      kind::i8   A = X_q  [T x K] (K-major), B = W_q int8 [N x K] (K-major)
-//                           epilogue y = (acc * gamma) / s_t  (P3 §3.1 output * scale)
+//                           epilogue y = acc * (gamma / s_t)   (P3 §3.1: the linear of the
+//                           dequantised operands times the scales, one factor per token)
 //   grad input   kind::f16  A = dY   [T x N] (K-major), B = W_q bf16 [N x K] read MN-major
-//                           epilogue dX_hat = gamma * acc     (STE: dY . W_dq)
+//                           epilogue dX_hat = gamma * acc       (STE: dY . W_dq)
 //   grad weight  kind::f16  A = dY read MN-major (contraction over tokens),
 //                           B = X_dq [T x K] read MN-major; epilogue dW = acc
 //
 // Structure (one CTA per SM, persistent over output tiles of 128 x kBN):
 //   warp 0      TMA producer: one elected thread streams A/B k-blocks (128 bytes of K per
-//               operand row, 128-byte swizzle) into a kStages-deep shared-memory ring.
+//               operand row, 128-byte swizzle) into a kTcStages-deep shared-memory ring.
 //   warp 1      allocates 2*kBN TMEM columns (two fp32/int32 accumulators), then one elected
 //               thread issues tcgen05.mma (M=128, N=kBN, K=32 bytes per instruction) and
 //               tcgen05.commit to release ring slots and to publish finished accumulators.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, rescale, store.
-//               Accumulators are double-buffered, so the epilogue of tile i overlaps the
-//               main loop of tile i+1.
-// Out-of-range rows/columns/k are zero-filled by TMA; the epilogue masks stores.
+//   warps 2..5  epilogue: each warp owns 32 accumulator rows (its TMEM lane quadrant).  Per
+//               128-byte column chunk it loads the accumulators with tcgen05.ld, rescales,
+//               writes its 32 rows into a 128-byte-swizzled shared-memory buffer (conflict
+//               free, one 16-byte chunk per store) and one lane issues a TMA tensor store of
+//               the 32-row box.  Two buffers per warp overlap the store of one chunk with
+//               the math of the next; the TMA store clips rows/columns past the matrix edge.
+//               Accumulators are double-buffered in TMEM, so the epilogue of tile i
+//               overlaps the main loop of tile i+1.
+// Out-of-range rows/columns/k of the operands are zero-filled by TMA.
 // Every mbarrier wait is bounded (see common.cuh): on a timeout all roles unwind, the
 // producer drains the loads it issued, the MMA thread drains its MMAs, TMEM is freed.
 #pragma once
@@ -28,22 +34,26 @@
 
 namespace bl {
 
-enum TcEpilogue : int { kEpiLinear = 0, kEpiScaleF32 = 1, kEpiF32 = 2 };
+enum TcEpilogue : int {
+    kEpiLinearBf16 = 0,   // y = acc * (gamma / s_t) -> bf16
+    kEpiScaleF32 = 1,     // gamma * acc -> fp32
+    kEpiF32 = 2,          // acc -> fp32
+    kEpiLinearF32 = 3,    // y = acc * (gamma / s_t) -> fp32
+};
 
 constexpr int kTcStages = 4;
 constexpr int kTcThreads = 192;
 constexpr int kTcBM = 128;
 constexpr int kTcABytes = kTcBM * 128;   // one stage of A: 128 rows x 128 bytes
+constexpr int kEpiBufBytes = 32 * 128;   // one staging buffer: 32 rows x 128 bytes
+constexpr int kEpiBytes = 4 * 2 * kEpiBufBytes;
 
 struct TcGemmArgs {
     int M, N, K;                 // D is M x N, contraction length K (elements)
     int m_tiles, n_tiles, k_blocks;
-    void* out;                   // D, row stride ldo elements
-    int64_t ldo;
-    int out_bf16;                // kEpiLinear: 1 = bf16 output, 0 = fp32
-    int32_t* acc_out;            // kEpiLinear: optional int32 accumulators (row stride ldo)
-    const float* row_scale;      // kEpiLinear: s_t of each output row
-    const float* gamma;          // kEpiLinear / kEpiScaleF32
+    int32_t* acc_out;            // linear epilogues: optional int32 accumulators [M x N] (plain stores)
+    const float* row_scale;      // linear epilogues: s_t of each output row
+    const float* gamma;          // linear / scale epilogues
     uint64_t wait_ns;            // bound of every mbarrier wait
 };
 
@@ -52,14 +62,18 @@ __host__ __device__ constexpr int tc_b_bytes() { return kBN * 128; }
 
 template <int kBN>
 __host__ __device__ constexpr size_t tc_smem_bytes() {
-    return 1024 /* alignment slack */ + (size_t)kTcStages * (kTcABytes + tc_b_bytes<kBN>()) +
+    return 1024 /* alignment slack */ + (size_t)kTcStages * (kTcABytes + tc_b_bytes<kBN>()) + kEpiBytes +
            (2 * kTcStages + 4) * sizeof(uint64_t) + 16;
 }
+
+__host__ __device__ constexpr bool epi_is_linear(int e) { return e == kEpiLinearBf16 || e == kEpiLinearF32; }
+// Output columns per 128-byte chunk.
+__host__ __device__ constexpr int epi_chunk_cols(int e) { return e == kEpiLinearBf16 ? 64 : 32; }
 
 template <bool kInt8, bool kAMN, bool kBMN, int kBN, int kEpi>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmD, const TcGemmArgs args) {
     static_assert(kBN % 64 == 0 && kBN <= 256, "kBN");
     static_assert(!kInt8 || (!kAMN && !kBMN), "int8 operands are K-major here");
     constexpr int kBBytes = tc_b_bytes<kBN>();
@@ -68,12 +82,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kInstrK = 4;                            // MMAs per stage (32 bytes of K each)
     constexpr uint32_t kIdesc = umma_idesc(kInt8, kAMN, kBMN, kTcBM, kBN);
     constexpr uint32_t kTmemCols = 2 * kBN;
+    constexpr int kChunkCols = epi_chunk_cols(kEpi);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + kTcStages * kTcABytes;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + kTcStages * kBBytes);
+    uint8_t* sE = sB + kTcStages * kBBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiBytes);
     uint64_t* empty = full + kTcStages;
     uint64_t* tfull = empty + kTcStages;
     uint64_t* tempty = tfull + 2;
@@ -98,6 +114,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmD);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -195,7 +212,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
     } else {
         // ----------------------------------------------------------------- epilogue
-        const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad + 32) belong to this warp
+        const int quad = warp & 3;          // TMEM lanes [32*quad, 32*quad + 32) belong to this warp
+        uint8_t* ebuf = sE + (warp - 2) * 2 * kEpiBufBytes;
+        int buf = 0;
         int tcount = 0;
         float gm = 1.0f;
         if constexpr (kEpi != kEpiF32) gm = __ldg(args.gamma);
@@ -206,55 +225,83 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             const int mb = tile % args.m_tiles;
             const int nb = tile / args.m_tiles;
-            const int row = mb * kTcBM + quad * 32 + lane;
+            const int row0 = mb * kTcBM + quad * 32;
+            const int row = row0 + lane;
             const bool row_ok = row < args.M;
-            float rs = 1.0f;
-            if constexpr (kEpi == kEpiLinear) rs = row_ok ? __ldg(args.row_scale + row) : 1.0f;
+            float cs = 1.0f;   // per-token factor gamma / s_t
+            if constexpr (epi_is_linear(kEpi)) cs = row_ok ? __fdiv_rn(gm, __ldg(args.row_scale + row)) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(b * kBN);
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += 32) {
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(t_row + c0, r);
-                tmem_ld_wait();
+            for (int c0 = 0; c0 < kBN; c0 += kChunkCols) {
                 const int col0 = nb * kBN + c0;
+                if (col0 >= args.N) break;                     // warp-uniform
+                uint32_t ra[32], rb[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + c0, ra);
+                if constexpr (kChunkCols == 64) {
+                    tmem_ld_32x32b_x32(t_row + c0 + 32, rb);
+                } else {
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int col = col0 + g8 * 8;
-                    // N % 16 == 0: a group of 8 columns is entirely in or entirely out
-                    if (!row_ok || col >= args.N) continue;
-                    float v[8];
+                    for (int i = 0; i < 32; ++i) rb[i] = 0u;
+                }
+                tmem_ld_wait();
+                auto r = [&](int i) -> uint32_t { return i < 32 ? ra[i] : rb[i - 32]; };
+                // this lane's 128-byte row segment as 8 x 16-byte chunks
+                uint4 v[8];
+                if constexpr (kEpi == kEpiLinearBf16) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t raw = r[g8 * 8 + e];
-                        if constexpr (kEpi == kEpiLinear) {
-                            v[e] = __fdiv_rn(__fmul_rn(static_cast<float>(static_cast<int32_t>(raw)), gm), rs);
-                        } else if constexpr (kEpi == kEpiScaleF32) {
-                            v[e] = __fmul_rn(gm, __uint_as_float(raw));
-                        } else {
-                            v[e] = __uint_as_float(raw);
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e))), cs);
+                            const float hi = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e + 1))), cs);
+                            w[e] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
                         }
+                        v[j] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    const int64_t off = static_cast<int64_t>(row) * args.ldo + col;
-                    if (kEpi == kEpiLinear && args.out_bf16) {
-                        uint4 o;
-                        o.x = (uint32_t)float_to_bf16_bits(v[0]) | ((uint32_t)float_to_bf16_bits(v[1]) << 16);
-                        o.y = (uint32_t)float_to_bf16_bits(v[2]) | ((uint32_t)float_to_bf16_bits(v[3]) << 16);
-                        o.z = (uint32_t)float_to_bf16_bits(v[4]) | ((uint32_t)float_to_bf16_bits(v[5]) << 16);
-                        o.w = (uint32_t)float_to_bf16_bits(v[6]) | ((uint32_t)float_to_bf16_bits(v[7]) << 16);
-                        *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.out) + off) = o;
-                    } else {
-                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.out) + off);
-                        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-                    }
-                    if constexpr (kEpi == kEpiLinear) {
-                        if (args.acc_out != nullptr) {
-                            int4* dst = reinterpret_cast<int4*>(args.acc_out + off);
-                            dst[0] = make_int4((int)r[g8 * 8 + 0], (int)r[g8 * 8 + 1], (int)r[g8 * 8 + 2], (int)r[g8 * 8 + 3]);
-                            dst[1] = make_int4((int)r[g8 * 8 + 4], (int)r[g8 * 8 + 5], (int)r[g8 * 8 + 6], (int)r[g8 * 8 + 7]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float f[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t raw = r(4 * j + e);
+                            if constexpr (kEpi == kEpiLinearF32)
+                                f[e] = __fmul_rn(static_cast<float>(static_cast<int32_t>(raw)), cs);
+                            else if constexpr (kEpi == kEpiScaleF32)
+                                f[e] = __fmul_rn(gm, __uint_as_float(raw));
+                            else
+                                f[e] = __uint_as_float(raw);
                         }
+                        v[j] = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                          __float_as_uint(f[3]));
+                    }
+                }
+                // the staging buffer's previous store (two chunks ago) must have been read
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint8_t* sb = ebuf + buf * kEpiBufBytes;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) = v[j];
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmD, sb, col0, row0);
+                    bulk_commit_group();
+                }
+                buf ^= 1;
+                if constexpr (epi_is_linear(kEpi)) {
+                    if (args.acc_out != nullptr && row_ok) {
+                        // debug copy of the exact int32 accumulators (plain stores)
+                        int32_t* dst = args.acc_out + static_cast<int64_t>(row) * args.N + col0;
+#pragma unroll
+                        for (int j = 0; j < kChunkCols / 4; ++j)
+                            if (col0 + 4 * j < args.N)
+                                reinterpret_cast<int4*>(dst)[j] = make_int4((int)r(4 * j), (int)r(4 * j + 1),
+                                                                            (int)r(4 * j + 2), (int)r(4 * j + 3));
                     }
                 }
             }
@@ -262,6 +309,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);
         }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     tc_fence_before();

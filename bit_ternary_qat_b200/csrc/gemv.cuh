@@ -2,7 +2,8 @@
 //
 // P5 ("1.58-bit量化技术…") §3.1: a ternary weight turns the multiply-accumulate into
 // add (W = +1), subtract (W = -1) or skip (W = 0); §4.1: codes 00 -> 0, 01 -> +1,
-// 10 -> -1, 11 reserved (decodes to 0 here).  Output y = (acc * gamma) / s_b.
+// 10 -> -1, 11 reserved (decodes to 0 here).  Output y = acc * (gamma / s_b), the factor
+// formed once per activation row.
 //
 // The weights are streamed from HBM exactly once (N x K/4 bytes, one warp per output row,
 // lanes on consecutive 8-byte chunks so any K % 32 == 0 row is aligned).  No code is ever decoded to a
@@ -74,42 +75,53 @@ __global__ void __launch_bounds__(kGemvThreads) ternary_gemv_kernel(const uint8_
 #pragma unroll
             for (int a = 0; a < kAcc; ++a) acc[b][a] = 0;
         const uint2* row = reinterpret_cast<const uint2*>(packed + static_cast<int64_t>(n) * (K / 4));
-#pragma unroll 2
-        for (int c = lane; c < nchunk; c += 32) {
-            const uint2 pw = __ldcs(row + c);
+        constexpr int kU = 8;   // 8-byte chunks per lane loaded before any math (64 codes x 8)
+        for (int cb = 0; cb < nchunk; cb += 32 * kU) {
+            uint2 pw[kU];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t w = h == 0 ? pw.x : pw.y;
-                int lo[4], hi[4];
-                if constexpr (kInPlace) {
+            for (int u = 0; u < kU; ++u) {
+                const int c = cb + lane + 32 * u;
+                pw[u] = c < nchunk ? __ldcs(row + c) : make_uint2(0u, 0u);
+            }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        lo[j] = static_cast<int>(w & (0x01010101u << (2 * j)));
-                        hi[j] = static_cast<int>(w & (0x02020202u << (2 * j)));
-                    }
-                } else {
-                    const uint32_t w1 = w >> 1;
+            for (int u = 0; u < kU; ++u) {
+                const int c = cb + lane + 32 * u;
+                if (c >= nchunk) continue;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        lo[j] = static_cast<int>((w >> (2 * j)) & 0x01010101u);
-                        hi[j] = static_cast<int>((w1 >> (2 * j)) & 0x01010101u);
-                    }
-                }
-#pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    if (b < B) {
-                        const int4 xv = xs[gemv_xs_index(b, h, c, nchunk)];
-                        const int xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t w = h == 0 ? pw[u].x : pw[u].y;
+                    int lo[4], hi[4];
+                    if constexpr (kInPlace) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            if constexpr (kInPlace) {
-                                // bytes of lo[j]/hi[j] are 0 or 2^(2j) / 2^(2j+1): read them as
-                                // unsigned (2^7 does not fit a signed byte)
-                                acc[b][2 * j] = dp4a_us(static_cast<uint32_t>(lo[j]), xw[j], acc[b][2 * j]);
-                                acc[b][2 * j + 1] = dp4a_us(static_cast<uint32_t>(hi[j]), xw[j], acc[b][2 * j + 1]);
-                            } else {
-                                acc[b][0] = __dp4a(lo[j], xw[j], acc[b][0]);
-                                acc[b][1] = __dp4a(hi[j], xw[j], acc[b][1]);
+                            lo[j] = static_cast<int>(w & (0x01010101u << (2 * j)));
+                            hi[j] = static_cast<int>(w & (0x02020202u << (2 * j)));
+                        }
+                    } else {
+                        const uint32_t w1 = w >> 1;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            lo[j] = static_cast<int>((w >> (2 * j)) & 0x01010101u);
+                            hi[j] = static_cast<int>((w1 >> (2 * j)) & 0x01010101u);
+                        }
+                    }
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        if (b < B) {
+                            const int4 xv = xs[gemv_xs_index(b, h, c, nchunk)];
+                            const int xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if constexpr (kInPlace) {
+                                    // bytes of lo[j]/hi[j] are 0 or 2^(2j) / 2^(2j+1): read them as
+                                    // unsigned (2^7 does not fit a signed byte)
+                                    acc[b][2 * j] = dp4a_us(static_cast<uint32_t>(lo[j]), xw[j], acc[b][2 * j]);
+                                    acc[b][2 * j + 1] =
+                                        dp4a_us(static_cast<uint32_t>(hi[j]), xw[j], acc[b][2 * j + 1]);
+                                } else {
+                                    acc[b][0] = __dp4a(lo[j], xw[j], acc[b][0]);
+                                    acc[b][1] = __dp4a(hi[j], xw[j], acc[b][1]);
+                                }
                             }
                         }
                     }
@@ -130,7 +142,7 @@ __global__ void __launch_bounds__(kGemvThreads) ternary_gemv_kernel(const uint8_
                 const int tot = warp_sum(part);
                 if (lane == 0) {
                     const int64_t o = static_cast<int64_t>(b) * N + n;
-                    y[o] = __fdiv_rn(__fmul_rn(static_cast<float>(tot), gm), __ldg(sx + b));
+                    y[o] = __fmul_rn(static_cast<float>(tot), __fdiv_rn(gm, __ldg(sx + b)));
                     if (acc_out != nullptr) acc_out[o] = tot;
                 }
             }

@@ -13,7 +13,7 @@
 //
 // The ternary decision needs no per-element division.  fl32(w / gamma) is monotone in w,
 // so {w > 0 : fl32(w/gamma) > 0.5} = {w >= w*} for one fp32 threshold w*, found by a
-// 31-step bisection over fp32 bit patterns that evaluates the IEEE division itself.
+// bisection over fp32 bit patterns (near gamma/2) that evaluates the IEEE division itself.
 // Because the division is sign-symmetric, W_q = sign(w) * [|w| >= w*] reproduces
 // clamp(round_half_even(fl32(w/gamma)), -1, 1) exactly for every finite w.
 #pragma once
@@ -24,11 +24,11 @@ namespace bl {
 constexpr int kWqThreads = 256;
 constexpr int kWqMaxPartials = 1184;   // 8 blocks per SM on 148 SMs
 
-// Number of pass-1 blocks for n elements: depends on n only, so gamma is the same on
-// every device.
+// Number of pass-1 blocks for n elements (4 float4 loads per thread): depends on n only, so
+// gamma is the same on every device.
 __host__ __device__ inline int wq_num_partials(int64_t n) {
     int64_t vecs = n / 4;
-    int64_t p = (vecs + kWqThreads * 16 - 1) / (kWqThreads * 16);
+    int64_t p = (vecs + kWqThreads * 4 - 1) / (kWqThreads * 4);
     if (p < 1) p = 1;
     if (p > kWqMaxPartials) p = kWqMaxPartials;
     return static_cast<int>(p);
@@ -39,8 +39,23 @@ __global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float
     __shared__ double red[kWqThreads / 32];
     const int64_t nvec = n / 4;
     const float4* w4 = reinterpret_cast<const float4*>(W);
+    const int64_t stride = (int64_t)gridDim.x * kWqThreads;
     double acc = 0.0;
-    for (int64_t i = blockIdx.x * (int64_t)kWqThreads + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * kWqThreads) {
+    int64_t i = blockIdx.x * (int64_t)kWqThreads + threadIdx.x;
+    // four independent loads in flight per thread
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(w4 + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc += (double)fabsf(v[u].x);
+            acc += (double)fabsf(v[u].y);
+            acc += (double)fabsf(v[u].z);
+            acc += (double)fabsf(v[u].w);
+        }
+    }
+    for (; i < nvec; i += stride) {
         float4 v = __ldg(w4 + i);
         acc += (double)fabsf(v.x);
         acc += (double)fabsf(v.y);
@@ -57,13 +72,20 @@ __global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float
     }
 }
 
-// Smallest positive fp32 w with fl32(w / gamma) > 0.5 (gamma >= 1e-5 > 0).
+// Smallest positive fp32 w with fl32(w / gamma) > 0.5 (gamma >= 1e-5 > 0).  The answer is
+// within a few ulps of gamma/2, so the bisection starts on +-8 ulps around it and falls
+// back to the whole positive range if that window does not bracket the answer.
 __device__ __forceinline__ float ternary_threshold(float gamma) {
-    uint32_t lo = 0u;            // 0 / gamma = 0      -> not above 0.5
-    uint32_t hi = 0x7f7fffffu;   // FLT_MAX / gamma   -> above 0.5
+    auto above = [gamma](uint32_t bits) { return __fdiv_rn(__uint_as_float(bits), gamma) > 0.5f; };
+    const uint32_t c = __float_as_uint(__fmul_rn(0.5f, gamma));
+    uint32_t lo = c - 8u, hi = c + 8u;
+    if (above(lo) || !above(hi)) {
+        lo = 0u;            // 0 / gamma = 0      -> not above 0.5
+        hi = 0x7f7fffffu;   // FLT_MAX / gamma    -> above 0.5
+    }
     while (hi - lo > 1u) {
-        uint32_t mid = lo + ((hi - lo) >> 1);
-        if (__fdiv_rn(__uint_as_float(mid), gamma) > 0.5f) hi = mid; else lo = mid;
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        if (above(mid)) hi = mid; else lo = mid;
     }
     return __uint_as_float(hi);
 }

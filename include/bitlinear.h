@@ -25,7 +25,9 @@
  * Sizes and alignment (validated on the host before anything is launched):
  *   - T >= 1, N >= 1, K >= 1; K % 32 == 0 (whole 64-bit words of 2-bit codes per row,
  *     P5 §5.1); N % 16 == 0 (16-byte aligned rows of Y and dY for TMA and vector
- *     stores); every pointer 16-byte aligned; T, N, K < 2^31.
+ *     stores); every pointer 16-byte aligned; T, N, K < 2^31;
+ *   - K <= 16384 for the entry points with a per-token row kernel (act quant, forward,
+ *     backward input, RMSNorm backward): those kernels hold a whole row in registers.
  * Numerics: fp32 quantiser arithmetic with round-half-to-even (torch.round in the
  * pages' snippets), fp64 reductions, exact int32 accumulation for the int8 x ternary
  * contraction.  Inputs must be finite.
@@ -123,7 +125,8 @@ BL_API bl_status bitlinear_act_quant(const void* X, bl_dtype x_dt, int64_t T, in
  * The int8 x ternary contraction with its rescale (P3 §3.1 F.linear(x_quant, w_quant)
  * * scale; P5 §3.1 add / subtract / skip):
  *   acc[t,n] = sum_k X_q[t,k] * W_q[n,k]          exact int32 (tcgen05 kind::i8)
- *   Y[t,n]   = (acc[t,n] * gamma) / s_t            fp32, then rounded to y_dt
+ *   Y[t,n]   = acc[t,n] * (gamma / s_t)            fp32 (the factor formed once per token),
+ *                                                  then rounded to y_dt
  * Xq int8 [T x K], sx fp32 [T], Wq_i8 int8 [N x K], gamma fp32 [1] (device).
  * Y [T x N] of y_dt.  acc int32 [T x N] optional (debug / parity). */
 BL_API bl_status bitlinear_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
@@ -195,7 +198,7 @@ BL_API bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t
  * Decode GEMV over packed ternary weights (P5 §3.1 W=+1 -> y += x, W=-1 -> y -= x,
  * W=0 -> skip; P5 §4.1 codes, reserved 11 decodes to 0):
  *   acc[b,n] = sum_k decode(Wpacked[n,k]) * xq[b,k]   exact int32
- *   y[b,n]   = (acc[b,n] * gamma) / sx[b]              fp32
+ *   y[b,n]   = acc[b,n] * (gamma / sx[b])              fp32
  * Wpacked uint8 [N x K/4]; gamma fp32 [1]; xq int8 [B x K]; sx fp32 [B];
  * y fp32 [B x N]; acc int32 [B x N] optional.  1 <= B <= 16, K <= 65536. */
 BL_API bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K,

@@ -85,6 +85,7 @@ def test_forward_validation(L):
     assert call(N=8) == 2
     assert call(Y=ODD) == 3
     assert call(eps=-1.0) == 1
+    assert call(K=16384 + 32) == 2          # row kernels hold a row in registers
 
 
 def test_backward_and_gemv_validation(L):

@@ -1,0 +1,126 @@
+"""Host-side checks of the exact-arithmetic shortcuts the CUDA kernels take.
+
+The kernels avoid per-element divisions and float<->int conversions while reproducing
+the oracle's fp32 results bit for bit.  These tests check the identities they rely on
+with exact rational arithmetic (fractions) or exact fp32 emulation (numpy float32 ops
+are IEEE round-to-nearest-even), independently of any GPU:
+
+* act quant: fl(q / s) == fl(y1 + fl(q - s*y1) * c) with c = fl(1/s), y0 = fl(q*c),
+  y1 = fl(y0 + fl(q - s*y0) * c) (one reciprocal per row, two FMA corrections), for
+  every q in [-128, 127];
+* act quant: round-half-to-even of v via fl(v + 1.5*2^23) for |v| <= 128;
+* weight quant: the ternary code equals sign(w) * [|w| >= w*] with w* found by the
+  narrow bisection around gamma/2;
+* decode GEMV: sum_k dec(c_k) x_k == sum_j dp4a(lo_j, x_j) - dp4a(hi_j, x_j) with the
+  interleaved activation words.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+
+def rn32(x: Fraction) -> Fraction:
+    """Round a rational to the nearest fp32 value, ties to even (normal range)."""
+    if x == 0:
+        return Fraction(0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = math.floor(math.log2(a.numerator) - math.log2(a.denominator))
+    # fix e so that 2^e <= a < 2^(e+1)
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    scale = Fraction(2) ** (23 - e)
+    m = round(a * scale)            # Python rounds half to even
+    return sign * Fraction(m) / scale
+
+
+def f32(x: Fraction) -> np.float32:
+    return np.float32(float(x))
+
+
+def test_markstein_quotient_is_correctly_rounded():
+    rng = np.random.default_rng(0)
+    # s = fl(127 / m) over a wide range of row absmax values m, plus the clamp value
+    ms = np.concatenate([10.0 ** rng.uniform(-5, 4, size=150), [1e-5, 1.0, 2.0, 127.0, 1e4]])
+    for m in ms:
+        s = Fraction(np.float32(np.float32(127.0) / np.float32(max(np.float32(m), np.float32(1e-5)))).item())
+        c = rn32(Fraction(1) / s)
+        for qi in range(0, 129):
+            for q in (Fraction(qi), Fraction(-qi)):
+                if q < -128 or q > 127:
+                    continue
+                y0 = rn32(q * c)
+                y1 = rn32(y0 + rn32(q - s * y0) * c)
+                e1 = rn32(q - s * y1)
+                assert q - s * y1 == e1         # y1 is faithful: the second residual is exact
+                y = rn32(y1 + e1 * c)
+                assert y == rn32(q / s), (float(q), float(s))
+
+
+def test_magic_constant_rounds_half_to_even():
+    magic = np.float32(12582912.0)
+    v = np.concatenate([np.arange(-128, 128.5, 0.5, dtype=np.float32),
+                        np.random.default_rng(1).uniform(-128, 128, 200000).astype(np.float32),
+                        np.nextafter(np.arange(-128, 129, dtype=np.float32) + np.float32(0.5), np.float32(0)),
+                        np.nextafter(np.arange(-128, 129, dtype=np.float32) + np.float32(0.5), np.float32(1e9))])
+    t = (v + magic).astype(np.float32)
+    q = t.view(np.int32) - 0x4B400000
+    assert np.array_equal(q, np.rint(v).astype(np.int32))
+    assert np.array_equal((t - magic).astype(np.float32), np.rint(v))
+
+
+def _threshold_narrow(gamma: np.float32) -> np.float32:
+    def above(bits):
+        return np.float32(np.uint32(bits).view(np.float32)) / gamma > np.float32(0.5)
+    c = int(np.float32(np.float32(0.5) * gamma).view(np.uint32))
+    lo, hi = c - 8, c + 8
+    if above(lo) or not above(hi):
+        lo, hi = 0, 0x7F7FFFFF
+    while hi - lo > 1:
+        mid = lo + ((hi - lo) >> 1)
+        if above(mid):
+            hi = mid
+        else:
+            lo = mid
+    return np.uint32(hi).view(np.float32)
+
+
+def test_ternary_threshold_equals_round_clamp():
+    rng = np.random.default_rng(2)
+    for gamma in [np.float32(1e-5), np.float32(0.0159), np.float32(0.265625), np.float32(3.7)] + \
+            [np.float32(g) for g in 10.0 ** rng.uniform(-5, 2, 40)]:
+        thr = _threshold_narrow(gamma)
+        # dense neighbourhood of the threshold and random weights
+        b = int(thr.view(np.uint32))
+        near = np.arange(b - 64, b + 64, dtype=np.uint32).view(np.float32)
+        w = np.concatenate([near, -near, rng.normal(0, float(gamma), 4096).astype(np.float32),
+                            np.array([0.0, -0.0, 1.5 * gamma, -2.5 * gamma], dtype=np.float32)])
+        ref = np.clip(np.rint((w / gamma).astype(np.float32)), -1, 1).astype(np.int8)
+        got = np.where(w >= thr, 1, np.where(w <= -thr, -1, 0)).astype(np.int8)
+        assert np.array_equal(got, ref), float(gamma)
+
+
+def test_gemv_bitplane_identity():
+    rng = np.random.default_rng(3)
+    K = 64
+    codes = rng.integers(0, 4, size=K)           # includes the reserved 11
+    x = rng.integers(-128, 128, size=K).astype(np.int64)
+    dec = np.where(codes == 1, 1, np.where(codes == 2, -1, 0))
+    ref = int(np.sum(dec * x))
+    # pack 16 codes per 32-bit word, element k at bits 2*(k % 16) of word k // 16
+    words = [sum(int(codes[16 * g + i]) << (2 * i) for i in range(16)) for g in range(K // 16)]
+    tot = 0
+    for g, w in enumerate(words):
+        for j in range(4):
+            xs = [int(x[16 * g + 4 * i + j]) for i in range(4)]        # interleaved activation word
+            lo = [(w >> (8 * i + 2 * j)) & 1 for i in range(4)]
+            hi = [(w >> (8 * i + 2 * j + 1)) & 1 for i in range(4)]
+            tot += sum(l * xv for l, xv in zip(lo, xs)) - sum(h * xv for h, xv in zip(hi, xs))
+            # in-place masks: byte i of w & (0x01010101 << 2j) is lo * 2^(2j)
+            m = w & (0x01010101 << (2 * j))
+            assert [(m >> (8 * i)) & 0xFF for i in range(4)] == [l << (2 * j) for l in lo]
+    assert tot == ref
