@@ -94,11 +94,14 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
     const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
     const uint4* xrow = reinterpret_cast<const uint4*>(X) + row_vec0;
 
-    uint4 raw[VPT];
+    // the row, widened to fp32, in registers (read from HBM once)
+    float x[VPT][E];
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
         const int v = threadIdx.x + j * NT;
-        raw[j] = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 raw = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[j][e] = V::elem(raw, e);
     }
 
     // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order
@@ -109,25 +112,26 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
         for (int j = 0; j < VPT; ++j)
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const double x = static_cast<double>(V::elem(raw[j], e));
-                ss = fma(x, x, ss);
+                const double xd = static_cast<double>(x[j][e]);
+                ss = fma(xd, xd, ss);
             }
         ss = block_sum_f64<NT>(ss, red_d);
         r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(eps)));
     }
 
-    // x_hat = fl(fl(x * r) * g) and its absmax
+    // x_hat = fl(fl(x * r) * g) (kept in place of x) and its absmax
     float m = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
         const int v = threadIdx.x + j * NT;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            float h = V::elem(raw[j], e);
+            float h = x[j][e];
             if (apply_norm) {
                 h = __fmul_rn(h, r);
                 if (g != nullptr && v < nvec) h = __fmul_rn(h, __ldg(g + v * E + e));
             }
+            x[j][e] = h;
             m = fmaxf(m, fabsf(h));
         }
     }
@@ -139,45 +143,37 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
         if (apply_norm) rinv[t] = r;
     }
 
-    // codes and dequantised values
+    // codes and dequantised values.  |x_hat * s| <= 127 * (1 + 2^-23) for finite inputs,
+    // so rint(x_hat * s) is in [-127, 127]; the integer clamp is kept for robustness.
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
         const int v = threadIdx.x + j * NT;
         if (v >= nvec) continue;
-        int q[E];
+        uint32_t qb[E];
         float dq[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            float h = V::elem(raw[j], e);
-            if (apply_norm) {
-                h = __fmul_rn(h, r);
-                if (g != nullptr) h = __fmul_rn(h, __ldg(g + v * E + e));
-            }
-            const float tq = __fadd_rn(__fmul_rn(h, s), kRoundMagic);     // 1.5*2^23 + rint(h*s)
-            int qi = __float_as_int(tq) - kRoundMagicBits;
-            qi = max(-128, min(127, qi));
-            q[e] = qi;
-            dq[e] = div_by_scale(static_cast<float>(qi), s, c);
+            const float tq = __fadd_rn(__fmul_rn(x[j][e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
+            const int qi = max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
+            qb[e] = static_cast<uint32_t>(qi) & 0xFFu;
+            dq[e] = div_by_scale(__fsub_rn(tq, kRoundMagic), s, c);
         }
         if constexpr (kBf16) {
             uint2 packed;
-            packed.x = (uint32_t)(q[0] & 0xFF) | ((uint32_t)(q[1] & 0xFF) << 8) | ((uint32_t)(q[2] & 0xFF) << 16) |
-                       ((uint32_t)(q[3] & 0xFF) << 24);
-            packed.y = (uint32_t)(q[4] & 0xFF) | ((uint32_t)(q[5] & 0xFF) << 8) | ((uint32_t)(q[6] & 0xFF) << 16) |
-                       ((uint32_t)(q[7] & 0xFF) << 24);
+            packed.x = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
+            packed.y = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
             reinterpret_cast<uint2*>(Xq)[row_vec0 + v] = packed;
             if (Xdq != nullptr) {
-                uint4 o;
-                o.x = (uint32_t)float_to_bf16_bits(dq[0]) | ((uint32_t)float_to_bf16_bits(dq[1]) << 16);
-                o.y = (uint32_t)float_to_bf16_bits(dq[2]) | ((uint32_t)float_to_bf16_bits(dq[3]) << 16);
-                o.z = (uint32_t)float_to_bf16_bits(dq[4]) | ((uint32_t)float_to_bf16_bits(dq[5]) << 16);
-                o.w = (uint32_t)float_to_bf16_bits(dq[6]) | ((uint32_t)float_to_bf16_bits(dq[7]) << 16);
-                reinterpret_cast<uint4*>(Xdq)[row_vec0 + v] = o;
+                uint32_t o[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(dq[2 * i], dq[2 * i + 1]);
+                    o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                reinterpret_cast<uint4*>(Xdq)[row_vec0 + v] = make_uint4(o[0], o[1], o[2], o[3]);
             }
         } else {
-            const uint32_t packed = (uint32_t)(q[0] & 0xFF) | ((uint32_t)(q[1] & 0xFF) << 8) |
-                                    ((uint32_t)(q[2] & 0xFF) << 16) | ((uint32_t)(q[3] & 0xFF) << 24);
-            reinterpret_cast<uint32_t*>(Xq)[row_vec0 + v] = packed;
+            reinterpret_cast<uint32_t*>(Xq)[row_vec0 + v] = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
             if (Xdq != nullptr) reinterpret_cast<float4*>(Xdq)[row_vec0 + v] = make_float4(dq[0], dq[1], dq[2], dq[3]);
         }
     }

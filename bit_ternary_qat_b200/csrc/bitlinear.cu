@@ -378,7 +378,7 @@ bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K, int8_t* W
     BL_TRY(launched("absmean_partial"));
     const int64_t groups = n / 16;
     int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
-    const int64_t cap = (int64_t)dev.sms * 8;
+    const int64_t cap = (int64_t)dev.sms * 4;
     if (blocks > cap) blocks = cap;
     bl::ternary_quant_kernel<<<(unsigned)blocks, bl::kWqThreads, 0, st>>>(W, n, partials, parts, Wq_i8, Wq_bf16,
                                                                           Wpacked, gamma);
@@ -551,29 +551,36 @@ bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, in
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t smem = (size_t)B * (size_t)K;   // B x K/16 groups x 16 bytes
+    const int ntiles = B <= 8 ? 1 : 2;
+    const size_t smem = (size_t)(8 * ntiles) * (size_t)(K / 16 + 1) * 16;   // padded activation words
     BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
-               "GEMV stages B*K = %zu activation bytes in shared memory; at most %d fit", smem, dev.max_smem_optin);
-    const int rows_per_block = bl::kGemvWarps;
-    int64_t need = (N + rows_per_block - 1) / rows_per_block;
-#define BL_GEMV_CASE(NBV)                                                                                          \
+               "GEMV stages %zu activation bytes in shared memory; at most %d fit (reduce B or K)", smem,
+               dev.max_smem_optin);
+    const int64_t row_groups = N / 16;
+    // warps per row group: enough that each warp streams about one load batch per row group
+    const int64_t nsc = (K / 16 + 7) / 8;
+    const int64_t batch = ntiles == 1 ? 8 : 4;
+    int ks = 1;
+    while (ks < bl::kGemvMmaWarps && (nsc + ks - 1) / ks > batch) ks *= 2;
+    // few row groups: split K further so that every SM gets work
+    while (ks < bl::kGemvMmaWarps && row_groups * ks < (int64_t)dev.sms * bl::kGemvMmaWarps) ks *= 2;
+    const int64_t rs = bl::kGemvMmaWarps / ks;
+    const int64_t need = (row_groups + rs - 1) / rs;
+#define BL_GEMV_CASE(NTV)                                                                                          \
     {                                                                                                              \
-        auto kern = bl::ternary_gemv_kernel<NBV>;                                                                  \
-        if (smem > 48 * 1024) {                                                                                    \
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);    \
-            if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));     \
-        }                                                                                                          \
+        auto kern = bl::ternary_gemv_mma_kernel<NTV>;                                                              \
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));         \
         int per_sm = 0;                                                                                            \
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kGemvThreads, smem);                      \
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kGemvMmaThreads, smem);                   \
         if (per_sm < 1) per_sm = 1;                                                                                \
         int64_t grid = (int64_t)dev.sms * per_sm;                                                                  \
         if (grid > need) grid = need;                                                                              \
-        kern<<<(unsigned)grid, bl::kGemvThreads, smem, st>>>(Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, y,   \
-                                                             acc);                                                 \
+        kern<<<(unsigned)grid, bl::kGemvMmaThreads, smem, st>>>(Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, ks, \
+                                                                y, acc);                                           \
     }
-    if (B == 1) BL_GEMV_CASE(1)
-    else if (B <= 4) BL_GEMV_CASE(4)
-    else BL_GEMV_CASE(16)
+    if (ntiles == 1) BL_GEMV_CASE(1)
+    else BL_GEMV_CASE(2)
 #undef BL_GEMV_CASE
     return launched("ternary_gemv");
 }

@@ -136,25 +136,25 @@ __global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_kernel(const void* __
 }
 
 // dg[k] = sum_p partial[p][k] in a fixed order.  A block handles 32 columns with 32 warps:
-// lane = column, warp w sums partial rows w, w + 32, ... (four independent accumulators,
-// so four loads are in flight per thread), then warp 0 adds the 32 warp sums in order.
+// lane = column, warp w loads partial rows w, w + 32, ... all at once (at most
+// kBwdMaxBlocks / 32 loads, all in flight), adds them in order, then warp 0 adds the 32
+// warp sums in order.
 __global__ void __launch_bounds__(1024) dg_reduce_kernel(const float* __restrict__ partial, int nparts, int K,
                                                          float* __restrict__ dg) {
+    constexpr int kPerWarp = (kBwdMaxBlocks + 31) / 32;
     __shared__ float red[32][33];
     const int c = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int k = blockIdx.x * 32 + c;
-    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-    if (k < K) {
-        int p = w;
-        for (; p + 96 < nparts; p += 128) {
-            a0 += partial[static_cast<int64_t>(p) * K + k];
-            a1 += partial[static_cast<int64_t>(p + 32) * K + k];
-            a2 += partial[static_cast<int64_t>(p + 64) * K + k];
-            a3 += partial[static_cast<int64_t>(p + 96) * K + k];
-        }
-        for (; p < nparts; p += 32) a0 += partial[static_cast<int64_t>(p) * K + k];
+    float v[kPerWarp];
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+        const int p = w + 32 * i;
+        v[i] = (k < K && p < nparts) ? __ldcs(partial + static_cast<int64_t>(p) * K + k) : 0.0f;
     }
-    red[w][c] = (a0 + a1) + (a2 + a3);
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) s += v[i];
+    red[w][c] = s;
     __syncthreads();
     if (w == 0 && k < K) {
         float tot = 0.0f;

@@ -72,87 +72,114 @@ __global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float
     }
 }
 
-// Smallest positive fp32 w with fl32(w / gamma) > 0.5 (gamma >= 1e-5 > 0).  The answer is
-// within a few ulps of gamma/2, so the bisection starts on +-8 ulps around it and falls
-// back to the whole positive range if that window does not bracket the answer.
-__device__ __forceinline__ float ternary_threshold(float gamma) {
-    auto above = [gamma](uint32_t bits) { return __fdiv_rn(__uint_as_float(bits), gamma) > 0.5f; };
-    const uint32_t c = __float_as_uint(__fmul_rn(0.5f, gamma));
-    uint32_t lo = c - 8u, hi = c + 8u;
-    if (above(lo) || !above(hi)) {
-        lo = 0u;            // 0 / gamma = 0      -> not above 0.5
-        hi = 0x7f7fffffu;   // FLT_MAX / gamma    -> above 0.5
-    }
-    while (hi - lo > 1u) {
-        const uint32_t mid = lo + ((hi - lo) >> 1);
-        if (above(mid)) hi = mid; else lo = mid;
-    }
-    return __uint_as_float(hi);
+__device__ __forceinline__ bool above_half(uint32_t bits, float gamma) {
+    return __fdiv_rn(__uint_as_float(bits), gamma) > 0.5f;
 }
 
-// grid-stride over 16-element groups; n % 32 == 0.
+// Smallest positive fp32 w with fl32(w / gamma) > 0.5 (gamma >= 1e-5 > 0), computed by the
+// 32 lanes of one warp.  The answer is within a few ulps of gamma/2: lane i tests the bit
+// pattern of gamma/2 - 16 + i (monotone predicate, so the ballot is 0..01..1) and the first
+// set bit is the answer; if the window does not bracket it, lane 0 bisects the whole
+// positive range.
+__device__ __forceinline__ float ternary_threshold_warp(float gamma) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t c = __float_as_uint(__fmul_rn(0.5f, gamma));
+    const uint32_t base = c - 16u;
+    const unsigned mask = __ballot_sync(0xffffffffu, above_half(base + lane, gamma));
+    uint32_t thr = base + (uint32_t)(__ffs((int)mask) - 1);
+    if (mask == 0u || (mask & 1u)) {
+        uint32_t lo = 0u, hi = 0x7f7fffffu;      // 0/gamma = 0 is not above; FLT_MAX/gamma is
+        while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            if (above_half(mid, gamma)) hi = mid; else lo = mid;
+        }
+        thr = hi;
+    }
+    return __uint_as_float(thr);
+}
+
+__device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int64_t gi, int8_t* __restrict__ wq_i8,
+                                           uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed) {
+    int q[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = (w[e] >= thr) ? 1 : ((w[e] <= -thr) ? -1 : 0);
+    if (wq_i8 != nullptr) {
+        uint32_t b[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            b[j] = (uint32_t)(q[4 * j] & 0xFF) | ((uint32_t)(q[4 * j + 1] & 0xFF) << 8) |
+                   ((uint32_t)(q[4 * j + 2] & 0xFF) << 16) | ((uint32_t)(q[4 * j + 3] & 0xFF) << 24);
+        reinterpret_cast<uint4*>(wq_i8)[gi] = make_uint4(b[0], b[1], b[2], b[3]);
+    }
+    if (wq_bf16 != nullptr) {
+        // bf16 bits of -1, 0, +1
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t lo = q[2 * j] == 0 ? 0u : (q[2 * j] > 0 ? 0x3F80u : 0xBF80u);
+            const uint32_t hi = q[2 * j + 1] == 0 ? 0u : (q[2 * j + 1] > 0 ? 0x3F80u : 0xBF80u);
+            h[j] = lo | (hi << 16);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(wq_bf16) + gi * 2;
+        dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+    if (packed != nullptr) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) word |= (q[e] > 0 ? 1u : (q[e] < 0 ? 2u : 0u)) << (2 * e);
+        reinterpret_cast<uint32_t*>(packed)[gi] = word;
+    }
+}
+
+// grid-stride over 16-element groups; n % 32 == 0.  Each thread issues the loads of its
+// first group before the block waits for gamma and the threshold.
 __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
     const float* __restrict__ W, int64_t n, const double* __restrict__ partials, int nparts,
     int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
     float* __restrict__ gamma_out) {
     __shared__ float s_thr;
+    const int64_t ngroups = n / 16;
+    const int64_t stride = (int64_t)gridDim.x * kWqThreads;
+    const float4* w4 = reinterpret_cast<const float4*>(W);
+    int64_t gi = blockIdx.x * (int64_t)kWqThreads + threadIdx.x;
+    float w[16];
+    if (gi < ngroups) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = __ldg(w4 + gi * 4 + j);
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        }
+    }
     if (threadIdx.x < 32) {
-        // fixed-order sum of the partials: lane-strided, then a fixed butterfly
-        double s = 0.0;
-        for (int i = threadIdx.x; i < nparts; i += 32) s += partials[i];
-        s = warp_sum(s);
+        // fixed-order sum of the partials: lane-strided with four accumulators, fixed butterfly
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        int i = threadIdx.x;
+        for (; i + 96 < nparts; i += 128) {
+            a0 += partials[i];
+            a1 += partials[i + 32];
+            a2 += partials[i + 64];
+            a3 += partials[i + 96];
+        }
+        for (; i < nparts; i += 32) a0 += partials[i];
+        const double sum = warp_sum((a0 + a1) + (a2 + a3));
+        const float gamma = fmaxf(static_cast<float>(sum / static_cast<double>(n)), 1e-5f);
+        const float thr = ternary_threshold_warp(gamma);
         if (threadIdx.x == 0) {
-            float mean = static_cast<float>(s / static_cast<double>(n));
-            float gamma = fmaxf(mean, 1e-5f);
-            s_thr = ternary_threshold(gamma);
+            s_thr = thr;
             if (blockIdx.x == 0) *gamma_out = gamma;
         }
     }
     __syncthreads();
     const float thr = s_thr;
-    const int64_t ngroups = n / 16;
-    const float4* w4 = reinterpret_cast<const float4*>(W);
-    for (int64_t gi = blockIdx.x * (int64_t)kWqThreads + threadIdx.x; gi < ngroups;
-         gi += (int64_t)gridDim.x * kWqThreads) {
-        float w[16];
+    if (gi < ngroups) quantise16(w, thr, gi, wq_i8, wq_bf16, packed);
+    for (gi += stride; gi < ngroups; gi += stride) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            float4 v = __ldg(w4 + gi * 4 + j);
+            const float4 v = __ldg(w4 + gi * 4 + j);
             w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
         }
-        int q[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) q[e] = (w[e] >= thr) ? 1 : ((w[e] <= -thr) ? -1 : 0);
-        if (wq_i8 != nullptr) {
-            uint32_t b[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                b[j] = (uint32_t)(uint8_t)(int8_t)q[4 * j] | ((uint32_t)(uint8_t)(int8_t)q[4 * j + 1] << 8) |
-                       ((uint32_t)(uint8_t)(int8_t)q[4 * j + 2] << 16) | ((uint32_t)(uint8_t)(int8_t)q[4 * j + 3] << 24);
-            reinterpret_cast<uint4*>(wq_i8)[gi] = make_uint4(b[0], b[1], b[2], b[3]);
-        }
-        if (wq_bf16 != nullptr) {
-            // bf16 bits of -1, 0, +1
-            uint32_t h[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t lo = q[2 * j] == 0 ? 0u : (q[2 * j] > 0 ? 0x3F80u : 0xBF80u);
-                uint32_t hi = q[2 * j + 1] == 0 ? 0u : (q[2 * j + 1] > 0 ? 0x3F80u : 0xBF80u);
-                h[j] = lo | (hi << 16);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(wq_bf16) + gi * 2;
-            dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
-        }
-        if (packed != nullptr) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                uint32_t code = q[e] > 0 ? 1u : (q[e] < 0 ? 2u : 0u);
-                word |= code << (2 * e);
-            }
-            reinterpret_cast<uint32_t*>(packed)[gi] = word;
-        }
+        quantise16(w, thr, gi, wq_i8, wq_bf16, packed);
     }
 }
 

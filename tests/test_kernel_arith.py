@@ -10,7 +10,7 @@ are IEEE round-to-nearest-even), independently of any GPU:
   every q in [-128, 127];
 * act quant: round-half-to-even of v via fl(v + 1.5*2^23) for |v| <= 128;
 * weight quant: the ternary code equals sign(w) * [|w| >= w*] with w* found by the
-  narrow bisection around gamma/2;
+  32-wide window search around gamma/2;
 * decode GEMV: sum_k dec(c_k) x_k == sum_j dp4a(lo_j, x_j) - dp4a(hi_j, x_j) with the
   interleaved activation words.
 """
@@ -73,13 +73,17 @@ def test_magic_constant_rounds_half_to_even():
     assert np.array_equal((t - magic).astype(np.float32), np.rint(v))
 
 
-def _threshold_narrow(gamma: np.float32) -> np.float32:
+def _threshold_window(gamma: np.float32) -> np.float32:
+    """The kernel's search: 32 lanes test the bit patterns gamma/2 - 16 + lane; the first
+    pattern above 0.5 is the threshold unless the window fails to bracket it, in which case
+    a bisection over the whole positive range runs."""
     def above(bits):
         return np.float32(np.uint32(bits).view(np.float32)) / gamma > np.float32(0.5)
     c = int(np.float32(np.float32(0.5) * gamma).view(np.uint32))
-    lo, hi = c - 8, c + 8
-    if above(lo) or not above(hi):
-        lo, hi = 0, 0x7F7FFFFF
+    mask = [above(c - 16 + lane) for lane in range(32)]
+    if any(mask) and not mask[0]:
+        return np.uint32(c - 16 + mask.index(True)).view(np.float32)
+    lo, hi = 0, 0x7F7FFFFF
     while hi - lo > 1:
         mid = lo + ((hi - lo) >> 1)
         if above(mid):
@@ -93,7 +97,7 @@ def test_ternary_threshold_equals_round_clamp():
     rng = np.random.default_rng(2)
     for gamma in [np.float32(1e-5), np.float32(0.0159), np.float32(0.265625), np.float32(3.7)] + \
             [np.float32(g) for g in 10.0 ** rng.uniform(-5, 2, 40)]:
-        thr = _threshold_narrow(gamma)
+        thr = _threshold_window(gamma)
         # dense neighbourhood of the threshold and random weights
         b = int(thr.view(np.uint32))
         near = np.arange(b - 64, b + 64, dtype=np.uint32).view(np.float32)
