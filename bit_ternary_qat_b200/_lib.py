@@ -37,6 +37,7 @@ SIGNATURES = {
     "bl_set_wait_limit_ns": (None, [U64]),
     "bl_launch_count": (U64, []),
     "bitlinear_quant_weight": (INT, [P, I64, I64, P, P, P, P, P, SZ, P]),
+    "bitlinear_quant_weight_noalloc": (INT, [P, I64, I64, P, P, P, P, P]),
     "bitlinear_act_quant": (INT, [P, INT, I64, I64, INT, P, F, P, P, P, P, P]),
     "bitlinear_linear": (INT, [P, P, I64, I64, P, P, I64, P, INT, P, P]),
     "bitlinear_forward": (INT, [P, INT, I64, I64, P, F, P, P, I64, P, P, P, P, P, P, P]),

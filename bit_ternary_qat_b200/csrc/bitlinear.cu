@@ -22,6 +22,13 @@
 #include "rmsnorm_bwd.cuh"
 #include "gemv.cuh"
 
+// Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
+// file-scope device array instead of a caller workspace.  Every device that loads the
+// library holds it until the process exits.  Host code must not pass the symbol itself to
+// a kernel (on the host it names a host-side shadow, not device memory): the device
+// address is looked up with cudaGetSymbolAddress once per device and passed instead.
+static __device__ __align__(256) double g_quant_scratch[bl::kWqMaxPartials];
+
 namespace {
 
 thread_local std::string g_last_error = "no error";
@@ -583,6 +590,51 @@ bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, in
     else BL_GEMV_CASE(2)
 #undef BL_GEMV_CASE
     return launched("ternary_gemv");
+}
+
+bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
+                                         uint8_t* Wpacked, float* gamma, void* stream) {
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", false));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_dims(1, N, K));
+    const int64_t n = N * K;
+    const int parts = bl::wq_num_partials(n);
+    BL_REQUIRE(parts <= bl::kWqMaxPartials, BL_ERR_UNSUPPORTED_SHAPE,
+               "the built-in scratch holds %d partial sums, this weight needs %d", bl::kWqMaxPartials, parts);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    // set-up, once per device: the device address of the scratch array
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev_id = 0;
+    cudaError_t e = cudaGetDevice(&dev_id);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (addr[dev_id] == nullptr) {
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_quant_scratch);
+            if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+            addr[dev_id] = p;
+        }
+        scratch = addr[dev_id];
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    double* partials = static_cast<double*>(scratch);
+    // pass 1 writes every partial that pass 2 reads, so nothing in the scratch needs clearing
+    bl::absmean_partial_kernel<<<parts, bl::kWqThreads, 0, st>>>(W, n, partials);
+    BL_TRY(launched("absmean_partial"));
+    const int64_t groups = n / 16;
+    int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
+    const int64_t cap = (int64_t)dev.sms * 4;
+    if (blocks > cap) blocks = cap;
+    bl::ternary_quant_kernel<<<(unsigned)blocks, bl::kWqThreads, 0, st>>>(W, n, partials, parts, Wq_i8, Wq_bf16,
+                                                                          Wpacked, gamma);
+    return launched("ternary_quant");
 }
 
 bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

@@ -69,6 +69,17 @@ def bitlinear_quant_weight(W: torch.Tensor, want_i8: bool = True, want_bf16: boo
     return o
 
 
+def bitlinear_quant_weight_noalloc(W: torch.Tensor, gamma: torch.Tensor, wq_i8: Optional[torch.Tensor] = None,
+                                   wq_bf16: Optional[torch.Tensor] = None, packed: Optional[torch.Tensor] = None):
+    """bitlinear_quant_weight without a workspace: the caller passes every output and the
+    library uses its built-in scratch (see include/bitlinear.h)."""
+    _cuda(W, "W", torch.float32)
+    N, K = W.shape
+    _lib.call("bitlinear_quant_weight_noalloc", W.data_ptr(), N, K, _ptr(wq_i8), _ptr(wq_bf16), _ptr(packed),
+              gamma.data_ptr(), _stream(W.device))
+    return gamma
+
+
 def bitlinear_act_quant(X: torch.Tensor, apply_rmsnorm: bool = True, g: Optional[torch.Tensor] = None,
                         eps: float = 1e-6, want_xdq: bool = True, out=None):
     """Returns dict(xq [T,K] i8, sx [T] f32, rinv [T] f32 or None, xdq [T,K] X.dtype or None)."""

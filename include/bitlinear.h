@@ -106,6 +106,30 @@ BL_API bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K,
                                  float* gamma, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------
+ * bitlinear_quant_weight without a workspace.  (Not from the pages: they have no
+ * counterpart; it exists for callers.)  Some callers cannot allocate device memory at
+ * all -- for example a serving process whose device memory is handed out by another
+ * allocator that owns the whole pool -- so they cannot pass the workspace that
+ * bitlinear_quant_weight needs for its per-block partial sums of |W|.  This variant
+ * computes exactly the same gamma and codes (bit-identical outputs), but keeps those
+ * partial sums in a scratch array compiled into the library: 1184 fp64 values
+ * (9,472 bytes) per device, held by every GPU that loads the library until the process
+ * exits.  It allocates nothing and calls no allocating routine.
+ *   - Sizes: any N x K accepted by bitlinear_quant_weight fits (the number of partial
+ *     sums is capped at 1184); a weight that needed more would be rejected with
+ *     BL_ERR_UNSUPPORTED_SHAPE.
+ *   - Set-up: the first call on each device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.
+ *   - Sharing: all calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (every partial a call reads was
+ *     written by that call), but calls that overlap on the GPU (for example on two
+ *     streams) race on it: serialise them. */
+BL_API bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K,
+                                         int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                         float* gamma, void* stream);
+
+/* ------------------------------------------------------------------------------
  * Activation quantiser with optional RMSNorm in front (P3 §3.1 RMSNorm before
  * activation_quant; P3 §2.2 activation_quant; P2 per-token absmax 8-bit).
  *   r_t   = 1 / sqrt( mean_k X[t,k]^2 + eps )        (fp64 sum; only if apply_rmsnorm)
