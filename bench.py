@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
     return ap.parse_args()
 
 
@@ -220,6 +221,12 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.only_gemv:
+        blbuild.build()
+        bl.load()
+        flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        print(json.dumps({"decode_gemv": gemv_measure(bl, torch, dev, flush, peaks())}), flush=True)
+        return
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     if rank == 0:
@@ -427,9 +434,9 @@ def main():
         peak, peak_note = pk["bf16_sust"], f"bf16 sustained ({pk['src']})"
     else:
         peak, peak_note = 2.0 * pk["bf16_sust"], f"int8 = 2 x bf16 sustained ({pk['src']}; nominal 4.5/2.25 ratio)"
-    kernel_names = {"linear_i8": "tc_gemm_kernel<int8,K,K,256,linear>",
-                    "grad_input": "tc_gemm_kernel<bf16,K,MN,256,scale_f32>",
-                    "grad_weight": "tc_gemm_kernel<bf16,MN,MN,256,f32>"}
+    kernel_names = {"linear_i8": "tc_gemm2_kernel<int8,K,K,linear> (2-SM, 256x256)",
+                    "grad_input": "tc_gemm2_kernel<bf16,K,MN,scale_f32> (2-SM, 256x256)",
+                    "grad_weight": "tc_gemm2_kernel<bf16,MN,MN,f32> (2-SM, 256x256)"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": ncu_traffic(dom), "kernel": kernel_names[dom], "peak_kind": peak_note,
                 "launch_ms": dom_ms}

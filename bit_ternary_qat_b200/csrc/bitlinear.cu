@@ -195,6 +195,48 @@ bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensor
     return launched("tc_gemm");
 }
 
+// 2-SM variant: clusters of two CTAs, 256 x 256 tiles.  The grid is as many clusters as
+// fit on the device at once (queried once per device and kernel), at most one per tile.
+template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
+bl_status launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td, bl::TcGemmArgs a,
+                     cudaStream_t st, const DeviceInfo& dev) {
+    auto kern = bl::tc_gemm2_kernel<kInt8, kAMN, kBMN, kEpi>;
+    const size_t smem = bl::tc2_smem_bytes();
+    BL_REQUIRE((int)smem <= dev.max_smem_optin, BL_ERR_DEVICE, "GEMM needs %zu bytes of shared memory", smem);
+    static std::atomic<int> max_clusters[64] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (dev_id < 0 || dev_id >= 64) return fail(BL_ERR_DEVICE, "device ordinal %d out of range", dev_id);
+    int mc = max_clusters[dev_id].load();
+    if (mc == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)(dev.sms / 2));
+        cfg.blockDim = dim3(bl::kTcThreads);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s", cudaGetErrorString(e));
+        if (n < 1) return fail(BL_ERR_DEVICE, "no 2-CTA cluster of the GEMM fits on the device");
+        mc = n;
+        max_clusters[dev_id].store(mc);
+    }
+    a.m_tiles = (a.M + 255) / 256;
+    a.n_tiles = (a.N + 255) / 256;
+    const int kb_elems = kInt8 ? 128 : 64;
+    a.k_blocks = (a.K + kb_elems - 1) / kb_elems;
+    a.wait_ns = g_wait_ns.load();
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int clusters = tiles < mc ? tiles : mc;
+    kern<<<2 * clusters, bl::kTcThreads, smem, st>>>(ta, tb, td, a);
+    return launched("tc_gemm2");
+}
+
+// The 2-SM kernel computes 256-row tiles; for a single 128-row tile the 1-SM kernel wastes
+// nothing and needs no partner CTA.
+inline bool use_2sm(int64_t M) { return M > bl::kTcBM; }
+
 // ------------------------------------------------------------------------------------
 // pieces shared by the entry points (validation already done by the caller)
 // ------------------------------------------------------------------------------------
@@ -232,16 +274,19 @@ bl_status run_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int 
 bl_status run_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq, const float* gamma,
                      int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
     CUtensorMap ta, tb, td;
+    const bool two = use_2sm(T);
     BL_TRY(make_tmap(&ta, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, 128));
-    BL_TRY(make_tmap(&tb, Wq, kTmU8, (uint64_t)K, (uint64_t)N, 128, kBN));
+    BL_TRY(make_tmap(&tb, Wq, kTmU8, (uint64_t)K, (uint64_t)N, 128, two ? 128 : kBN));
     bl::TcGemmArgs a{};
     a.M = (int)T; a.N = (int)N; a.K = (int)K;
     a.acc_out = acc; a.row_scale = sx; a.gamma = gamma;
     if (y_dt == BL_BF16) {
         BL_TRY(make_tmap(&td, Y, kTmBf16, (uint64_t)N, (uint64_t)T, 64, 32));
+        if (two) return launch_tc2<true, false, false, bl::kEpiLinearBf16>(ta, tb, td, a, st, dev);
         return launch_tc<true, false, false, bl::kEpiLinearBf16>(ta, tb, td, a, st, dev);
     }
     BL_TRY(make_tmap(&td, Y, kTmF32, (uint64_t)N, (uint64_t)T, 32, 32));
+    if (two) return launch_tc2<true, false, false, bl::kEpiLinearF32>(ta, tb, td, a, st, dev);
     return launch_tc<true, false, false, bl::kEpiLinearF32>(ta, tb, td, a, st, dev);
 }
 
@@ -255,6 +300,7 @@ bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf
         bl::TcGemmArgs a{};
         a.M = (int)T; a.N = (int)K; a.K = (int)N;
         a.gamma = gamma;
+        if (use_2sm(T)) return launch_tc2<false, false, true, bl::kEpiScaleF32>(ta, tb, td, a, st, dev);
         return launch_tc<false, false, true, bl::kEpiScaleF32>(ta, tb, td, a, st, dev);
     }
     // fp32 layer: CUDA-core fp32 contraction, C[t,k] = gamma * sum_n dY[t,n] W_q[n,k]
@@ -274,6 +320,7 @@ bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int
         BL_TRY(make_tmap(&td, dW, kTmF32, (uint64_t)K, (uint64_t)N, 32, 32));
         bl::TcGemmArgs a{};
         a.M = (int)N; a.N = (int)K; a.K = (int)T;
+        if (use_2sm(N)) return launch_tc2<false, true, true, bl::kEpiF32>(ta, tb, td, a, st, dev);
         return launch_tc<false, true, true, bl::kEpiF32>(ta, tb, td, a, st, dev);
     }
     dim3 grid((unsigned)((K + 63) / 64), (unsigned)((N + 63) / 64));
@@ -326,6 +373,29 @@ bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const f
 
 // Row kernels keep a whole row in registers: d_in is limited to 16384.
 constexpr int64_t kMaxRowK = 16384;
+
+template <int NTILES, int WB, int S>
+bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
+                      const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
+    CUtensorMap tw;
+    BL_TRY(make_tmap(&tw, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, 16));
+    const size_t smem = 1024 + bl::gemv_ring_bytes<WB, S>() + (size_t)B * (size_t)(K / 16 + 1) * 16 +
+                        sizeof(uint64_t) * WB * S;
+    BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
+               "GEMV needs %zu bytes of shared memory for B = %lld, K = %lld; at most %d fit", smem, (long long)B,
+               (long long)K, dev.max_smem_optin);
+    auto kern = bl::ternary_gemv_tma_kernel<NTILES, WB, S>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WB * 32, smem);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t need = (N / 16 + WB - 1) / WB;
+    int64_t grid = (int64_t)dev.sms * per_sm;
+    if (grid > need) grid = need;
+    kern<<<(unsigned)grid, WB * 32, smem, st>>>(tw, gamma, (int)N, (int)K, xq, sx, (int)B, y, acc, g_wait_ns.load());
+    return launched("ternary_gemv");
+}
 
 }  // namespace
 
@@ -553,43 +623,15 @@ bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, in
     BL_TRY(check_ptr(y, "y", true));
     BL_TRY(check_ptr(acc, "acc", false));
     BL_TRY(check_dims(1, N, K));
+    BL_REQUIRE(K % 64 == 0, BL_ERR_UNSUPPORTED_SHAPE,
+               "the GEMV reads packed rows with TMA: K must be a multiple of 64 (16-byte rows), got %lld", (long long)K);
     BL_REQUIRE(B >= 1 && B <= 16, BL_ERR_UNSUPPORTED_SHAPE, "batch must be in [1, 16], got %lld", (long long)B);
     BL_REQUIRE(K <= 65536, BL_ERR_UNSUPPORTED_SHAPE, "K must be <= 65536 for the GEMV, got %lld", (long long)K);
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int ntiles = B <= 8 ? 1 : 2;
-    const size_t smem = (size_t)(8 * ntiles) * (size_t)(K / 16 + 1) * 16;   // padded activation words
-    BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
-               "GEMV stages %zu activation bytes in shared memory; at most %d fit (reduce B or K)", smem,
-               dev.max_smem_optin);
-    const int64_t row_groups = N / 16;
-    // warps per row group: enough that each warp streams about one load batch per row group
-    const int64_t nsc = (K / 16 + 7) / 8;
-    const int64_t batch = ntiles == 1 ? 8 : 4;
-    int ks = 1;
-    while (ks < bl::kGemvMmaWarps && (nsc + ks - 1) / ks > batch) ks *= 2;
-    // few row groups: split K further so that every SM gets work
-    while (ks < bl::kGemvMmaWarps && row_groups * ks < (int64_t)dev.sms * bl::kGemvMmaWarps) ks *= 2;
-    const int64_t rs = bl::kGemvMmaWarps / ks;
-    const int64_t need = (row_groups + rs - 1) / rs;
-#define BL_GEMV_CASE(NTV)                                                                                          \
-    {                                                                                                              \
-        auto kern = bl::ternary_gemv_mma_kernel<NTV>;                                                              \
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);        \
-        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));         \
-        int per_sm = 0;                                                                                            \
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, bl::kGemvMmaThreads, smem);                   \
-        if (per_sm < 1) per_sm = 1;                                                                                \
-        int64_t grid = (int64_t)dev.sms * per_sm;                                                                  \
-        if (grid > need) grid = need;                                                                              \
-        kern<<<(unsigned)grid, bl::kGemvMmaThreads, smem, st>>>(Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, ks, \
-                                                                y, acc);                                           \
-    }
-    if (ntiles == 1) BL_GEMV_CASE(1)
-    else BL_GEMV_CASE(2)
-#undef BL_GEMV_CASE
-    return launched("ternary_gemv");
+    if (B <= 8) return launch_gemv<1, 8, 4>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
+    return launch_gemv<2, 16, 2>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
 }
 
 bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,

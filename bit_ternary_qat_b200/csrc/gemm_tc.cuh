@@ -321,4 +321,277 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
+// ====================================================================================
+// 2-SM variant: a cluster of two CTAs computes a 256 x 256 tile with tcgen05.mma
+// .cta_group::2 (M = 256, N = 256).  CTA r of the pair loads rows [128 r, 128 r + 128) of
+// the tile's A and of the tile's B (its half of the N columns) into its own shared memory;
+// the leader (r = 0) issues the MMAs, which read both CTAs' shared memory and write the
+// accumulators of rows [128 r, 128 r + 128) into CTA r's TMEM.  Per SM a pipeline stage is
+// 16 KB of A + 16 KB of B for the same MMA work that costs 16 + 32 KB in the 1-SM kernel,
+// so six stages fit and 1.5x more MMA work is in flight per byte of shared memory.
+// Barrier protocol:
+//   full[s]   leader only: the leader's producer posts the pair's bytes (expect_tx); both
+//             CTAs' TMA loads complete bytes on it (2-SM TMA form, no multicast);
+//   empty[s]  each CTA: arrived by the leader's tcgen05.commit multicast to both CTAs;
+//   tfull[b]  each CTA: arrived by the leader's commit multicast after a tile's last MMA;
+//   tempty[b] leader only: 4 epilogue warps of each CTA arrive when they drained TMEM.
+// Cross-CTA barrier addresses come from mapa.  Cluster barriers only at set-up and
+// teardown; every other wait is bounded.
+// ====================================================================================
+constexpr int kTc2Stages = 6;
+constexpr int kTc2HalfBytes = 128 * 128;   // one operand half per stage per CTA: 128 rows x 128 bytes
+
+__host__ __device__ constexpr size_t tc2_smem_bytes() {
+    return 1024 + (size_t)kTc2Stages * 2 * kTc2HalfBytes + kEpiBytes + (2 * kTc2Stages + 4) * sizeof(uint64_t) + 16;
+}
+
+template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+    tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmD, const TcGemmArgs args) {
+    static_assert(!kInt8 || (!kAMN && !kBMN), "int8 operands are K-major here");
+    constexpr int kBN = 256;                              // pair tile columns
+    constexpr uint32_t kStageTxPair = 2u * 2u * kTc2HalfBytes;
+    constexpr int kKbElems = kInt8 ? 128 : 64;
+    constexpr int kInstrK = 4;
+    constexpr uint32_t kIdesc = umma_idesc(kInt8, kAMN, kBMN, 256, kBN);
+    constexpr uint32_t kTmemCols = 2 * kBN;
+    constexpr int kChunkCols = epi_chunk_cols(kEpi);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kTc2Stages * kTc2HalfBytes;
+    uint8_t* sE = sB + kTc2Stages * kTc2HalfBytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + kEpiBytes);
+    uint64_t* empty = full + kTc2Stages;
+    uint64_t* tfull = empty + kTc2Stages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTc2Stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmD);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int num_tiles = args.m_tiles * args.n_tiles;   // m_tiles counts 256-row pair tiles
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const uint64_t lim = args.wait_ns;
+
+    if (warp == 0) {
+        // ----------------------------------------------------------------- producer (both CTAs)
+        if (elect_one()) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const int mb = tile % args.m_tiles;
+                const int nb = tile / args.m_tiles;
+                const int arow = mb * 256 + static_cast<int>(rank) * 128;
+                const int brow = nb * kBN + static_cast<int>(rank) * 128;
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&full[s], kStageTxPair);
+                    const uint32_t fbar = mapa_shared(smem_u32(&full[s]), 0);
+                    uint8_t* a_dst = sA + s * kTc2HalfBytes;
+                    uint8_t* b_dst = sB + s * kTc2HalfBytes;
+                    if constexpr (!kAMN) {
+                        tma_load_2d_pair(a_dst, &tmA, fbar, kb * kKbElems, arow);
+                    } else {
+                        tma_load_2d_pair(a_dst, &tmA, fbar, arow, kb * 64);
+                        tma_load_2d_pair(a_dst + 8192, &tmA, fbar, arow + 64, kb * 64);
+                    }
+                    if constexpr (!kBMN) {
+                        tma_load_2d_pair(b_dst, &tmB, fbar, kb * kKbElems, brow);
+                    } else {
+                        tma_load_2d_pair(b_dst, &tmB, fbar, brow, kb * 64);
+                        tma_load_2d_pair(b_dst + 8192, &tmB, fbar, brow + 64, kb * 64);
+                    }
+                    if (++s == kTc2Stages) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok && leader) {
+                // the leader's full barriers count both CTAs' loads: wait (briefly) for them
+                for (int i = 0; i < kTc2Stages; ++i) {
+                    int ss = (s - 1 - i + 2 * kTc2Stages) % kTc2Stages;
+                    uint32_t pp = (s - 1 - i < 0) ? (ph ^ 1u) : ph;
+                    mbar_wait(&full[ss], pp, 100000000ull, nullptr);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ----------------------------------------------------------------- MMA issuer (leader)
+        if (leader && elect_one()) {
+            int s = 0;
+            uint32_t ph = 0;
+            int tcount = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++tcount) {
+                const int b = tcount & 1;
+                const uint32_t tph = (tcount >> 1) & 1;
+                if (!mbar_wait(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!mbar_wait(&full[s], ph, lim, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + s * kTc2HalfBytes);
+                    const uint32_t b_base = smem_u32(sB + s * kTc2HalfBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kInstrK; ++kk) {
+                        uint64_t adesc, bdesc;
+                        if constexpr (!kAMN) adesc = umma_desc_sw128(a_base + kk * 32, 16, 1024);
+                        else adesc = umma_desc_sw128(a_base + kk * 2048, 8192, 1024);
+                        if constexpr (!kBMN) bdesc = umma_desc_sw128(b_base + kk * 32, 16, 1024);
+                        else bdesc = umma_desc_sw128(b_base + kk * 2048, 8192, 1024);
+                        tc_mma_pair<kInt8>(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair(&empty[s], 0x3);
+                    if (++s == kTc2Stages) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair(&tfull[b], 0x3);
+            }
+            if (!ok) {
+                tc_commit_pair(&tfull[tcount & 1], 0x3);
+                mbar_wait(&tfull[tcount & 1], ((tcount >> 1) & 1), 100000000ull, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------------------- epilogue (both CTAs)
+        const int quad = warp & 3;
+        uint8_t* ebuf = sE + (warp - 2) * 2 * kEpiBufBytes;
+        int buf = 0;
+        int tcount = 0;
+        float gm = 1.0f;
+        if constexpr (kEpi != kEpiF32) gm = __ldg(args.gamma);
+        for (int tile = pair; tile < num_tiles; tile += npairs, ++tcount) {
+            const int b = tcount & 1;
+            const uint32_t tph = (tcount >> 1) & 1;
+            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            tc_fence_after();
+            const int mb = tile % args.m_tiles;
+            const int nb = tile / args.m_tiles;
+            const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
+            const int row = row0 + lane;
+            const bool row_ok = row < args.M;
+            float cs = 1.0f;
+            if constexpr (epi_is_linear(kEpi)) cs = row_ok ? __fdiv_rn(gm, __ldg(args.row_scale + row)) : 0.0f;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                   static_cast<uint32_t>(b * kBN);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kBN; c0 += kChunkCols) {
+                const int col0 = nb * kBN + c0;
+                if (col0 >= args.N) break;                     // warp-uniform
+                uint32_t ra[32], rb[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + c0, ra);
+                if constexpr (kChunkCols == 64) {
+                    tmem_ld_32x32b_x32(t_row + c0 + 32, rb);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) rb[i] = 0u;
+                }
+                tmem_ld_wait();
+                auto r = [&](int i) -> uint32_t { return i < 32 ? ra[i] : rb[i - 32]; };
+                uint4 v[8];
+                if constexpr (kEpi == kEpiLinearBf16) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e))), cs);
+                            const float hi = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e + 1))), cs);
+                            w[e] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
+                        }
+                        v[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float f[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t raw = r(4 * j + e);
+                            if constexpr (kEpi == kEpiLinearF32)
+                                f[e] = __fmul_rn(static_cast<float>(static_cast<int32_t>(raw)), cs);
+                            else if constexpr (kEpi == kEpiScaleF32)
+                                f[e] = __fmul_rn(gm, __uint_as_float(raw));
+                            else
+                                f[e] = __uint_as_float(raw);
+                        }
+                        v[j] = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                          __float_as_uint(f[3]));
+                    }
+                }
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint8_t* sb = ebuf + buf * kEpiBufBytes;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4*>(sb + lane * 128 + ((j ^ (lane & 7)) << 4)) = v[j];
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmD, sb, col0, row0);
+                    bulk_commit_group();
+                }
+                buf ^= 1;
+                if constexpr (epi_is_linear(kEpi)) {
+                    if (args.acc_out != nullptr && row_ok) {
+                        int32_t* dst = args.acc_out + static_cast<int64_t>(row) * args.N + col0;
+#pragma unroll
+                        for (int j = 0; j < kChunkCols / 4; ++j)
+                            if (col0 + 4 * j < args.N)
+                                reinterpret_cast<int4*>(dst)[j] = make_int4((int)r(4 * j), (int)r(4 * j + 1),
+                                                                            (int)r(4 * j + 2), (int)r(4 * j + 3));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[b]), 0));
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs done with TMEM, with their barriers and with remote arrivals
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
 }  // namespace bl

@@ -224,7 +224,8 @@ BL_API bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t
  *   acc[b,n] = sum_k decode(Wpacked[n,k]) * xq[b,k]   exact int32
  *   y[b,n]   = acc[b,n] * (gamma / sx[b])              fp32
  * Wpacked uint8 [N x K/4]; gamma fp32 [1]; xq int8 [B x K]; sx fp32 [B];
- * y fp32 [B x N]; acc int32 [B x N] optional.  1 <= B <= 16, K <= 65536. */
+ * y fp32 [B x N]; acc int32 [B x N] optional.  1 <= B <= 16, K <= 65536, and K % 64 == 0
+ * (packed rows are read with TMA, which needs 16-byte aligned rows). */
 BL_API bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K,
                        const int8_t* xq, const float* sx, int64_t B,
                        float* y, int32_t* acc, void* stream);

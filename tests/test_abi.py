@@ -101,6 +101,7 @@ def test_backward_and_gemv_validation(L):
     assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 64, FAKE, FAKE, 17, FAKE, None, None) == 2
     assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 1 << 17, FAKE, FAKE, 1, FAKE, None, None) == 2
     assert _lib.status("ternary_pack", FAKE, 16, 33, FAKE, None) == 2
+    assert _lib.status("ternary_gemv", FAKE, FAKE, 32, 96, FAKE, FAKE, 1, FAKE, None, None) == 2   # K % 64
     assert _lib.status("bl_selftest_bounded_wait", 0, None) == 1
 
 

@@ -259,7 +259,7 @@ def test_square_workload_full_size(bl):
 # decode GEMV over packed weights
 # ------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K", [(48, 64), (400, 160), (1024, 8192), (272, 4096)])
+@pytest.mark.parametrize("N,K", [(48, 64), (400, 192), (1024, 8192), (272, 4096), (160, 704)])
 @pytest.mark.parametrize("B", [1, 2, 4, 5, 16])
 def test_gemv_parity(bl, N, K, B):
     W, x = synth.decode_inputs(B, N, K, seed=N + K + B)
