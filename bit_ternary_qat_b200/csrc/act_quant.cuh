@@ -5,9 +5,10 @@
 // round, clamp to [-128, 127], dequantised value forwarded through the STE), and
 // P2 ("BitNet 三元权重量化训练工程…") per-token 8-bit absmax.
 //
-// One block per token row; each thread loads its 16-byte vectors of the row once into
-// registers (the row is read from HBM exactly once) and the three steps -- sum of
-// squares, absmax, quantise -- run from registers with two block reductions in between.
+// One block per R adjacent token rows; each thread loads its 16-byte vectors of the rows
+// once into registers (every row is read from HBM exactly once) and the three steps -- sum
+// of squares, absmax, quantise -- run from registers with two block reductions in between
+// (each reduction covers the R rows at once).
 // Memory-bound: X is read once, X_q / X_dq / s / r are written once.
 //
 // Exactness (the codes must equal the fp32 oracle's bit for bit):
@@ -56,52 +57,192 @@ __device__ __forceinline__ float div_by_scale(float q, float s, float c) {
     return __fmaf_rn(e1, c, y1);
 }
 
-template <int NT>
-__device__ __forceinline__ double block_sum_f64(double v, double* red) {
-    v = warp_sum(v);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    double s = 0.0;
+// R independent block sums / maxima with one barrier each (fixed order: per thread, then a
+// fixed butterfly, then the warps in order).
+template <int NT, int R>
+__device__ __forceinline__ void block_sum_f64(double (&v)[R], double (*red)[NT / 32]) {
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) s += red[w];
-    return s;
+    for (int q = 0; q < R; ++q) {
+        const double w = warp_sum(v[q]);
+        if ((threadIdx.x & 31) == 0) red[q][threadIdx.x >> 5] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        double s = 0.0;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) s += red[q][w];
+        v[q] = s;
+    }
 }
 
-template <int NT>
-__device__ __forceinline__ float block_max_f32(float v, float* red) {
-    v = warp_max(v);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    float m = red[0];
+template <int NT, int R>
+__device__ __forceinline__ void block_max_f32(float (&v)[R], float (*red)[NT / 32]) {
 #pragma unroll
-    for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, red[w]);
-    return m;
+    for (int q = 0; q < R; ++q) {
+        const float w = warp_max(v[q]);
+        if ((threadIdx.x & 31) == 0) red[q][threadIdx.x >> 5] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        float m = red[q][0];
+#pragma unroll
+        for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, red[q][w]);
+        v[q] = m;
+    }
 }
 
-// grid = T blocks, block = NT threads; thread i owns vectors i + j*NT, j < VPT.
-template <bool kBf16, int NT, int VPT>
-__global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ X, int K, int apply_norm,
+// grid = ceil(T / R) blocks, block = NT threads; block b quantises rows R*b .. R*b + R - 1
+// (adjacent rows: one contiguous span), thread i owns vectors i + j*NT of each row, j < VPT.
+// All R rows are loaded before the first reduction, so R rows of loads are in flight per block.
+template <bool kBf16, int NT, int VPT, int R>
+__global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
                                                        const float* __restrict__ g, float eps,
                                                        int8_t* __restrict__ Xq, float* __restrict__ sx,
                                                        float* __restrict__ rinv, void* __restrict__ Xdq) {
     using V = ActVec<kBf16>;
     constexpr int E = V::kElems;
-    __shared__ double red_d[NT / 32];
-    __shared__ float red_f[NT / 32];
+    __shared__ double red_d[R][NT / 32];
+    __shared__ float red_f[R][NT / 32];
+    pdl_trigger_and_wait();
 
-    const int64_t t = blockIdx.x;
+    const int nvec = K / E;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * R;
+
+    // the rows, widened to fp32, in registers (read from HBM once)
+    float x[R][VPT][E];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        const bool live = t0 + q < T;
+        const uint4* xrow = reinterpret_cast<const uint4*>(X) + (t0 + q) * static_cast<int64_t>(nvec);
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+            const uint4 raw = (live && v < nvec) ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int e = 0; e < E; ++e) x[q][j][e] = V::elem(raw, e);
+        }
+    }
+
+    // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order
+    float r[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) r[q] = 1.0f;
+    if (apply_norm) {
+        double ss[R];
+#pragma unroll
+        for (int q = 0; q < R; ++q) {
+            ss[q] = 0.0;
+#pragma unroll
+            for (int j = 0; j < VPT; ++j)
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const double xd = static_cast<double>(x[q][j][e]);
+                    ss[q] = fma(xd, xd, ss[q]);
+                }
+        }
+        block_sum_f64<NT, R>(ss, red_d);
+#pragma unroll
+        for (int q = 0; q < R; ++q)
+            r[q] = static_cast<float>(1.0 / sqrt(ss[q] / static_cast<double>(K) + static_cast<double>(eps)));
+    }
+
+    // x_hat = fl(fl(x * r) * g) (kept in place of x) and its absmax
+    float m[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        m[q] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                float h = x[q][j][e];
+                if (apply_norm) {
+                    h = __fmul_rn(h, r[q]);
+                    if (g != nullptr && v < nvec) h = __fmul_rn(h, __ldg(g + v * E + e));
+                }
+                x[q][j][e] = h;
+                m[q] = fmaxf(m[q], fabsf(h));
+            }
+        }
+    }
+    block_max_f32<NT, R>(m, red_f);
+
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        const int64_t t = t0 + q;
+        if (t >= T) break;
+        const float s = __fdiv_rn(127.0f, fmaxf(m[q], 1e-5f));
+        const float c = __frcp_rn(s);
+        if (threadIdx.x == 0) {
+            sx[t] = s;
+            if (apply_norm) rinv[t] = r[q];
+        }
+        const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
+        // codes and dequantised values.  |x_hat * s| <= 127 * (1 + 2^-23) for finite inputs,
+        // so rint(x_hat * s) is in [-127, 127]; the integer clamp is kept for robustness.
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+            if (v >= nvec) continue;
+            uint32_t qb[E];
+            float dq[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const float tq = __fadd_rn(__fmul_rn(x[q][j][e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
+                const int qi = max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
+                qb[e] = static_cast<uint32_t>(qi) & 0xFFu;
+                dq[e] = div_by_scale(__fsub_rn(tq, kRoundMagic), s, c);
+            }
+            if constexpr (kBf16) {
+                uint2 packed;
+                packed.x = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
+                packed.y = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
+                reinterpret_cast<uint2*>(Xq)[row_vec0 + v] = packed;
+                if (Xdq != nullptr) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dq[2 * i], dq[2 * i + 1]);
+                        o[i] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
+                    reinterpret_cast<uint4*>(Xdq)[row_vec0 + v] = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            } else {
+                reinterpret_cast<uint32_t*>(Xq)[row_vec0 + v] = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
+                if (Xdq != nullptr)
+                    reinterpret_cast<float4*>(Xdq)[row_vec0 + v] = make_float4(dq[0], dq[1], dq[2], dq[3]);
+            }
+        }
+    }
+}
+
+// Short rows (at most 32 * VPL 16-byte vectors): one warp per row, 8 rows per block, no
+// shared memory and no block barrier -- both reductions are warp butterflies (fixed order).
+// Each lane keeps its VPL raw vectors of the row in registers and widens them on use, so a
+// warp has the whole row in flight at once and many rows fit on an SM.
+template <bool kBf16, int VPL>
+__global__ void __launch_bounds__(256, 4) act_quant_warp_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
+                                                             const float* __restrict__ g, float eps,
+                                                             int8_t* __restrict__ Xq, float* __restrict__ sx,
+                                                             float* __restrict__ rinv, void* __restrict__ Xdq) {
+    using V = ActVec<kBf16>;
+    constexpr int E = V::kElems;
+    pdl_trigger_and_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
     const int nvec = K / E;
     const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
     const uint4* xrow = reinterpret_cast<const uint4*>(X) + row_vec0;
 
-    // the row, widened to fp32, in registers (read from HBM once)
-    float x[VPT][E];
+    uint4 raw[VPL];
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-        const int v = threadIdx.x + j * NT;
-        const uint4 raw = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int e = 0; e < E; ++e) x[j][e] = V::elem(raw, e);
+    for (int j = 0; j < VPL; ++j) {
+        const int v = lane + 32 * j;
+        raw[j] = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
     }
 
     // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order
@@ -109,51 +250,62 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
     if (apply_norm) {
         double ss = 0.0;
 #pragma unroll
-        for (int j = 0; j < VPT; ++j)
+        for (int j = 0; j < VPL; ++j)
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const double xd = static_cast<double>(x[j][e]);
+                const double xd = static_cast<double>(V::elem(raw[j], e));
                 ss = fma(xd, xd, ss);
             }
-        ss = block_sum_f64<NT>(ss, red_d);
+        ss = warp_sum(ss);
         r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(eps)));
     }
-
-    // x_hat = fl(fl(x * r) * g) (kept in place of x) and its absmax
-    float m = 0.0f;
+    // x_hat = fl(fl(x * r) * g) of the E elements of vector j (recomputed where needed)
+    auto xhat = [&](int j, float (&h)[E]) {
+        const int v = lane + 32 * j;
+        float gk[E];
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-        const int v = threadIdx.x + j * NT;
+        for (int e = 0; e < E; e += 4) {
+            const float4 gv = (apply_norm && g != nullptr && v < nvec)
+                                  ? __ldg(reinterpret_cast<const float4*>(g + static_cast<int64_t>(v) * E + e))
+                                  : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            gk[e] = gv.x; gk[e + 1] = gv.y; gk[e + 2] = gv.z; gk[e + 3] = gv.w;
+        }
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            float h = x[j][e];
+            float x = V::elem(raw[j], e);
             if (apply_norm) {
-                h = __fmul_rn(h, r);
-                if (g != nullptr && v < nvec) h = __fmul_rn(h, __ldg(g + v * E + e));
+                x = __fmul_rn(x, r);
+                if (g != nullptr) x = __fmul_rn(x, gk[e]);
             }
-            x[j][e] = h;
-            m = fmaxf(m, fabsf(h));
+            h[e] = x;
         }
+    };
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        float h[E];
+        xhat(j, h);
+#pragma unroll
+        for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(h[e]));
     }
-    m = block_max_f32<NT>(m, red_f);
+    m = warp_max(m);
     const float s = __fdiv_rn(127.0f, fmaxf(m, 1e-5f));
     const float c = __frcp_rn(s);
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
         sx[t] = s;
         if (apply_norm) rinv[t] = r;
     }
-
-    // codes and dequantised values.  |x_hat * s| <= 127 * (1 + 2^-23) for finite inputs,
-    // so rint(x_hat * s) is in [-127, 127]; the integer clamp is kept for robustness.
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-        const int v = threadIdx.x + j * NT;
+    for (int j = 0; j < VPL; ++j) {
+        const int v = lane + 32 * j;
         if (v >= nvec) continue;
+        float h[E];
+        xhat(j, h);
         uint32_t qb[E];
         float dq[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-            const float tq = __fadd_rn(__fmul_rn(x[j][e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
+            const float tq = __fadd_rn(__fmul_rn(h[e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
             const int qi = max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
             qb[e] = static_cast<uint32_t>(qi) & 0xFFu;
             dq[e] = div_by_scale(__fsub_rn(tq, kRoundMagic), s, c);

@@ -124,6 +124,26 @@ bl_status launched(const char* what) {
     return BL_OK;
 }
 
+// Every kernel is launched with programmatic dependent launch: its blocks may be scheduled
+// while the previous kernel in the stream drains (each kernel signals this at its start),
+// and each kernel runs its set-up (barriers, TMEM, descriptor prefetch) and then waits
+// (griddepcontrol.wait) for the previous grid's completion and memory before it touches
+// global memory.  After a kernel launched without the attribute the wait is a no-op.
+template <typename... KArgs, typename... Args>
+void pdl_launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);   // errors surface in launched()
+}
+
 // ------------------------------------------------------------------------------------
 // TMA tensor maps
 // ------------------------------------------------------------------------------------
@@ -191,7 +211,7 @@ bl_status launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensor
     a.wait_ns = g_wait_ns.load();
     const int tiles = a.m_tiles * a.n_tiles;
     const int grid = tiles < dev.sms ? tiles : dev.sms;
-    kern<<<grid, bl::kTcThreads, smem, st>>>(ta, tb, td, a);
+    pdl_launch(kern, dim3(grid), dim3(bl::kTcThreads), smem, st, ta, tb, td, a);
     return launched("tc_gemm");
 }
 
@@ -229,7 +249,7 @@ bl_status launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtenso
     a.wait_ns = g_wait_ns.load();
     const int tiles = a.m_tiles * a.n_tiles;
     const int clusters = tiles < mc ? tiles : mc;
-    kern<<<2 * clusters, bl::kTcThreads, smem, st>>>(ta, tb, td, a);
+    pdl_launch(kern, dim3(2 * clusters), dim3(bl::kTcThreads), smem, st, ta, tb, td, a);
     return launched("tc_gemm2");
 }
 
@@ -240,19 +260,35 @@ inline bool use_2sm(int64_t M) { return M > bl::kTcBM; }
 // ------------------------------------------------------------------------------------
 // pieces shared by the entry points (validation already done by the caller)
 // ------------------------------------------------------------------------------------
+// One row per block (the kernel can take R adjacent rows per block; measured slower here).
 template <bool kBf16, int VPT>
 void launch_act_quant_v(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
                         float* sx, float* rinv, void* Xdq, cudaStream_t st) {
     constexpr int NT = bl::act_threads<kBf16>();
-    bl::act_quant_kernel<kBf16, NT, VPT><<<(unsigned)T, NT, 0, st>>>(X, (int)K, apply_norm, g, eps, Xq, sx, rinv,
-                                                                     Xdq);
+    constexpr int R = 1;
+    const unsigned grid = (unsigned)((T + R - 1) / R);
+    pdl_launch(bl::act_quant_kernel<kBf16, NT, VPT, R>, dim3(grid), dim3(NT), 0, st, X, (int)T, (int)K, apply_norm, g,
+               eps, Xq, sx, rinv, Xdq);
 }
 
+template <bool kBf16, int VPL>
+void launch_act_quant_w(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
+                        float* sx, float* rinv, void* Xdq, cudaStream_t st) {
+    pdl_launch(bl::act_quant_warp_kernel<kBf16, VPL>, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, st, X, (int)T,
+               (int)K, apply_norm, g, eps, Xq, sx, rinv, Xdq);
+}
+
+// Rows of at most 256 vectors (2048 bf16 / 1024 fp32 elements): warp per row; longer rows:
+// block per row.
 template <bool kBf16>
 void launch_act_quant(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
                       float* sx, float* rinv, void* Xdq, cudaStream_t st) {
     constexpr int NT = bl::act_threads<kBf16>();
     const int64_t nvec = K / (kBf16 ? 8 : 4);
+    if (nvec <= 32) return launch_act_quant_w<kBf16, 1>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    if (nvec <= 64) return launch_act_quant_w<kBf16, 2>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    if (nvec <= 128) return launch_act_quant_w<kBf16, 4>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    if (nvec <= 256) return launch_act_quant_w<kBf16, 8>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     const int64_t vpt = (nvec + NT - 1) / NT;
     if (vpt <= 1) launch_act_quant_v<kBf16, 1>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     else if (vpt <= 2) launch_act_quant_v<kBf16, 2>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
@@ -305,9 +341,8 @@ bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf
     }
     // fp32 layer: CUDA-core fp32 contraction, C[t,k] = gamma * sum_n dY[t,n] W_q[n,k]
     dim3 grid((unsigned)((K + 63) / 64), (unsigned)((T + 63) / 64));
-    bl::simt_gemm_kernel<float, uint16_t><<<grid, 256, 0, st>>>((int)T, (int)K, (int)N,
-                                                               static_cast<const float*>(dY), N, 1, Wq_bf16, 1, K,
-                                                               gamma, dXhat, K);
+    pdl_launch(bl::simt_gemm_kernel<float, uint16_t>, grid, dim3(256), 0, st, (int)T, (int)K, (int)N,
+               static_cast<const float*>(dY), N, (int64_t)1, Wq_bf16, (int64_t)1, K, gamma, dXhat, K);
     return launched("simt_gemm(grad_input)");
 }
 
@@ -324,9 +359,9 @@ bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int
         return launch_tc<false, true, true, bl::kEpiF32>(ta, tb, td, a, st, dev);
     }
     dim3 grid((unsigned)((K + 63) / 64), (unsigned)((N + 63) / 64));
-    bl::simt_gemm_kernel<float, float><<<grid, 256, 0, st>>>((int)N, (int)K, (int)T, static_cast<const float*>(dY),
-                                                            1, N, static_cast<const float*>(Xdq), 1, K, nullptr, dW,
-                                                            K);
+    pdl_launch(bl::simt_gemm_kernel<float, float>, grid, dim3(256), 0, st, (int)N, (int)K, (int)T,
+               static_cast<const float*>(dY), (int64_t)1, N, static_cast<const float*>(Xdq), (int64_t)1, K,
+               static_cast<const float*>(nullptr), dW, K);
     return launched("simt_gemm(grad_weight)");
 }
 
@@ -340,8 +375,8 @@ int launch_rmsnorm_bwd_v(const void* X, const float* rinv, const float* g, float
     int64_t grid = (T + R - 1) / R;
     const int64_t cap = sms * 4 < bl::kBwdMaxBlocks ? sms * 4 : bl::kBwdMaxBlocks;
     if (grid > cap) grid = cap;
-    bl::rmsnorm_bwd_kernel<kBf16X, VPT, R><<<(unsigned)grid, bl::kBwdThreads, 0, st>>>(X, rinv, g, dX, (int)T, (int)K,
-                                                                                       partial);
+    pdl_launch(bl::rmsnorm_bwd_kernel<kBf16X, VPT, R>, dim3((unsigned)grid), dim3(bl::kBwdThreads), 0, st, X, rinv, g,
+               dX, (int)T, (int)K, partial);
     return (int)grid;
 }
 
@@ -365,7 +400,8 @@ bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const f
                                    : launch_rmsnorm_bwd<false>(X, rinv, g, dX, T, K, partial, sms, st);
     BL_TRY(launched("rmsnorm_bwd"));
     if (dg != nullptr) {
-        bl::dg_reduce_kernel<<<(unsigned)((K + 31) / 32), 1024, 0, st>>>(partial, grid, (int)K, dg);
+        pdl_launch(bl::dg_reduce_kernel, dim3((unsigned)((K + 31) / 32)), dim3(1024), 0, st,
+                   static_cast<const float*>(partial), grid, (int)K, dg);
         BL_TRY(launched("dg_reduce"));
     }
     return BL_OK;
@@ -374,26 +410,31 @@ bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const f
 // Row kernels keep a whole row in registers: d_in is limited to 16384.
 constexpr int64_t kMaxRowK = 16384;
 
-template <int NTILES, int WB, int S>
+// One block per SM (at most one per row group) of 16 warps (12 for two n-tiles, whose
+// accumulators need more registers).
+template <int NTILES>
 bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
                       const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
-    CUtensorMap tw;
-    BL_TRY(make_tmap(&tw, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, 16));
-    const size_t smem = 1024 + bl::gemv_ring_bytes<WB, S>() + (size_t)B * (size_t)(K / 16 + 1) * 16 +
-                        sizeof(uint64_t) * WB * S;
+    constexpr int WB = NTILES == 1 ? 16 : 12;
+    const int64_t n_rg = N / 16;
+    const int64_t nb = n_rg < dev.sms ? n_rg : dev.sms;
+    const int max_rgs = (int)((n_rg + nb - 1) / nb);
+    const size_t smem = bl::gemv_smem_bytes((int)B, (int)K, max_rgs);
     BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
                "GEMV needs %zu bytes of shared memory for B = %lld, K = %lld; at most %d fit", smem, (long long)B,
                (long long)K, dev.max_smem_optin);
-    auto kern = bl::ternary_gemv_tma_kernel<NTILES, WB, S>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WB * 32, smem);
-    if (per_sm < 1) per_sm = 1;
-    const int64_t need = (N / 16 + WB - 1) / WB;
-    int64_t grid = (int64_t)dev.sms * per_sm;
-    if (grid > need) grid = need;
-    kern<<<(unsigned)grid, WB * 32, smem, st>>>(tw, gamma, (int)N, (int)K, xq, sx, (int)B, y, acc, g_wait_ns.load());
+    auto kern = bl::ternary_gemv_kernel<NTILES, WB>;
+    static std::atomic<uint64_t> attr_set{0};   // bit d: attribute set on device d
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (dev_id < 0 || dev_id >= 64) return fail(BL_ERR_DEVICE, "device ordinal %d out of range", dev_id);
+    if (!(attr_set.load() & (1ull << dev_id))) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_set.fetch_or(1ull << dev_id);
+    }
+    pdl_launch(kern, dim3((unsigned)nb), dim3(WB * 32), smem, st, Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, y,
+               acc, g_wait_ns.load());
     return launched("ternary_gemv");
 }
 
@@ -451,14 +492,14 @@ bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K, int8_t* W
     const int64_t n = N * K;
     const int parts = bl::wq_num_partials(n);
     double* partials = static_cast<double*>(ws);
-    bl::absmean_partial_kernel<<<parts, bl::kWqThreads, 0, st>>>(W, n, partials);
+    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
     BL_TRY(launched("absmean_partial"));
     const int64_t groups = n / 16;
     int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
     const int64_t cap = (int64_t)dev.sms * 4;
     if (blocks > cap) blocks = cap;
-    bl::ternary_quant_kernel<<<(unsigned)blocks, bl::kWqThreads, 0, st>>>(W, n, partials, parts, Wq_i8, Wq_bf16,
-                                                                          Wpacked, gamma);
+    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
+               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
     return launched("ternary_quant");
 }
 
@@ -610,7 +651,8 @@ bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t* Wpack
     const int64_t groups = N * K / 16;
     int64_t blocks = (groups + 255) / 256;
     if (blocks > (int64_t)dev.sms * 8) blocks = (int64_t)dev.sms * 8;
-    bl::ternary_pack_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(Wq_i8, N * K, Wpacked);
+    pdl_launch(bl::ternary_pack_kernel, dim3((unsigned)blocks), dim3(256), 0, static_cast<cudaStream_t>(stream), Wq_i8,
+               N * K, Wpacked);
     return launched("ternary_pack");
 }
 
@@ -624,14 +666,14 @@ bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, in
     BL_TRY(check_ptr(acc, "acc", false));
     BL_TRY(check_dims(1, N, K));
     BL_REQUIRE(K % 64 == 0, BL_ERR_UNSUPPORTED_SHAPE,
-               "the GEMV reads packed rows with TMA: K must be a multiple of 64 (16-byte rows), got %lld", (long long)K);
+               "the GEMV reads packed rows in 16-byte pieces: K must be a multiple of 64, got %lld", (long long)K);
     BL_REQUIRE(B >= 1 && B <= 16, BL_ERR_UNSUPPORTED_SHAPE, "batch must be in [1, 16], got %lld", (long long)B);
     BL_REQUIRE(K <= 65536, BL_ERR_UNSUPPORTED_SHAPE, "K must be <= 65536 for the GEMV, got %lld", (long long)K);
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (B <= 8) return launch_gemv<1, 8, 4>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
-    return launch_gemv<2, 16, 2>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
+    if (B <= 8) return launch_gemv<1>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
+    return launch_gemv<2>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
 }
 
 bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
@@ -668,14 +710,14 @@ bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, i
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     double* partials = static_cast<double*>(scratch);
     // pass 1 writes every partial that pass 2 reads, so nothing in the scratch needs clearing
-    bl::absmean_partial_kernel<<<parts, bl::kWqThreads, 0, st>>>(W, n, partials);
+    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
     BL_TRY(launched("absmean_partial"));
     const int64_t groups = n / 16;
     int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
     const int64_t cap = (int64_t)dev.sms * 4;
     if (blocks > cap) blocks = cap;
-    bl::ternary_quant_kernel<<<(unsigned)blocks, bl::kWqThreads, 0, st>>>(W, n, partials, parts, Wq_i8, Wq_bf16,
-                                                                          Wpacked, gamma);
+    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
+               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
     return launched("ternary_quant");
 }
 
@@ -683,7 +725,7 @@ bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
     BL_REQUIRE(limit_ns > 0 && limit_ns <= 10000000000ull, BL_ERR_INVALID_ARG, "limit must be in (0, 10 s]");
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
-    bl::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    pdl_launch(bl::selftest_wait_kernel, dim3(1), dim3(32), 0, static_cast<cudaStream_t>(stream), limit_ns);
     return launched("selftest_wait");
 }
 

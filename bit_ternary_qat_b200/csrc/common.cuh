@@ -28,6 +28,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch (every kernel of the library is launched with it): let the
+// next kernel in the stream be scheduled, and wait until the previous kernel has completed
+// and its memory operations are visible.  Each kernel calls pdl_trigger_and_wait() after
+// its set-up and before its first global-memory access.
+__device__ __forceinline__ void pdl_trigger_and_wait() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// 1024-byte aligned start inside the dynamic shared-memory array.  Offsetting the
+// __shared__ array itself (rather than round-tripping the pointer through an integer) keeps
+// the shared address space visible to the compiler, so accesses through the result are
+// shared-memory instructions and not generic ones.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* smem_raw) {
+    return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
     asm volatile(
@@ -70,6 +87,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a waiting warp sleeps (up to the hint) until the phase
+// completes instead of spinning, which leaves the issue slots to the warps that have work.
+constexpr uint32_t kWaitHintNs = 10000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar_addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "n"(kWaitHintNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Bounded: gives up after
 // `limit_ns` of wall-clock time or as soon as *abort becomes non-zero (another role of
 // the same block gave up).  Returns false when it gave up.
@@ -79,8 +111,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if ((i & 63u) == 0u) {
+        if (mbar_try_wait_sleep(a, parity)) return true;
+        if ((i & 7u) == 0u) {
             if (abort != nullptr && *abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 record_status(6 /* BL_ERR_TIMEOUT */);
@@ -108,6 +140,14 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* desc, ui
 }
 
 // TMA store (shared -> global) of one 2-D box; completion tracked with bulk groups.
+// Plain bulk copy global -> shared (no tensor map, no multicast): `bytes` and both addresses
+// multiples of 16; completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 __device__ __forceinline__ void tma_store_2d(const void* desc, const void* smem_src, int32_t x, int32_t y) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(desc)),

@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(int M, int N, int K, con
     constexpr int BM = 64, BN = 64, BK = 16;
     __shared__ float As[BK][BM + 4];
     __shared__ float Bs[BK][BN + 4];
+    pdl_trigger_and_wait();
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     float acc[4][4] = {};

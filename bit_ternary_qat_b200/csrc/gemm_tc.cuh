@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kChunkCols = epi_chunk_cols(kEpi);
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align1024(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + kTcStages * kTcABytes;
     uint8_t* sE = sB + kTcStages * kBBytes;
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger_and_wait();
 
     const int num_tiles = args.m_tiles * args.n_tiles;
     const uint64_t lim = args.wait_ns;
@@ -359,7 +360,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     constexpr int kChunkCols = epi_chunk_cols(kEpi);
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = smem_align1024(smem_raw);
     uint8_t* sA = smem;
     uint8_t* sB = smem + kTc2Stages * kTc2HalfBytes;
     uint8_t* sE = sB + kTc2Stages * kTc2HalfBytes;
@@ -400,6 +401,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger_and_wait();
 
     const int num_tiles = args.m_tiles * args.n_tiles;   // m_tiles counts 256-row pair tiles
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;

@@ -5,35 +5,27 @@
 // 10 -> -1, 11 reserved (decodes to 0 here).  Output y = acc * (gamma / s_b), the factor
 // formed once per activation row.
 //
-// The weights are streamed from HBM exactly once, by TMA, and no code is ever decoded to a
-// value: for a 32-bit word of 16 codes (code 16g + 4i + j at bits 8i + 2j), the in-place
-// mask w & (0x01010101 << (2j + p)) keeps bit p of code j of each byte, i.e. four bytes
-// that are 0 or 2^(2j+p).  With the activations staged once per block as interleaved words
+// The weights are streamed from HBM exactly once, into registers, and no code is ever decoded to a
+// separate value.  Two identities do the decoding inside 32-bit words of 16 codes (code
+// 16g + 4i + j of row n at bits 8i + 2j of word g):
+//   (1) with L = w & 0x5555..., H = (w >> 1) & 0x5555..., the word
+//         F = (L | 0xAAAA...) - H
+//       holds in every 2-bit field f = 2 + lo - hi = dec(c) + 2, in {1, 2, 3} (no borrow
+//       crosses a field because 2 + lo >= 1 + hi), and the reserved code 11 gives f = 2,
+//       i.e. dec = 0;
+//   (2) F & (0x03030303 << 2j) keeps field j of each byte in place: four bytes f * 4^j,
+//       exactly the four u8 entries of one mma A register.
+// With the activations staged once per block as interleaved words
 // x_j = (x[16g+j], x[16g+4+j], x[16g+8+j], x[16g+12+j]),
-//   sum_k dec(c_k) x_k = sum_j (lo-plane . x_j) / 4^j - (hi-plane . x_j) / (2 4^j),
-// which also maps the reserved 11 to 0.  The dot products run on the tensor cores
-// (mma.sync m16n8k32, u8 x s8 -> s32).
+//   sum_k dec(c_k) x_k = sum_j D_j / 4^j - 2 sum_k x_k,   D_j = sum (F & mask_j) . x_j,
+// where every D_j is an exact multiple of 4^j and sum_k x_k is a property of the
+// activation row alone.  The dot products D_j run on the tensor cores (mma.sync m16n8k32,
+// u8 x s8 -> s32): one byte slot per code.
 #pragma once
 #include "common.cuh"
 
 namespace bl {
 
-// ------------------------------------------------------------------------------------
-// Tensor-core variant (mma.sync m16n8k32, u8 x s8 -> s32).
-//
-// A warp owns 16 weight rows.  For a "super-chunk" of 8 packed words per row (128 codes),
-// lane (g = lane/4, t = lane%4) holds words 2t and 2t+1 of rows g and g+8.  For a bit
-// plane p (lo = bit 0, hi = bit 1) and a position j (code j of each byte), masking a word
-// in place, w & (0x01010101 << (2j + p)), gives 4 bytes that are 0 or 2^(2j+p): exactly
-// the 4 int8 entries one mma A register holds.  So with logical k = 4t + i (word 2t) and
-// 16 + 4t + i (word 2t+1), the A fragment of (j, p) is 4 masked words, and the matching B
-// fragment is the interleaved activation word x_j of groups 2t and 2t+1 (already staged in
-// shared memory), for batch column g.  Eight mma per n-tile per super-chunk (4 j x 2
-// planes) accumulate into D[j][p]; the result is sum_j D_lo[j] / 4^j - D_hi[j] / (2 4^j),
-// exact since every term of D[j][p] is a multiple of its scale.  The K reduction happens
-// inside the mma, so no cross-lane reduction is needed; 16 rows x 128 codes cost 32
-// masking instructions per lane.
-// ------------------------------------------------------------------------------------
 __device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -42,184 +34,213 @@ __device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], const uint32_t (&a)[
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-constexpr int kGemvTileBytes = 16 * 128;   // one TMA box: 16 weight rows x 128 bytes (512 codes)
+// identity (1): fields dec(c) + 2
+__device__ __forceinline__ uint32_t ternary_fields(uint32_t w) {
+    return ((w & 0x55555555u) | 0xAAAAAAAAu) - ((w >> 1) & 0x55555555u);
+}
 
-template <int WB, int S>
-__host__ __device__ constexpr size_t gemv_ring_bytes() { return (size_t)WB * S * kGemvTileBytes; }
+constexpr int kGemvStepBytes = 64;          // one step: 64 bytes (256 codes) of each of 16 rows
+constexpr int kGemvU = 4;                   // steps per batch of loads (software pipelined)
 
-// Weights reach shared memory through TMA: every warp streams its own row groups through a
-// private ring of S boxes (16 rows x 128 bytes, 128-byte swizzle) and keeps S boxes in
-// flight; a per-slot mbarrier (bounded wait) says when a box has landed.  Within a box,
-// lane (g, t) reads words (2t, 2t+1) of each 32-byte super-chunk of rows g and g+8 from
-// the swizzled layout -- conflict free -- and runs the mma of the comment above.  A warp
-// owns whole row groups, so its accumulators are final when the row group ends.
-// NTILES n-tiles of 8 batch columns (B <= 8 * NTILES); only the first B batch rows of the
-// activations are staged.
-template <int NTILES, int WB, int S>
-__global__ void __launch_bounds__(WB * 32) ternary_gemv_tma_kernel(
-    const __grid_constant__ CUtensorMap tmW, const float* __restrict__ gamma, int N, int K,
+// Shared memory of one block: staged activations (+1 int4 of padding per row), int32
+// row-group accumulators (+ activation row sums), one mbarrier.  `max_rgs` row groups.
+__host__ __device__ inline size_t gemv_smem_bytes(int B, int K, int max_rgs) {
+    const int spr = (K / 16 + 15) / 16;     // steps per row
+    const size_t ld = (size_t)spr * 16 + 1;
+    const size_t acc_ints = ((size_t)max_rgs * 16 * B + B + 1) & ~(size_t)1;
+    return 16 + (size_t)B * ld * 16 + acc_ints * 4 + sizeof(uint64_t) + 16;
+}
+
+// ------------------------------------------------------------------------------------
+// Block b owns the row groups (16 rows each) [rg0, rg1) of a balanced partition of the
+// N/16 row groups; its work is split into steps (row group, 64-byte column block) numbered
+// row-group-major, and warp w takes one contiguous, equally long run of them (+-1), so a
+// warp's run touches one or two row groups and all warps stream the same number of bytes.
+// A warp reads its weights straight from HBM into registers: per step, lane (g = lane/4,
+// t = lane%4) loads words 4t..4t+3 of the step's 64 bytes of rows g and g+8 (one 16-byte
+// load each; 8 rows x 64 contiguous bytes per warp instruction), kGemvU steps per batch,
+// the next batch loading while the current one is multiplied.  Words 4t, 4t+1 feed one
+// m16n8k32 k-block and words 4t+2, 4t+3 the next: byte i of word q holds codes 16q + 4i + j,
+// so k-slot 4t + i (16 + 4t + i) of a k-block pairs with activation word x_j of group q =
+// 4t (4t + 1), etc.  When its run leaves a row group the warp folds its accumulators and
+// adds them into the block's shared int32 sums of that row group (shared-memory integer
+// atomics: exact, order free); after a block barrier the block writes y for its rows.
+// The activation rows reach shared memory by bulk copy (one bounded mbarrier wait) while
+// the first weight batch is already in flight, and are interleaved in place.
+// ------------------------------------------------------------------------------------
+template <int NTILES, int WB>
+__global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
+    const uint8_t* __restrict__ W, const float* __restrict__ gamma, int N, int K,
     const int8_t* __restrict__ xq, const float* __restrict__ sx, int B, float* __restrict__ y,
     int32_t* __restrict__ acc_out, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* rings = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int G = K / 16;                        // groups of 16 codes (one packed word) per row
-    const int ld = G + 1;                        // padded row stride (int4) -> conflict-free reads
-    int4* xs = reinterpret_cast<int4*>(rings + gemv_ring_bytes<WB, S>());   // [B][G + 1]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(xs + static_cast<size_t>(B) * ld);
-
-    for (int idx = threadIdx.x; idx < B * G; idx += WB * 32) {
-        const int b = idx / G, gg = idx - b * G;
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(b) * K) + gg);
-        int4 o;
-        int* ov = reinterpret_cast<int*>(&o);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t t01 = __byte_perm(raw.x, raw.y, j | ((4 + j) << 4));
-            const uint32_t t23 = __byte_perm(raw.z, raw.w, j | ((4 + j) << 4));
-            ov[j] = static_cast<int>(__byte_perm(t01, t23, 0x5410));
-        }
-        xs[b * ld + gg] = o;
-    }
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < WB * S; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
-        tma_prefetch_desc(&tmW);
-    }
-    __syncthreads();
+    uint8_t* base = smem_raw + ((16u - (smem_u32(smem_raw) & 15u)) & 15u);
+    const int row_bytes = K / 4;
+    const int G = K / 16;                        // packed words per weight row
+    const int spr = (G + 15) / 16;               // steps per row (16 words each)
+    const int Gp = spr * 16;                     // staged activation groups per row (zero past G)
+    const int ld = Gp + 1;
+    const int n_rg = N / 16;
+    const int rg0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_rg / gridDim.x);
+    const int rg1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_rg / gridDim.x);
+    const int nrg = rg1 - rg0;
+    int4* xs = reinterpret_cast<int4*>(base);                                  // [B][ld]
+    int* accs = reinterpret_cast<int*>(xs + static_cast<size_t>(B) * ld);      // [nrg*16][B]
+    int* xsum = accs + nrg * 16 * B;                                          // [B]
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(accs + ((nrg * 16 * B + B + 1) & ~1));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int KT = (K / 4 + 127) / 128;          // boxes per row
-    const int n_rg = N / 16;
-    const int first_rg = blockIdx.x * WB + warp;
-    const int rg_step = gridDim.x * WB;
-    const int my_rgs = first_rg < n_rg ? (n_rg - first_rg + rg_step - 1) / rg_step : 0;
-    const int total = my_rgs * KT;
-    uint8_t* ring = rings + static_cast<size_t>(warp) * S * kGemvTileBytes;
-    uint64_t* bar = bars + warp * S;
-    const float gm = __ldg(gamma);
-
-    auto issue = [&](int i, int rg, int kt) {
-        const int slot = i % S;
-        mbar_arrive_expect_tx(&bar[slot], kGemvTileBytes);
-        tma_load_2d(ring + slot * kGemvTileBytes, &tmW, &bar[slot], kt * 128, rg * 16);
-    };
-    // producer position (lane 0 only): the box S tiles ahead of the consumer
-    int p_rg = first_rg, p_kt = 0;
-    auto advance = [&](int& rg, int& kt) {
-        if (++kt == KT) { kt = 0; rg += rg_step; }
-    };
-    if (lane == 0)
-        for (int i = 0; i < S && i < total; ++i) { issue(i, p_rg, p_kt); advance(p_rg, p_kt); }
-
-    // per-lane constants: swizzled offsets of words (2t, 2t+1) of super-chunk sc in rows g and
-    // g+8 (same chunk permutation, since (g + 8) % 8 == g) and the activation-word indices
-    int off[4];
-#pragma unroll
-    for (int sc = 0; sc < 4; ++sc) off[sc] = g * 128 + (((2 * sc + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
-    int xbase[NTILES];
-    bool xlive[NTILES];
-#pragma unroll
-    for (int nt = 0; nt < NTILES; ++nt) {
-        xlive[nt] = nt * 8 + g < B;
-        xbase[nt] = (nt * 8 + g) * ld + 2 * t;
+    if (threadIdx.x == 0) {
+        mbar_init(xbar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_trigger_and_wait();
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(B * K));
+        for (int b = 0; b < B; ++b)
+            bulk_load(xs + static_cast<size_t>(b) * ld, xq + static_cast<int64_t>(b) * K, static_cast<uint32_t>(K), xbar);
     }
 
-    constexpr bool kShift = NTILES == 2;
-    constexpr int kJ = kShift ? 1 : 4;
-    int d[kJ][2][NTILES][4];
-    bool ok = true;
-    int i = 0;
-    int c_rg = first_rg, c_kt = 0;               // consumer position
-    for (; i < total; ++i) {
-        const int slot = i % S;
-        if (c_kt == 0) {
-#pragma unroll
-            for (int j = 0; j < kJ; ++j)
-#pragma unroll
-                for (int p = 0; p < 2; ++p)
-#pragma unroll
-                    for (int nt = 0; nt < NTILES; ++nt)
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) d[j][p][nt][q] = 0;
+    // this warp's run of steps [i0, i1) of the block's row-group-major sequence
+    const int nsteps = nrg * spr;
+    const int i0 = static_cast<int>(static_cast<int64_t>(warp) * nsteps / WB);
+    const int i1 = static_cast<int>(static_cast<int64_t>(warp + 1) * nsteps / WB);
+    // lane's 16-byte slice of rows g and g+8 of step i (zero past the row end)
+    auto load_step = [&](int i, uint4& ra, uint4& rb) {
+        ra = make_uint4(0u, 0u, 0u, 0u);
+        rb = ra;
+        if (i < i1) {
+            const int rgl = i / spr, s = i - (i / spr) * spr;
+            const int col = s * kGemvStepBytes + 16 * t;
+            if (col < row_bytes) {
+                const uint8_t* p = W + (static_cast<int64_t>(rg0 + rgl) * 16 + g) * row_bytes + col;
+                ra = __ldcs(reinterpret_cast<const uint4*>(p));
+                rb = __ldcs(reinterpret_cast<const uint4*>(p + 8 * static_cast<int64_t>(row_bytes)));
+            }
         }
-        if (!mbar_wait(&bar[slot], (i / S) & 1, wait_ns, nullptr)) { ok = false; break; }
-        const uint8_t* tile = ring + slot * kGemvTileBytes;
-        const int gbase = c_kt * 32;             // first group of this box
+    };
+    uint4 wa[kGemvU], wb[kGemvU];
 #pragma unroll
-        for (int sc = 0; sc < 4; ++sc) {
-            // NTILES == 1: planes masked in place (scale 2^(2j+p), one accumulator set per
-            // (j, p)).  NTILES == 2: planes shifted down to scale 1 first (one more instruction
-            // per register, two accumulator sets instead of eight).
-            const uint2 wa = *reinterpret_cast<const uint2*>(tile + off[sc]);
-            const uint2 wb = *reinterpret_cast<const uint2*>(tile + off[sc] + 8 * 128);
-            const int grp = gbase + sc * 8;      // + 2t (in xbase): group of word 2t
-            int4 xb0[NTILES], xb1[NTILES];
+    for (int u = 0; u < kGemvU; ++u) load_step(i0 + u, wa[u], wb[u]);
+
+    // activations: wait for the copies, interleave in place (zero past K), clear the sums
+    for (int idx = threadIdx.x; idx < nrg * 16 * B; idx += WB * 32) accs[idx] = 0;
+    mbar_wait(xbar, 0, wait_ns, nullptr);
+    for (int idx = threadIdx.x; idx < B * Gp; idx += WB * 32) {
+        const int b = idx / Gp, gg = idx - b * Gp;
+        int4 o = make_int4(0, 0, 0, 0);
+        if (gg < G) {
+            const int4 raw = xs[b * ld + gg];
+            int* ov = reinterpret_cast<int*>(&o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t t01 = __byte_perm(raw.x, raw.y, j | ((4 + j) << 4));
+                const uint32_t t23 = __byte_perm(raw.z, raw.w, j | ((4 + j) << 4));
+                ov[j] = static_cast<int>(__byte_perm(t01, t23, 0x5410));
+            }
+        }
+        xs[b * ld + gg] = o;
+    }
+    __syncthreads();
+    // sum_k x[b][k] (the "- 2 sum x" term), one warp per activation row
+    for (int b = warp; b < B; b += WB) {
+        int sacc = 0;
+        for (int gg = lane; gg < Gp; gg += 32) {
+            const int4 v = xs[b * ld + gg];
+            sacc = __dp4a(v.x, 0x01010101, sacc);
+            sacc = __dp4a(v.y, 0x01010101, sacc);
+            sacc = __dp4a(v.z, 0x01010101, sacc);
+            sacc = __dp4a(v.w, 0x01010101, sacc);
+        }
+        sacc = warp_sum(sacc);
+        if (lane == 0) xsum[b] = sacc;
+    }
+
+    // batch column of this lane in n-tile nt (columns past B read row B-1; never written)
+    int xbase[NTILES];
+#pragma unroll
+    for (int nt = 0; nt < NTILES; ++nt) xbase[nt] = min(nt * 8 + g, B - 1) * ld + 4 * t;
+
+    int d[4][NTILES][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NTILES; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) d[j][nt][q] = 0;
+    auto flush = [&](int rgl) {
+#pragma unroll
+        for (int nt = 0; nt < NTILES; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int tot = d[0][nt][q] + (d[1][nt][q] >> 2) + (d[2][nt][q] >> 4) + (d[3][nt][q] >> 6);
+                const int b = nt * 8 + 2 * t + (q & 1);
+                const int r = (q < 2) ? g : g + 8;
+                if (b < B) atomicAdd(&accs[(rgl * 16 + r) * B + b], tot);
+                d[0][nt][q] = d[1][nt][q] = d[2][nt][q] = d[3][nt][q] = 0;
+            }
+    };
+    // one step: two k-blocks (words 4t, 4t+1 and 4t+2, 4t+3 of rows g and g+8)
+    auto mma_step = [&](const uint4& ra, const uint4& rb, int s) {
+        const uint32_t fa[4] = {ternary_fields(ra.x), ternary_fields(ra.y), ternary_fields(ra.z), ternary_fields(ra.w)};
+        const uint32_t fb[4] = {ternary_fields(rb.x), ternary_fields(rb.y), ternary_fields(rb.z), ternary_fields(rb.w)};
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+            int4 x0[NTILES], x1[NTILES];
 #pragma unroll
             for (int nt = 0; nt < NTILES; ++nt) {
-                const bool live = xlive[nt] && grp + 2 * t < G;   // G is even: grp + 2t + 1 < G too
-                xb0[nt] = live ? xs[xbase[nt] + grp] : make_int4(0, 0, 0, 0);
-                xb1[nt] = live ? xs[xbase[nt] + grp + 1] : make_int4(0, 0, 0, 0);
+                x0[nt] = xs[xbase[nt] + s * 16 + 2 * kb];
+                x1[nt] = xs[xbase[nt] + s * 16 + 2 * kb + 1];
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
+                const uint32_t m = 0x03030303u << (2 * j);
+                const uint32_t a[4] = {fa[2 * kb] & m, fb[2 * kb] & m, fa[2 * kb + 1] & m, fb[2 * kb + 1] & m};
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    uint32_t a[4];
-                    if constexpr (kShift) {
-                        const int sh = 2 * j + p;
-                        a[0] = (wa.x >> sh) & 0x01010101u; a[1] = (wb.x >> sh) & 0x01010101u;
-                        a[2] = (wa.y >> sh) & 0x01010101u; a[3] = (wb.y >> sh) & 0x01010101u;
-                    } else {
-                        const uint32_t m = 0x01010101u << (2 * j + p);
-                        a[0] = wa.x & m; a[1] = wb.x & m; a[2] = wa.y & m; a[3] = wb.y & m;
-                    }
-                    const int jj = kShift ? 0 : j;
-#pragma unroll
-                    for (int nt = 0; nt < NTILES; ++nt) {
-                        const int* x0 = reinterpret_cast<const int*>(&xb0[nt]);
-                        const int* x1 = reinterpret_cast<const int*>(&xb1[nt]);
-                        mma_u8s8_16832(d[jj][p][nt], a, static_cast<uint32_t>(x0[j]), static_cast<uint32_t>(x1[j]));
-                    }
+                for (int nt = 0; nt < NTILES; ++nt) {
+                    const int* p0 = reinterpret_cast<const int*>(&x0[nt]);
+                    const int* p1 = reinterpret_cast<const int*>(&x1[nt]);
+                    mma_u8s8_16832(d[j][nt], a, static_cast<uint32_t>(p0[j]), static_cast<uint32_t>(p1[j]));
                 }
             }
         }
-        __syncwarp();                            // every lane is done with this slot
-        if (lane == 0 && i + S < total) { issue(i + S, p_rg, p_kt); advance(p_rg, p_kt); }
-        if (c_kt == KT - 1) {
-            // D[q]: rows (r0, r0, r1, r1) x batch columns (2t, 2t+1, 2t, 2t+1) of each n-tile
-            const int r0 = c_rg * 16 + g, r1 = r0 + 8;
+    };
+
+    int rgl = i0 / spr, s = i0 - (i0 / spr) * spr;
+    for (int i = i0; i < i1; i += kGemvU) {
+        uint4 na[kGemvU], nb[kGemvU];
 #pragma unroll
-            for (int nt = 0; nt < NTILES; ++nt)
+        for (int u = 0; u < kGemvU; ++u) load_step(i + kGemvU + u, na[u], nb[u]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    int tot = 0;
-                    if constexpr (kShift) {
-                        tot = d[0][0][nt][q] - d[0][1][nt][q];
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            tot += (d[j][0][nt][q] >> (2 * j)) - (d[j][1][nt][q] >> (2 * j + 1));
-                    }
-                    const int b = nt * 8 + 2 * t + (q & 1);
-                    if (b < B) {
-                        const int64_t o = static_cast<int64_t>(b) * N + ((q < 2) ? r0 : r1);
-                        y[o] = __fmul_rn(static_cast<float>(tot), __fdiv_rn(gm, __ldg(sx + b)));
-                        if (acc_out != nullptr) acc_out[o] = tot;
-                    }
-                }
+        for (int u = 0; u < kGemvU; ++u) {
+            if (i + u < i1) {
+                mma_step(wa[u], wb[u], s);
+                if (s == spr - 1 || i + u == i1 - 1) flush(rgl);
+                if (++s == spr) { s = 0; ++rgl; }
+            }
         }
-        advance(c_rg, c_kt);
+#pragma unroll
+        for (int u = 0; u < kGemvU; ++u) { wa[u] = na[u]; wb[u] = nb[u]; }
     }
-    if (!ok && lane == 0) {
-        // drain the boxes still in flight into this warp's ring before the block can exit
-        for (int k = i + 1; k < total && k < i + S; ++k) mbar_wait(&bar[k % S], (k / S) & 1, 100000000ull, nullptr);
+    __syncthreads();
+
+    // y[b][n] = (acc - 2 sum x_b) * fl(gamma / s_b) for this block's rows, row-fastest
+    const float gm = __ldg(gamma);
+    const int rows = nrg * 16;
+    for (int idx = threadIdx.x; idx < rows * B; idx += WB * 32) {
+        const int b = idx / rows, r = idx - b * rows;
+        const int acc = accs[r * B + b] - 2 * xsum[b];
+        const int64_t o = static_cast<int64_t>(b) * N + rg0 * 16 + r;
+        y[o] = __fmul_rn(static_cast<float>(acc), __fdiv_rn(gm, __ldg(sx + b)));
+        if (acc_out != nullptr) acc_out[o] = acc;
     }
-    __syncwarp();
 }
 
 // Bounded-wait self test: one thread waits on an mbarrier that nothing arrives on.
 __global__ void selftest_wait_kernel(uint64_t limit_ns) {
+    pdl_trigger_and_wait();
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
     if (threadIdx.x == 0) {

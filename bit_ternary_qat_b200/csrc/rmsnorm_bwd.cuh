@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_kernel(const void* __
                                                                   int K, float* __restrict__ dg_partial) {
     constexpr int NT = kBwdThreads;
     __shared__ float red[R][NT / 32];
+    pdl_trigger_and_wait();
     const int nvec = K / 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(1024) dg_reduce_kernel(const float* __restrict
                                                          float* __restrict__ dg) {
     constexpr int kPerWarp = (kBwdMaxBlocks + 31) / 32;
     __shared__ float red[32][33];
+    pdl_trigger_and_wait();
     const int c = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int k = blockIdx.x * 32 + c;
     float v[kPerWarp];

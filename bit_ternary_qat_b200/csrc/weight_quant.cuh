@@ -37,6 +37,7 @@ __host__ __device__ inline int wq_num_partials(int64_t n) {
 __global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float* __restrict__ W, int64_t n,
                                                                      double* __restrict__ partials) {
     __shared__ double red[kWqThreads / 32];
+    pdl_trigger_and_wait();
     const int64_t nvec = n / 4;
     const float4* w4 = reinterpret_cast<const float4*>(W);
     const int64_t stride = (int64_t)gridDim.x * kWqThreads;
@@ -139,6 +140,8 @@ __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
     int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
     float* __restrict__ gamma_out) {
     __shared__ float s_thr;
+    __shared__ double s_red[kWqThreads / 32];
+    pdl_trigger_and_wait();
     const int64_t ngroups = n / 16;
     const int64_t stride = (int64_t)gridDim.x * kWqThreads;
     const float4* w4 = reinterpret_cast<const float4*>(W);
@@ -151,18 +154,28 @@ __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
             w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
         }
     }
-    if (threadIdx.x < 32) {
-        // fixed-order sum of the partials: lane-strided with four accumulators, fixed butterfly
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        int i = threadIdx.x;
-        for (; i + 96 < nparts; i += 128) {
-            a0 += partials[i];
-            a1 += partials[i + 32];
-            a2 += partials[i + 64];
-            a3 += partials[i + 96];
+    {
+        // fixed-order sum of the partials by the whole block: thread i adds partials
+        // i, i + 256, ... (all loaded at once), then a fixed butterfly per warp and the warp
+        // sums in order
+        constexpr int kPerThread = (kWqMaxPartials + kWqThreads - 1) / kWqThreads;
+        double pv[kPerThread];
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) {
+            const int i = threadIdx.x + kWqThreads * k;
+            pv[k] = i < nparts ? partials[i] : 0.0;
         }
-        for (; i < nparts; i += 32) a0 += partials[i];
-        const double sum = warp_sum((a0 + a1) + (a2 + a3));
+        double a = 0.0;
+#pragma unroll
+        for (int k = 0; k < kPerThread; ++k) a += pv[k];
+        a = warp_sum(a);
+        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = a;
+        __syncthreads();
+    }
+    if (threadIdx.x < 32) {
+        double sum = 0.0;
+#pragma unroll
+        for (int wi = 0; wi < kWqThreads / 32; ++wi) sum += s_red[wi];
         const float gamma = fmaxf(static_cast<float>(sum / static_cast<double>(n)), 1e-5f);
         const float thr = ternary_threshold_warp(gamma);
         if (threadIdx.x == 0) {
@@ -186,6 +199,7 @@ __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
 // Standalone packing of int8 codes (ternary_pack): one thread per 16 codes.
 __global__ void __launch_bounds__(256) ternary_pack_kernel(const int8_t* __restrict__ wq, int64_t n,
                                                            uint8_t* __restrict__ packed) {
+    pdl_trigger_and_wait();
     const int64_t ngroups = n / 16;
     for (int64_t gi = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; gi < ngroups;
          gi += (int64_t)gridDim.x * blockDim.x) {

@@ -225,7 +225,10 @@ BL_API bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t
  *   y[b,n]   = acc[b,n] * (gamma / sx[b])              fp32
  * Wpacked uint8 [N x K/4]; gamma fp32 [1]; xq int8 [B x K]; sx fp32 [B];
  * y fp32 [B x N]; acc int32 [B x N] optional.  1 <= B <= 16, K <= 65536, and K % 64 == 0
- * (packed rows are read with TMA, which needs 16-byte aligned rows). */
+ * (packed rows are read in 16-byte pieces and activation rows are bulk-copied, both of
+ * which need 16-byte aligned rows).
+ * A block keeps B activation rows (B * K bytes) in shared memory: shapes whose rows do not
+ * fit (e.g. B * K well above 160 KB) return BL_ERR_UNSUPPORTED_SHAPE. */
 BL_API bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K,
                        const int8_t* xq, const float* sx, int64_t B,
                        float* y, int32_t* acc, void* stream);

@@ -259,8 +259,8 @@ def test_square_workload_full_size(bl):
 # decode GEMV over packed weights
 # ------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K", [(48, 64), (400, 192), (1024, 8192), (272, 4096), (160, 704)])
-@pytest.mark.parametrize("B", [1, 2, 4, 5, 16])
+@pytest.mark.parametrize("N,K", [(48, 64), (400, 192), (1024, 8192), (272, 4096), (160, 704), (4800, 704)])
+@pytest.mark.parametrize("B", [1, 2, 4, 5, 8, 9, 16])
 def test_gemv_parity(bl, N, K, B):
     W, x = synth.decode_inputs(B, N, K, seed=N + K + B)
     qw = bl.bitlinear_quant_weight(_gpu(W))
@@ -283,6 +283,28 @@ def test_gemv_reserved_code_decodes_to_zero(bl):
                              _gpu(torch.from_numpy(xq)), _gpu(torch.from_numpy(s)), want_acc=True)
     acc_o, _ = oracle.gemv(packed, 0.02, K, xq, s)
     assert np.array_equal(np_(acc), acc_o)
+
+
+def test_gemv_extreme_magnitudes(bl):
+    """Longest rows (K = 65536), all codes -1 / +1 / reserved, activations at -128 and 127."""
+    N, K, B = 64, 65536, 2                           # B * K bytes of activations fill shared memory
+    rows = []
+    for r in range(N):
+        code = (2, 1, 3, 0)[r % 4]                   # -1, +1, reserved, 0
+        byte = code | (code << 2) | (code << 4) | (code << 6)
+        rows.append(np.full(K // 4, byte, dtype=np.uint8))
+    packed = np.stack(rows)
+    xq = np.empty((B, K), dtype=np.int8)
+    xq[0] = -128
+    xq[1] = np.where(np.arange(K) % 2 == 0, -128, 127)
+    s = np.array([1.0, 0.25], dtype=np.float32)
+    y, acc = bl.ternary_gemv(_gpu(torch.from_numpy(packed)), _gpu(torch.tensor([0.75])), K,
+                             _gpu(torch.from_numpy(xq)), _gpu(torch.from_numpy(s)), want_acc=True)
+    torch.cuda.synchronize()
+    acc_o, y_o = oracle.gemv(packed, 0.75, K, xq, s)
+    assert int(np.abs(acc_o).max()) == 128 * K
+    assert np.array_equal(np_(acc), acc_o)
+    assert np.array_equal(np_(y), y_o)
 
 
 def test_decode_workload_full_size(bl):

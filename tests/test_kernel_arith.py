@@ -108,23 +108,47 @@ def test_ternary_threshold_equals_round_clamp():
         assert np.array_equal(got, ref), float(gamma)
 
 
-def test_gemv_bitplane_identity():
+def _ternary_fields(w):
+    """(w & 0x55..) | 0xAA.. minus (w >> 1) & 0x55.., in 32-bit arithmetic."""
+    return (((w & 0x55555555) | 0xAAAAAAAA) - ((w >> 1) & 0x55555555)) & 0xFFFFFFFF
+
+
+def test_gemv_field_identity():
+    """The GEMV's two in-word identities, emulated on the integers.
+
+    Every 2-bit field of F equals dec(code) + 2 (the reserved 11 included), and masking F
+    with 0x03030303 << 2j leaves bytes f_j * 4^j; then
+    sum_j D_j / 4^j - 2 sum x == sum dec * x with D_j the byte dot products.
+    """
     rng = np.random.default_rng(3)
-    K = 64
-    codes = rng.integers(0, 4, size=K)           # includes the reserved 11
-    x = rng.integers(-128, 128, size=K).astype(np.int64)
-    dec = np.where(codes == 1, 1, np.where(codes == 2, -1, 0))
-    ref = int(np.sum(dec * x))
-    # pack 16 codes per 32-bit word, element k at bits 2*(k % 16) of word k // 16
-    words = [sum(int(codes[16 * g + i]) << (2 * i) for i in range(16)) for g in range(K // 16)]
-    tot = 0
-    for g, w in enumerate(words):
-        for j in range(4):
-            xs = [int(x[16 * g + 4 * i + j]) for i in range(4)]        # interleaved activation word
-            lo = [(w >> (8 * i + 2 * j)) & 1 for i in range(4)]
-            hi = [(w >> (8 * i + 2 * j + 1)) & 1 for i in range(4)]
-            tot += sum(l * xv for l, xv in zip(lo, xs)) - sum(h * xv for h, xv in zip(hi, xs))
-            # in-place masks: byte i of w & (0x01010101 << 2j) is lo * 2^(2j)
-            m = w & (0x01010101 << (2 * j))
-            assert [(m >> (8 * i)) & 0xFF for i in range(4)] == [l << (2 * j) for l in lo]
-    assert tot == ref
+    dec_of = {0: 0, 1: 1, 2: -1, 3: 0}
+    # exhaustive over one byte of four codes, in each byte position of the word
+    for byte in range(256):
+        for pos in range(4):
+            w = byte << (8 * pos)
+            f = _ternary_fields(w)
+            for j in range(4):
+                c = (byte >> (2 * j)) & 3
+                assert (f >> (8 * pos + 2 * j)) & 3 == dec_of[c] + 2
+    for trial in range(20):
+        K = 64 * (1 + trial)
+        codes = rng.integers(0, 4, size=K)           # includes the reserved 11
+        x = rng.integers(-128, 128, size=K).astype(np.int64)
+        if trial == 0:
+            x[:] = -128                              # extreme activations
+        dec = np.where(codes == 1, 1, np.where(codes == 2, -1, 0))
+        ref = int(np.sum(dec * x))
+        # 16 codes per 32-bit word, code k at bits 2*(k % 16) of word k // 16
+        words = [sum(int(codes[16 * g + e]) << (2 * e) for e in range(16)) for g in range(K // 16)]
+        D = [0, 0, 0, 0]
+        for g, w in enumerate(words):
+            F = _ternary_fields(w)
+            for j in range(4):
+                xs = [int(x[16 * g + 4 * i + j]) for i in range(4)]    # interleaved activation word
+                m = F & (0x03030303 << (2 * j))
+                a = [(m >> (8 * i)) & 0xFF for i in range(4)]           # u8 entries of the mma A register
+                assert all(v % (4 ** j) == 0 and 4 ** j <= v <= 3 * 4 ** j for v in a)
+                D[j] += sum(av * xv for av, xv in zip(a, xs))
+        assert all(D[j] % (4 ** j) == 0 for j in range(4))
+        got = sum(D[j] >> (2 * j) for j in range(4)) - 2 * int(np.sum(x))
+        assert got == ref
