@@ -245,19 +245,26 @@ __global__ void __launch_bounds__(256, 4) act_quant_warp_kernel(const void* __re
         raw[j] = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
     }
 
-    // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order
+    // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order; max |x| on the way
     float r = 1.0f;
-    if (apply_norm) {
+    float mx = 0.0f;
+    {
         double ss = 0.0;
 #pragma unroll
         for (int j = 0; j < VPL; ++j)
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const double xd = static_cast<double>(V::elem(raw[j], e));
-                ss = fma(xd, xd, ss);
+                const float xf = V::elem(raw[j], e);
+                mx = fmaxf(mx, fabsf(xf));
+                if (apply_norm) {
+                    const double xd = static_cast<double>(xf);
+                    ss = fma(xd, xd, ss);
+                }
             }
-        ss = warp_sum(ss);
-        r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(eps)));
+        if (apply_norm) {
+            ss = warp_sum(ss);
+            r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(eps)));
+        }
     }
     // x_hat = fl(fl(x * r) * g) of the E elements of vector j (recomputed where needed)
     auto xhat = [&](int j, float (&h)[E]) {
@@ -280,13 +287,18 @@ __global__ void __launch_bounds__(256, 4) act_quant_warp_kernel(const void* __re
             h[e] = x;
         }
     };
+    // max |x_hat|: without a gain, rounding is monotone, so max |fl(x r)| = fl(max |x| * r)
     float m = 0.0f;
+    if (apply_norm && g != nullptr) {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        float h[E];
-        xhat(j, h);
+        for (int j = 0; j < VPL; ++j) {
+            float h[E];
+            xhat(j, h);
 #pragma unroll
-        for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(h[e]));
+            for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(h[e]));
+        }
+    } else {
+        m = apply_norm ? __fmul_rn(mx, r) : mx;
     }
     m = warp_max(m);
     const float s = __fdiv_rn(127.0f, fmaxf(m, 1e-5f));

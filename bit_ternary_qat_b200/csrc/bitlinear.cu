@@ -366,6 +366,24 @@ bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int
 }
 
 size_t quant_ws_bytes() { return sizeof(double) * bl::kWqMaxPartials; }
+
+// Weight quantiser: fp64 partial sums of |W| (pass 1), then gamma, threshold and codes
+// (pass 2, one round of kTqGroups groups per thread when the grid covers W).
+bl_status run_quant_weight(const float* W, int64_t n, void* scratch, int8_t* Wq_i8, uint16_t* Wq_bf16,
+                           uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev) {
+    double* partials = static_cast<double*>(scratch);
+    const int parts = bl::wq_num_partials(n);
+    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
+    BL_TRY(launched("absmean_partial"));
+    const int64_t groups = n / 16;
+    const int64_t per_block = (int64_t)bl::kWqThreads * bl::kTqGroups;
+    int64_t blocks = (groups + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)dev.sms * 4;
+    if (blocks > cap) blocks = cap;
+    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
+               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
+    return launched("ternary_quant");
+}
 size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
 
 template <bool kBf16X, int VPT>
@@ -489,18 +507,7 @@ bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K, int8_t* W
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t n = N * K;
-    const int parts = bl::wq_num_partials(n);
-    double* partials = static_cast<double*>(ws);
-    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
-    BL_TRY(launched("absmean_partial"));
-    const int64_t groups = n / 16;
-    int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
-    const int64_t cap = (int64_t)dev.sms * 4;
-    if (blocks > cap) blocks = cap;
-    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
-               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
-    return launched("ternary_quant");
+    return run_quant_weight(W, N * K, ws, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
 }
 
 bl_status bitlinear_act_quant(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int apply_rmsnorm, const float* g,
@@ -707,18 +714,8 @@ bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, i
         }
         scratch = addr[dev_id];
     }
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    double* partials = static_cast<double*>(scratch);
     // pass 1 writes every partial that pass 2 reads, so nothing in the scratch needs clearing
-    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
-    BL_TRY(launched("absmean_partial"));
-    const int64_t groups = n / 16;
-    int64_t blocks = (groups + bl::kWqThreads - 1) / bl::kWqThreads;
-    const int64_t cap = (int64_t)dev.sms * 4;
-    if (blocks > cap) blocks = cap;
-    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
-               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
-    return launched("ternary_quant");
+    return run_quant_weight(W, n, scratch, Wq_i8, Wq_bf16, Wpacked, gamma, static_cast<cudaStream_t>(stream), dev);
 }
 
 bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

@@ -133,8 +133,11 @@ __device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int6
     }
 }
 
-// grid-stride over 16-element groups; n % 32 == 0.  Each thread issues the loads of its
-// first group before the block waits for gamma and the threshold.
+// n % 32 == 0.  Each thread loads kTqGroups groups of 16 weights (all loads in flight)
+// before the block waits for gamma and the threshold, then quantises them; weights beyond
+// grid * kWqThreads * kTqGroups groups are handled in further rounds of the same kind.
+constexpr int kTqGroups = 2;
+
 __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
     const float* __restrict__ W, int64_t n, const double* __restrict__ partials, int nparts,
     int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
@@ -143,17 +146,22 @@ __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
     __shared__ double s_red[kWqThreads / 32];
     pdl_trigger_and_wait();
     const int64_t ngroups = n / 16;
-    const int64_t stride = (int64_t)gridDim.x * kWqThreads;
     const float4* w4 = reinterpret_cast<const float4*>(W);
-    int64_t gi = blockIdx.x * (int64_t)kWqThreads + threadIdx.x;
-    float w[16];
-    if (gi < ngroups) {
+    const int64_t round_groups = static_cast<int64_t>(gridDim.x) * kWqThreads * kTqGroups;
+    auto load = [&](int64_t r0, float (&w)[kTqGroups][16], int64_t (&gi)[kTqGroups]) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = __ldg(w4 + gi * 4 + j);
-            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        for (int q = 0; q < kTqGroups; ++q) {
+            gi[q] = r0 + (static_cast<int64_t>(blockIdx.x) * kTqGroups + q) * kWqThreads + threadIdx.x;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = gi[q] < ngroups ? __ldg(w4 + gi[q] * 4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                w[q][4 * j] = v.x; w[q][4 * j + 1] = v.y; w[q][4 * j + 2] = v.z; w[q][4 * j + 3] = v.w;
+            }
         }
-    }
+    };
+    float w[kTqGroups][16];
+    int64_t gi[kTqGroups];
+    load(0, w, gi);
     {
         // fixed-order sum of the partials by the whole block: thread i adds partials
         // i, i + 256, ... (all loaded at once), then a fixed butterfly per warp and the warp
@@ -185,14 +193,13 @@ __global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
     }
     __syncthreads();
     const float thr = s_thr;
-    if (gi < ngroups) quantise16(w, thr, gi, wq_i8, wq_bf16, packed);
-    for (gi += stride; gi < ngroups; gi += stride) {
+    for (int64_t r0 = 0;;) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = __ldg(w4 + gi * 4 + j);
-            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
-        }
-        quantise16(w, thr, gi, wq_i8, wq_bf16, packed);
+        for (int q = 0; q < kTqGroups; ++q)
+            if (gi[q] < ngroups) quantise16(w[q], thr, gi[q], wq_i8, wq_bf16, packed);
+        r0 += round_groups;
+        if (r0 >= ngroups) break;
+        load(r0, w, gi);
     }
 }
 
