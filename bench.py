@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
+    ap.add_argument("--table", action="store_true",
+                    help="time every configuration's full step (single, square, mlp7b, layer7b, decode) and the "
+                         "oracle on a bounded sample of each; one JSON object, not the bench line")
     return ap.parse_args()
 
 
@@ -226,11 +229,14 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if args.only_gemv:
+    if args.only_gemv or args.table:
         blbuild.build()
         bl.load()
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        print(json.dumps({"decode_gemv": gemv_measure(bl, torch, dev, flush, peaks())}), flush=True)
+        if args.table:
+            print(json.dumps({"table": table_measure(bl, torch, dev, flush, peaks())}), flush=True)
+        else:
+            print(json.dumps({"decode_gemv": gemv_measure(bl, torch, dev, flush, peaks())}), flush=True)
         return
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
@@ -541,6 +547,122 @@ def gemv_measure(bl, torch, dev, flush, pk):
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
                        "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5")
     return out
+
+
+def table_measure(bl, torch, dev, flush, pk, steps: int = 5):
+    """Every configuration's step -- for each of its layers: weight quantisation, activation
+    quantisation, forward GEMM, grad-input GEMM, RMSNorm backward, weight-gradient GEMM --
+    captured in one CUDA graph and timed with CUDA events after an L2 flush (median of
+    `steps`); tokens/s = T / step time.  Plus the oracle on a bounded token sample of each
+    layer (full weight quantisation), extrapolated linearly in tokens."""
+    import oracle as ora
+    from bit_ternary_qat_b200 import synth
+    ora.build()
+    out = {}
+    for name in ("single", "square", "mlp7b", "layer7b"):
+        wl = synth.WORKLOADS[name]
+        lis = synth.workload_inputs(name)
+        T = lis[0].X.shape[0]
+        dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        maxK = max(li.X.shape[1] for li in lis)
+        maxN = max(li.W.shape[0] for li in lis)
+        ws = bl.workspace(T, maxN, maxK, dev)
+        dev_layers = []
+        for li in lis:
+            N, K = li.W.shape
+            dev_layers.append(dict(
+                W=li.W.to(dev), X=li.X.to(dev), dY=li.dY.to(dev), N=N, K=K,
+                q=dict(gamma=torch.empty(1, dtype=torch.float32, device=dev),
+                       wq_i8=torch.empty(N, K, dtype=torch.int8, device=dev),
+                       wq_bf16=torch.empty(N, K, dtype=torch.bfloat16, device=dev),
+                       packed=torch.empty(N, K // 4, dtype=torch.uint8, device=dev))))
+        shared = dict(xq=torch.empty(T * maxK, dtype=torch.int8, device=dev),
+                      xdq=torch.empty(T * maxK, dtype=dt, device=dev),
+                      sx=torch.empty(T, dtype=torch.float32, device=dev),
+                      rinv=torch.empty(T, dtype=torch.float32, device=dev),
+                      y=torch.empty(T * maxN, dtype=dt, device=dev),
+                      dX=torch.empty(T * maxK, dtype=torch.float32, device=dev),
+                      dW=torch.empty(maxN * maxK, dtype=torch.float32, device=dev),
+                      dg=torch.empty(maxK, dtype=torch.float32, device=dev))
+
+        def step():
+            for L in dev_layers:
+                N, K = L["N"], L["K"]
+                a = dict(xq=shared["xq"][:T * K].view(T, K), xdq=shared["xdq"][:T * K].view(T, K),
+                         sx=shared["sx"], rinv=shared["rinv"])
+                bl.bitlinear_quant_weight(L["W"], ws=ws, out=L["q"])
+                bl.bitlinear_act_quant(L["X"], apply_rmsnorm=True, out=a)
+                bl.bitlinear_linear(a["xq"], a["sx"], L["q"]["wq_i8"], L["q"]["gamma"],
+                                    out_dtype=dt, y=shared["y"][:T * N].view(T, N))
+                dX = shared["dX"][:T * K].view(T, K)
+                bl.bitlinear_grad_input(L["dY"], L["q"]["wq_bf16"], L["q"]["gamma"], dXhat=dX)
+                bl.bitlinear_rmsnorm_backward(L["X"], a["rinv"], dX, ws=ws, dg=shared["dg"][:K])
+                bl.bitlinear_backward_weight(L["dY"], a["xdq"], dW=shared["dW"][:N * K].view(N, K))
+
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(steps):
+            flush.zero_()
+            a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_ev.record()
+            graph.replay()
+            b_ev.record()
+            torch.cuda.synchronize()
+            ms.append(a_ev.elapsed_time(b_ev))
+        del graph
+        assert bl.check_device_status() == 0
+        t = statistics.median(ms)
+        ops_fwd = sum(2.0 * T * L["N"] * L["K"] for L in dev_layers)
+        # oracle: bounded token sample per layer, extrapolated linearly in tokens
+        t_s = min(T, 64 if T <= 4096 else 16)
+        cpu_s = 0.0
+        for li in lis:
+            full = oracle_step(ora, li, t_s)
+            wq_only = oracle_weight_quant_s(ora, li)
+            cpu_s += wq_only + (full - wq_only) * (T / t_s)
+        out[name] = {"tokens": T, "layers": [f"{L['K']}->{L['N']}" for L in dev_layers], "dtype": wl.dtype,
+                     "ms_per_step": t, "tokens_per_s": T / (t * 1e-3),
+                     "step_tops_all_gemms": 3 * ops_fwd / (t * 1e-3) / 1e12,
+                     "oracle": {"tokens_per_s": T / cpu_s, "cores": ora.num_threads(),
+                                "sample": f"{t_s} of {T} tokens per layer, full weight quantisation, "
+                                          f"extrapolated linearly in tokens" if t_s < T else "full step"}}
+        print(json.dumps({name: out[name]}), flush=True)
+        del dev_layers, shared, ws
+        torch.cuda.empty_cache()
+    out["decode"] = gemv_measure(bl, torch, dev, flush, pk)
+    # oracle decode GEMV at batch 1 on the packed 28672 x 8192 weight (quantisation not timed)
+    W, x = synth.decode_inputs(1)
+    gamma, wq = ora.quant_weight(W.numpy())
+    packed = ora.pack(wq)
+    xq, s_b, _ = ora.act_quant(x.numpy(), None, None)
+    t0 = time.perf_counter()
+    ora.gemv(packed, gamma, 8192, xq, s_b)
+    dt_s = time.perf_counter() - t0
+    out["decode"]["oracle_B1"] = {"us": dt_s * 1e6, "GB/s": (28672 * 8192 // 4) / dt_s / 1e9,
+                                  "cores": ora.num_threads()}
+    return out
+
+
+def oracle_weight_quant_s(ora, li) -> float:
+    W = li.W.numpy()
+    t0 = time.perf_counter()
+    gamma, wq = ora.quant_weight(W)
+    ora.pack(wq)
+    return time.perf_counter() - t0
 
 
 if __name__ == "__main__":

@@ -134,10 +134,13 @@ def layer_inputs(wl: Workload, layer: LayerShape, gen: torch.Generator,
     return LayerInputs(layer, X, W, dY, None)
 
 
-def workload_inputs(name: str, tokens: Optional[int] = None) -> List[LayerInputs]:
+def workload_inputs(name: str, tokens: Optional[int] = None, first: Optional[int] = None) -> List[LayerInputs]:
+    """Inputs of every layer of a workload (or of its first `first` layers: the draws are
+    sequential, so these equal the leading layers of the full list)."""
     wl = WORKLOADS[name]
     gen = generator(wl.seed)
-    return [layer_inputs(wl, ly, gen, tokens) for ly in wl.layers]
+    layers = wl.layers if first is None else wl.layers[:first]
+    return [layer_inputs(wl, ly, gen, tokens) for ly in layers]
 
 
 def decode_inputs(batch: int, d_out: int = 28672, d_in: int = 8192, seed: int = 4):

@@ -223,11 +223,14 @@ def test_layer_parity(bl, T, K, N, dtype, gain):
     assert max_rel_err(np_(dg), dg_o) <= tol
 
 
-def test_square_workload_full_size(bl):
-    """d_in = d_out = 2048, 4096 tokens, bf16: every code exact, sampled rows of the
+@pytest.mark.parametrize("workload,layer", [("square", 0), ("mlp7b", 0), ("mlp7b", 1), ("layer7b", 0)])
+def test_workload_full_size(bl, workload, layer):
+    """Full-size layers of the benchmark workloads (square 2048->2048 x 4096 tokens; the
+    7B MLP's 4096->11008 and 11008->4096 x 8192 tokens with Student-t weights; the 7B
+    layer's 4096->4096 x 16384 tokens), bf16: every code exact, sampled rows of the
     accumulators / outputs / gradients against the oracle, the rest through exact
     properties."""
-    li = synth.workload_inputs("square")[0]
+    li = synth.workload_inputs(workload, first=layer + 1)[layer]
     dt, g_gpu, wq, f, dX, dW, dg = _layer_case(bl, li)
     T, K = li.X.shape
     r_gpu = np_(f["rinv"])
@@ -236,8 +239,14 @@ def test_square_workload_full_size(bl):
     assert np.array_equal(np_(f["xq"]), xq)
     assert np.array_equal(np_(f["sx"]), s)
     assert np.array_equal(np_(f["xdq"]), oracle.round_bf16(xdq))
-    # zero fraction of the ternary codes (P3 §6: healthy 30-50%; Gaussian -> 31.0%)
-    assert abs(float(np.mean(wq == 0)) - 0.31006) < 0.002
+    # zero fraction of the ternary codes (P3 §6: healthy 30-50%; closed forms 0.31006 for
+    # Gaussian and 0.38019 for Student-t3 weights, the latter with a wider band because the
+    # sample mean of |t3| converges slowly)
+    zf = float(np.mean(wq == 0))
+    if synth.WORKLOADS[workload].w_dist == "normal":
+        assert abs(zf - 0.31006) < 0.002
+    else:
+        assert abs(zf - 0.38019) < 0.004
     rows = sample_rows(T, 32, seed=1)
     acc_o = oracle.int_gemm(xq, wq, rows=rows)
     assert np.array_equal(np_(f["acc"])[rows], acc_o)
