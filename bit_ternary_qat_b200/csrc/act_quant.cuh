@@ -22,7 +22,9 @@
 //     faithful quotient, so e1 = q - s_t y1 is exact and fl(y1 + e1 c) is the correctly
 //     rounded quotient.  tests/test_kernel_arith.py checks this in exact rational
 //     arithmetic for every q in [-128, 127] over a wide range of s_t, and the GPU parity
-//     tests compare X_dq with the oracle's division.
+//     tests compare X_dq with the oracle's division.  The 256 quotients of a row are
+//     computed once into a shared-memory table (already in the output type) and every
+//     element looks its value up by code.
 #pragma once
 #include "common.cuh"
 
@@ -59,6 +61,58 @@ __device__ __forceinline__ float div_by_scale(float q, float s, float c) {
 
 // R independent block sums / maxima with one barrier each (fixed order: per thread, then a
 // fixed butterfly, then the warps in order).
+// X_dq through a per-row table: entry q + 128 holds fl32(q / s_t) (computed with
+// div_by_scale), stored as the output element type (bf16 bits after one RNE rounding, or
+// fp32), so each element costs one shared-memory load instead of the five-op division.
+template <bool kBf16>
+struct DqLut;
+template <>
+struct DqLut<true> {
+    using T = uint16_t;
+    __device__ __forceinline__ static uint16_t make(float d) { return float_to_bf16_bits(d); }
+};
+template <>
+struct DqLut<false> {
+    using T = float;
+    __device__ __forceinline__ static float make(float d) { return d; }
+};
+
+// Quantise one vector of E values of x_hat with scale s and store its codes (E int8) and,
+// when wanted, its dequantised values from the row's table; elements are handled in pairs
+// so few values are live at once.
+__device__ __forceinline__ int quant_code(float h, float s) {
+    const float tq = __fadd_rn(__fmul_rn(h, s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
+    return max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
+}
+
+template <bool kBf16, int E>
+__device__ __forceinline__ void quant_store_vec(const float (&h)[E], float s, int8_t* Xq, void* Xdq, int64_t vec,
+                                                const typename DqLut<kBf16>::T* lut) {
+    uint32_t cw[E / 4];
+    uint32_t o[E / 2];
+#pragma unroll
+    for (int w = 0; w < E / 4; ++w) cw[w] = 0u;
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+        const int q0 = quant_code(h[2 * i], s), q1 = quant_code(h[2 * i + 1], s);
+        cw[i >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
+                      << (16 * (i & 1));
+        if (Xdq != nullptr) {
+            if constexpr (kBf16)
+                o[i] = static_cast<uint32_t>(lut[q0 + 128]) | (static_cast<uint32_t>(lut[q1 + 128]) << 16);
+            else
+                o[i] = 0u, reinterpret_cast<float*>(Xdq)[vec * E + 2 * i] = lut[q0 + 128],
+                reinterpret_cast<float*>(Xdq)[vec * E + 2 * i + 1] = lut[q1 + 128];
+        }
+    }
+    if constexpr (kBf16) {
+        reinterpret_cast<uint2*>(Xq)[vec] = make_uint2(cw[0], cw[1]);
+        if (Xdq != nullptr) reinterpret_cast<uint4*>(Xdq)[vec] = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+        reinterpret_cast<uint32_t*>(Xq)[vec] = cw[0];
+    }
+}
+
 template <int NT, int R>
 __device__ __forceinline__ void block_sum_f64(double (&v)[R], double (*red)[NT / 32]) {
 #pragma unroll
@@ -102,9 +156,11 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
                                                        int8_t* __restrict__ Xq, float* __restrict__ sx,
                                                        float* __restrict__ rinv, void* __restrict__ Xdq) {
     using V = ActVec<kBf16>;
+    using LutT = typename DqLut<kBf16>::T;
     constexpr int E = V::kElems;
     __shared__ double red_d[R][NT / 32];
     __shared__ float red_f[R][NT / 32];
+    __shared__ LutT lut[R][256];
     pdl_trigger_and_wait();
 
     const int nvec = K / E;
@@ -170,14 +226,24 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
     }
     block_max_f32<NT, R>(m, red_f);
 
+    float s[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+        s[q] = __fdiv_rn(127.0f, fmaxf(m[q], 1e-5f));
+        if (Xdq != nullptr) {
+            // row q's table of fl(q / s) for q = -128..127
+            const float c = __frcp_rn(s[q]);
+            for (int i = threadIdx.x; i < 256; i += NT)
+                lut[q][i] = DqLut<kBf16>::make(div_by_scale(static_cast<float>(i - 128), s[q], c));
+        }
+    }
+    if (Xdq != nullptr) __syncthreads();
 #pragma unroll
     for (int q = 0; q < R; ++q) {
         const int64_t t = t0 + q;
         if (t >= T) break;
-        const float s = __fdiv_rn(127.0f, fmaxf(m[q], 1e-5f));
-        const float c = __frcp_rn(s);
         if (threadIdx.x == 0) {
-            sx[t] = s;
+            sx[t] = s[q];
             if (apply_norm) rinv[t] = r[q];
         }
         const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
@@ -187,34 +253,7 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
         for (int j = 0; j < VPT; ++j) {
             const int v = threadIdx.x + j * NT;
             if (v >= nvec) continue;
-            uint32_t qb[E];
-            float dq[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float tq = __fadd_rn(__fmul_rn(x[q][j][e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
-                const int qi = max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
-                qb[e] = static_cast<uint32_t>(qi) & 0xFFu;
-                dq[e] = div_by_scale(__fsub_rn(tq, kRoundMagic), s, c);
-            }
-            if constexpr (kBf16) {
-                uint2 packed;
-                packed.x = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
-                packed.y = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
-                reinterpret_cast<uint2*>(Xq)[row_vec0 + v] = packed;
-                if (Xdq != nullptr) {
-                    uint32_t o[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dq[2 * i], dq[2 * i + 1]);
-                        o[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                    }
-                    reinterpret_cast<uint4*>(Xdq)[row_vec0 + v] = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            } else {
-                reinterpret_cast<uint32_t*>(Xq)[row_vec0 + v] = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
-                if (Xdq != nullptr)
-                    reinterpret_cast<float4*>(Xdq)[row_vec0 + v] = make_float4(dq[0], dq[1], dq[2], dq[3]);
-            }
+            quant_store_vec<kBf16, E>(x[q][j], s[q], Xq, Xdq, row_vec0 + v, lut[q]);
         }
     }
 }
@@ -224,16 +263,19 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
 // Each lane keeps its VPL raw vectors of the row in registers and widens them on use, so a
 // warp has the whole row in flight at once and many rows fit on an SM.
 template <bool kBf16, int VPL>
-__global__ void __launch_bounds__(256, 4) act_quant_warp_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
+__global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
                                                              const float* __restrict__ g, float eps,
                                                              int8_t* __restrict__ Xq, float* __restrict__ sx,
                                                              float* __restrict__ rinv, void* __restrict__ Xdq) {
     using V = ActVec<kBf16>;
+    using LutT = typename DqLut<kBf16>::T;
     constexpr int E = V::kElems;
+    __shared__ LutT lut_all[8][256];
     pdl_trigger_and_wait();
     const int lane = threadIdx.x & 31;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
+    LutT* lut = lut_all[threadIdx.x >> 5];
     const int nvec = K / E;
     const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
     const uint4* xrow = reinterpret_cast<const uint4*>(X) + row_vec0;
@@ -307,39 +349,19 @@ __global__ void __launch_bounds__(256, 4) act_quant_warp_kernel(const void* __re
         sx[t] = s;
         if (apply_norm) rinv[t] = r;
     }
+    if (Xdq != nullptr) {
+        // this row's table of fl(q / s) for q = -128..127 (8 entries per lane)
+#pragma unroll
+        for (int i = lane; i < 256; i += 32) lut[i] = DqLut<kBf16>::make(div_by_scale(static_cast<float>(i - 128), s, c));
+        __syncwarp();
+    }
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
         const int v = lane + 32 * j;
         if (v >= nvec) continue;
         float h[E];
         xhat(j, h);
-        uint32_t qb[E];
-        float dq[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const float tq = __fadd_rn(__fmul_rn(h[e], s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
-            const int qi = max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
-            qb[e] = static_cast<uint32_t>(qi) & 0xFFu;
-            dq[e] = div_by_scale(__fsub_rn(tq, kRoundMagic), s, c);
-        }
-        if constexpr (kBf16) {
-            uint2 packed;
-            packed.x = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
-            packed.y = qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24);
-            reinterpret_cast<uint2*>(Xq)[row_vec0 + v] = packed;
-            if (Xdq != nullptr) {
-                uint32_t o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(dq[2 * i], dq[2 * i + 1]);
-                    o[i] = *reinterpret_cast<const uint32_t*>(&h2);
-                }
-                reinterpret_cast<uint4*>(Xdq)[row_vec0 + v] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-        } else {
-            reinterpret_cast<uint32_t*>(Xq)[row_vec0 + v] = qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24);
-            if (Xdq != nullptr) reinterpret_cast<float4*>(Xdq)[row_vec0 + v] = make_float4(dq[0], dq[1], dq[2], dq[3]);
-        }
+        quant_store_vec<kBf16, E>(h, s, Xq, Xdq, row_vec0 + v, lut);
     }
 }
 
