@@ -59,8 +59,10 @@ __host__ __device__ inline size_t gemv_smem_bytes(int B, int K, int max_rgs) {
 // A warp reads its weights straight from HBM into registers: per step, lane (g = lane/4,
 // t = lane%4) loads words 4t..4t+3 of the step's 64 bytes of rows g and g+8 (one 16-byte
 // load each; 8 rows x 64 contiguous bytes per warp instruction), kGemvU steps per batch,
-// the next batch loading while the current one is multiplied.  Words 4t, 4t+1 feed one
-// m16n8k32 k-block and words 4t+2, 4t+3 the next: byte i of word q holds codes 16q + 4i + j,
+// two batches in registers (the next loading while the current one is multiplied), with
+// the load and compute positions advanced incrementally (no division in the loop).
+// Words 4t, 4t+1 feed one m16n8k32 k-block and words 4t+2, 4t+3 the next: byte i of word q
+// holds codes 16q + 4i + j,
 // so k-slot 4t + i (16 + 4t + i) of a k-block pairs with activation word x_j of group q =
 // 4t (4t + 1), etc.  When its run leaves a row group the warp folds its accumulators and
 // adds them into the block's shared int32 sums of that row group (shared-memory integer
@@ -107,23 +109,33 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     const int nsteps = nrg * spr;
     const int i0 = static_cast<int>(static_cast<int64_t>(warp) * nsteps / WB);
     const int i1 = static_cast<int>(static_cast<int64_t>(warp + 1) * nsteps / WB);
-    // lane's 16-byte slice of rows g and g+8 of step i (zero past the row end)
-    auto load_step = [&](int i, uint4& ra, uint4& rb) {
+    // Load cursor: the next step to load, its position in its row, and this lane's address of
+    // its 16-byte slice of row g (row g+8 is 8 rows further).  A slice past the row end (the
+    // last step of a row when K/4 is not a multiple of 64) loads as zeros.
+    const int64_t r8 = 8 * static_cast<int64_t>(row_bytes);
+    const int64_t rg_jump = 16 * static_cast<int64_t>(row_bytes) - static_cast<int64_t>(spr) * kGemvStepBytes;
+    const bool tail_ok = (spr - 1) * kGemvStepBytes + 16 * t < row_bytes;
+    int li = i0, l_s = i0 % spr;
+    const uint8_t* lp = W + (static_cast<int64_t>(rg0 + i0 / spr) * 16 + g) * row_bytes +
+                        static_cast<int64_t>(l_s) * kGemvStepBytes + 16 * t;
+    auto load_next = [&](uint4& ra, uint4& rb) {
         ra = make_uint4(0u, 0u, 0u, 0u);
         rb = ra;
-        if (i < i1) {
-            const int rgl = i / spr, s = i - (i / spr) * spr;
-            const int col = s * kGemvStepBytes + 16 * t;
-            if (col < row_bytes) {
-                const uint8_t* p = W + (static_cast<int64_t>(rg0 + rgl) * 16 + g) * row_bytes + col;
-                ra = __ldcs(reinterpret_cast<const uint4*>(p));
-                rb = __ldcs(reinterpret_cast<const uint4*>(p + 8 * static_cast<int64_t>(row_bytes)));
-            }
+        if (li < i1 && (l_s != spr - 1 || tail_ok)) {
+            ra = __ldcs(reinterpret_cast<const uint4*>(lp));
+            rb = __ldcs(reinterpret_cast<const uint4*>(lp + r8));
+        }
+        ++li;
+        lp += kGemvStepBytes;
+        if (++l_s == spr) {
+            l_s = 0;
+            lp += rg_jump;
         }
     };
-    uint4 wa[kGemvU], wb[kGemvU];
+    // two batches of kGemvU steps in registers: one multiplied while the other loads
+    uint4 Aa[kGemvU], Ab[kGemvU], Ba[kGemvU], Bb[kGemvU];
 #pragma unroll
-    for (int u = 0; u < kGemvU; ++u) load_step(i0 + u, wa[u], wb[u]);
+    for (int u = 0; u < kGemvU; ++u) load_next(Aa[u], Ab[u]);
 
     // activations: wait for the copies, interleave in place (zero past K), clear the sums
     for (int idx = threadIdx.x; idx < nrg * 16 * B; idx += WB * 32) accs[idx] = 0;
@@ -208,21 +220,29 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
         }
     };
 
-    int rgl = i0 / spr, s = i0 - (i0 / spr) * spr;
-    for (int i = i0; i < i1; i += kGemvU) {
-        uint4 na[kGemvU], nb[kGemvU];
-#pragma unroll
-        for (int u = 0; u < kGemvU; ++u) load_step(i + kGemvU + u, na[u], nb[u]);
+    int ci = i0, c_s = i0 % spr, c_rgl = i0 / spr;   // compute cursor
+    auto process = [&](uint4 (&pa)[kGemvU], uint4 (&pb)[kGemvU]) {
 #pragma unroll
         for (int u = 0; u < kGemvU; ++u) {
-            if (i + u < i1) {
-                mma_step(wa[u], wb[u], s);
-                if (s == spr - 1 || i + u == i1 - 1) flush(rgl);
-                if (++s == spr) { s = 0; ++rgl; }
+            if (ci < i1) {
+                mma_step(pa[u], pb[u], c_s);
+                if (c_s == spr - 1 || ci == i1 - 1) flush(c_rgl);
+                ++ci;
+                if (++c_s == spr) {
+                    c_s = 0;
+                    ++c_rgl;
+                }
             }
         }
+    };
+    while (ci < i1) {
 #pragma unroll
-        for (int u = 0; u < kGemvU; ++u) { wa[u] = na[u]; wb[u] = nb[u]; }
+        for (int u = 0; u < kGemvU; ++u) load_next(Ba[u], Bb[u]);
+        process(Aa, Ab);
+        if (ci >= i1) break;
+#pragma unroll
+        for (int u = 0; u < kGemvU; ++u) load_next(Aa[u], Ab[u]);
+        process(Ba, Bb);
     }
     __syncthreads();
 
