@@ -168,7 +168,8 @@ def oracle_step(ora, li, t_s: int):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(target_s: float = 15.0):
+def cpu_baseline(target_s: float = 12.0):
+    """The oracle on the square workload, repeated until about `target_s` seconds of CPU work."""
     import oracle as ora
     from bit_ternary_qat_b200 import synth
     ora.build()
@@ -178,9 +179,13 @@ def cpu_baseline(target_s: float = 15.0):
     while dt < target_s / 4 and t_s < T_TOK:
         t_s = min(T_TOK, t_s * 4)
         dt = oracle_step(ora, li, t_s)
-    return {"value": t_s / dt, "unit": "tokens/s", "cores": ora.num_threads(), "kind": "oracle",
-            "sample": f"one oracle step on {t_s} of the {T_TOK} tokens of the square workload "
-                      f"(weight quantisation over the full 2048x2048 W included), {dt:.1f} s"}
+    steps, tot = 1, dt
+    while tot < target_s:
+        tot += oracle_step(ora, li, t_s)
+        steps += 1
+    return {"value": steps * t_s / tot, "unit": "tokens/s", "cores": ora.num_threads(), "kind": "oracle",
+            "sample": f"{steps} oracle step(s) on {t_s} of the {T_TOK} tokens of the square workload "
+                      f"(weight quantisation over the full 2048x2048 W included), {tot:.1f} s"}
 
 
 def run_reference(args, rank, world):
