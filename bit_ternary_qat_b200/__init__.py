@@ -10,7 +10,8 @@ from . import ops  # noqa: F401
 from .ops import (  # noqa: F401
     bitlinear_act_quant, bitlinear_backward, bitlinear_backward_input, bitlinear_backward_weight,
     bitlinear_grad_input, bitlinear_rmsnorm_backward,
-    bitlinear_forward, bitlinear_linear, bitlinear_quant_weight, check_device_status, launch_count,
+    bitlinear_forward, bitlinear_forward_qat, bitlinear_linear, bitlinear_quant_weight,
+    bitlinear_quant_weight_noalloc, check_device_status, launch_count,
     selftest_bounded_wait, set_wait_limit_ns, ternary_gemv, ternary_pack, workspace, workspace_bytes,
 )
 

@@ -41,6 +41,7 @@ SIGNATURES = {
     "bitlinear_act_quant": (INT, [P, INT, I64, I64, INT, P, F, P, P, P, P, P]),
     "bitlinear_linear": (INT, [P, P, I64, I64, P, P, I64, P, INT, P, P]),
     "bitlinear_forward": (INT, [P, INT, I64, I64, P, F, P, P, I64, P, P, P, P, P, P, P]),
+    "bitlinear_forward_qat": (INT, [P, INT, I64, I64, P, F, P, I64, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
     "bitlinear_backward_input": (INT, [P, P, INT, I64, I64, I64, P, P, P, P, P, P, P, SZ, P]),
     "bitlinear_backward_weight": (INT, [P, P, INT, I64, I64, I64, P, P]),
     "bitlinear_grad_input": (INT, [P, INT, I64, I64, I64, P, P, P, P]),

@@ -263,17 +263,16 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
 // Each lane keeps its VPL raw vectors of the row in registers and widens them on use, so a
 // warp has the whole row in flight at once and many rows fit on an SM.
 template <bool kBf16, int VPL>
-__global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
-                                                             const float* __restrict__ g, float eps,
-                                                             int8_t* __restrict__ Xq, float* __restrict__ sx,
-                                                             float* __restrict__ rinv, void* __restrict__ Xdq) {
+__device__ __forceinline__ void act_quant_warp_rows(const void* __restrict__ X, int T, int K, int apply_norm,
+                                                    const float* __restrict__ g, float eps, int8_t* __restrict__ Xq,
+                                                    float* __restrict__ sx, float* __restrict__ rinv,
+                                                    void* __restrict__ Xdq, int row_block,
+                                                    typename DqLut<kBf16>::T (*lut_all)[256]) {
     using V = ActVec<kBf16>;
     using LutT = typename DqLut<kBf16>::T;
     constexpr int E = V::kElems;
-    __shared__ LutT lut_all[8][256];
-    pdl_trigger_and_wait();
     const int lane = threadIdx.x & 31;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int64_t t = static_cast<int64_t>(row_block) * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
     LutT* lut = lut_all[threadIdx.x >> 5];
     const int nvec = K / E;
@@ -363,6 +362,16 @@ __global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __re
         xhat(j, h);
         quant_store_vec<kBf16, E>(h, s, Xq, Xdq, row_vec0 + v, lut);
     }
+}
+
+template <bool kBf16, int VPL>
+__global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
+                                                                const float* __restrict__ g, float eps,
+                                                                int8_t* __restrict__ Xq, float* __restrict__ sx,
+                                                                float* __restrict__ rinv, void* __restrict__ Xdq) {
+    __shared__ typename DqLut<kBf16>::T lut_all[8][256];
+    pdl_trigger_and_wait();
+    act_quant_warp_rows<kBf16, VPL>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, blockIdx.x, lut_all);
 }
 
 // Largest row (elements) the register-resident kernel handles: 16 vectors per thread.

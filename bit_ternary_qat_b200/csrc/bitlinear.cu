@@ -21,6 +21,7 @@
 #include "gemm_simt.cuh"
 #include "rmsnorm_bwd.cuh"
 #include "gemv.cuh"
+#include "fused_quant.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -367,22 +368,51 @@ bl_status run_grad_weight_gemm(const void* dY, const void* Xdq, bl_dtype dt, int
 
 size_t quant_ws_bytes() { return sizeof(double) * bl::kWqMaxPartials; }
 
-// Weight quantiser: fp64 partial sums of |W| (pass 1), then gamma, threshold and codes
-// (pass 2, one round of kTqGroups groups per thread when the grid covers W).
+// Weight quantiser pass 2: gamma, threshold and codes (one round of kTqGroups groups per
+// thread when the grid covers W).
+bl_status run_ternary(const float* W, int64_t n, const double* partials, int parts, int8_t* Wq_i8, uint16_t* Wq_bf16,
+                      uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev) {
+    const int64_t groups = n / 16;
+    const int64_t per_block = (int64_t)bl::kWqThreads * bl::kTqGroups;
+    int64_t blocks = (groups + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)dev.sms * 4;
+    if (blocks > cap) blocks = cap;
+    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n, partials, parts,
+               Wq_i8, Wq_bf16, Wpacked, gamma);
+    return launched("ternary_quant");
+}
+
+// Weight quantiser: fp64 partial sums of |W| (pass 1), then pass 2.
 bl_status run_quant_weight(const float* W, int64_t n, void* scratch, int8_t* Wq_i8, uint16_t* Wq_bf16,
                            uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev) {
     double* partials = static_cast<double*>(scratch);
     const int parts = bl::wq_num_partials(n);
     pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
     BL_TRY(launched("absmean_partial"));
-    const int64_t groups = n / 16;
-    const int64_t per_block = (int64_t)bl::kWqThreads * bl::kTqGroups;
-    int64_t blocks = (groups + per_block - 1) / per_block;
-    const int64_t cap = (int64_t)dev.sms * 4;
-    if (blocks > cap) blocks = cap;
-    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
-               static_cast<const double*>(partials), parts, Wq_i8, Wq_bf16, Wpacked, gamma);
-    return launched("ternary_quant");
+    return run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
+}
+
+// Activation quantisation and the |W| partial sums in one launch (rows of <= 256 vectors).
+template <bool kBf16, int VPL>
+void launch_act_absmean(const void* X, int64_t T, int64_t K, const float* g, float eps, int8_t* Xq, float* sx,
+                        float* rinv, void* Xdq, const float* W, int64_t n, int parts, double* partials,
+                        cudaStream_t st) {
+    const unsigned grid = (unsigned)(parts + (T + 7) / 8);
+    pdl_launch(bl::act_quant_absmean_kernel<kBf16, VPL>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, 1, g, eps,
+               Xq, sx, rinv, Xdq, W, n, parts, partials);
+}
+
+template <bool kBf16>
+bool try_act_absmean(const void* X, int64_t T, int64_t K, const float* g, float eps, int8_t* Xq, float* sx,
+                     float* rinv, void* Xdq, const float* W, int64_t n, int parts, double* partials,
+                     cudaStream_t st) {
+    const int64_t nvec = K / (kBf16 ? 8 : 4);
+    if (nvec <= 32) launch_act_absmean<kBf16, 1>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
+    else if (nvec <= 64) launch_act_absmean<kBf16, 2>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
+    else if (nvec <= 128) launch_act_absmean<kBf16, 4>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
+    else if (nvec <= 256) launch_act_absmean<kBf16, 8>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
+    else return false;
+    return true;
 }
 size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
 
@@ -565,6 +595,51 @@ bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int64_t K, 
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
+    return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, x_dt, acc, st, dev);
+}
+
+bl_status bitlinear_forward_qat(const void* X, bl_dtype x_dt, int64_t T, int64_t K, const float* g, float eps,
+                                const float* W, int64_t N, int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                float* gamma, void* Y, int8_t* Xq, float* sx, float* rinv, void* Xdq, int32_t* acc,
+                                void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_dtype(x_dt));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", true));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Y, "Y", true));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(rinv, "rinv", true));
+    BL_TRY(check_ptr(Xdq, "Xdq", false));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_ptr(ws, "ws", true));
+    BL_TRY(check_dims(T, N, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
+    BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
+    BL_REQUIRE(ws_bytes >= quant_ws_bytes(), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu",
+               quant_ws_bytes(), ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = N * K;
+    const int parts = bl::wq_num_partials(n);
+    double* partials = static_cast<double*>(ws);
+    const bool fused = x_dt == BL_BF16
+                           ? try_act_absmean<true>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st)
+                           : try_act_absmean<false>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
+    if (fused) {
+        BL_TRY(launched("act_quant_absmean"));
+    } else {
+        pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
+        BL_TRY(launched("absmean_partial"));
+        BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
+    }
+    BL_TRY(run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev));
     return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, x_dt, acc, st, dev);
 }
 

@@ -34,15 +34,15 @@ __host__ __device__ inline int wq_num_partials(int64_t n) {
     return static_cast<int>(p);
 }
 
-__global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float* __restrict__ W, int64_t n,
-                                                                     double* __restrict__ partials) {
-    __shared__ double red[kWqThreads / 32];
-    pdl_trigger_and_wait();
+// Partial sum number `part` of `nparts` (256 threads, 4 float4 loads in flight per thread,
+// stride nparts * 256 vectors): the same slices whichever launch runs it.
+__device__ __forceinline__ void absmean_partial_block(const float* __restrict__ W, int64_t n, int part, int nparts,
+                                                      double* __restrict__ partials, double* red) {
     const int64_t nvec = n / 4;
     const float4* w4 = reinterpret_cast<const float4*>(W);
-    const int64_t stride = (int64_t)gridDim.x * kWqThreads;
+    const int64_t stride = (int64_t)nparts * kWqThreads;
     double acc = 0.0;
-    int64_t i = blockIdx.x * (int64_t)kWqThreads + threadIdx.x;
+    int64_t i = part * (int64_t)kWqThreads + threadIdx.x;
     // four independent loads in flight per thread
     for (; i + 3 * stride < nvec; i += 4 * stride) {
         float4 v[4];
@@ -69,8 +69,15 @@ __global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float
     if (threadIdx.x == 0) {
         double s = 0.0;
         for (int w = 0; w < kWqThreads / 32; ++w) s += red[w];
-        partials[blockIdx.x] = s;
+        partials[part] = s;
     }
+}
+
+__global__ void __launch_bounds__(kWqThreads) absmean_partial_kernel(const float* __restrict__ W, int64_t n,
+                                                                     double* __restrict__ partials) {
+    __shared__ double red[kWqThreads / 32];
+    pdl_trigger_and_wait();
+    absmean_partial_block(W, n, blockIdx.x, gridDim.x, partials, red);
 }
 
 __device__ __forceinline__ bool above_half(uint32_t bits, float gamma) {

@@ -140,6 +140,41 @@ def bitlinear_forward(X: torch.Tensor, wq_i8: torch.Tensor, gamma: torch.Tensor,
     return o
 
 
+def bitlinear_forward_qat(X: torch.Tensor, W: torch.Tensor, g: Optional[torch.Tensor] = None, eps: float = 1e-6,
+                          want_bf16: bool = True, want_packed: bool = True, want_acc: bool = False,
+                          want_xdq: bool = True, ws: Optional[torch.Tensor] = None, out=None):
+    """Quantisation-aware forward from the fp32 latent weight (weight and activation
+    quantisation, then the linear).  Returns dict(gamma, wq_i8, wq_bf16, packed, y, xq, sx,
+    rinv, xdq, acc) -- the union of bitlinear_quant_weight's and bitlinear_forward's."""
+    _cuda(X, "X")
+    _cuda(W, "W", torch.float32)
+    T, K = X.shape
+    N = W.shape[0]
+    dev = X.device
+    o = dict(out or {})
+    o.setdefault("gamma", torch.empty(1, dtype=torch.float32, device=dev))
+    o.setdefault("wq_i8", torch.empty(N, K, dtype=torch.int8, device=dev))
+    if want_bf16:
+        o.setdefault("wq_bf16", torch.empty(N, K, dtype=torch.bfloat16, device=dev))
+    if want_packed:
+        o.setdefault("packed", torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    o.setdefault("y", torch.empty(T, N, dtype=X.dtype, device=dev))
+    o.setdefault("xq", torch.empty(T, K, dtype=torch.int8, device=dev))
+    o.setdefault("sx", torch.empty(T, dtype=torch.float32, device=dev))
+    o.setdefault("rinv", torch.empty(T, dtype=torch.float32, device=dev))
+    if want_xdq:
+        o.setdefault("xdq", torch.empty(T, K, dtype=X.dtype, device=dev))
+    if want_acc:
+        o.setdefault("acc", torch.empty(T, N, dtype=torch.int32, device=dev))
+    if ws is None:
+        ws = workspace(T, N, K, dev)
+    _lib.call("bitlinear_forward_qat", X.data_ptr(), _dt(X), T, K, _ptr(g), float(eps), W.data_ptr(), N,
+              o["wq_i8"].data_ptr(), _ptr(o.get("wq_bf16")), _ptr(o.get("packed")), o["gamma"].data_ptr(),
+              o["y"].data_ptr(), o["xq"].data_ptr(), o["sx"].data_ptr(), o["rinv"].data_ptr(), _ptr(o.get("xdq")),
+              _ptr(o.get("acc")), ws.data_ptr(), ws.numel(), _stream(dev))
+    return o
+
+
 def bitlinear_backward_input(dY: torch.Tensor, X: torch.Tensor, rinv: torch.Tensor, wq_bf16: torch.Tensor,
                              gamma: torch.Tensor, g: Optional[torch.Tensor] = None, want_dg: bool = True,
                              ws: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,

@@ -168,6 +168,22 @@ BL_API bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int6
                             int32_t* acc, void* stream);
 
 /* ------------------------------------------------------------------------------
+ * Quantisation-aware forward from the fp32 latent weight: what P3 §3.1's BitLinear.forward
+ * computes (RMSNorm, activation_quant, weight_quant, then the linear), A1-A6 in three
+ * launches.  The activation quantiser and the weight quantiser's fp64 partial sums of |W|
+ * are independent and share one launch (for rows of <= 256 16-byte vectors: d_in <= 2048
+ * bf16 or 1024 fp32; longer rows take two launches), then the ternary codes, then the GEMM.
+ * Outputs: those of bitlinear_quant_weight (Wq_i8 required here -- the GEMM operand --,
+ * Wq_bf16 and Wpacked optional, gamma) and of bitlinear_forward; all bit-identical to
+ * bitlinear_quant_weight followed by bitlinear_forward.
+ * ws: at least bitlinear_workspace_bytes(T, N, K) bytes (no initialisation needed). */
+BL_API bl_status bitlinear_forward_qat(const void* X, bl_dtype x_dt, int64_t T, int64_t K,
+                                const float* g, float eps, const float* W, int64_t N,
+                                int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked, float* gamma,
+                                void* Y, int8_t* Xq, float* sx, float* rinv, void* Xdq,
+                                int32_t* acc, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------
  * Straight-through backward, input side (P3 §3.2; P5 §3.2 TernarySTE returns
  * grad_output unchanged; P4 §3.2 grad_w = grad_output), then the RMSNorm backward:
  *   dX_hat[t,k] = gamma * sum_n dY[t,n] * W_q[n,k]            (fp32 accumulation)

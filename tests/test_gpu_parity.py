@@ -223,6 +223,33 @@ def test_layer_parity(bl, T, K, N, dtype, gain):
     assert max_rel_err(np_(dg), dg_o) <= tol
 
 
+@pytest.mark.parametrize("T,K,N,dtype,gain", [
+    (7, 256, 144, "bf16", False),        # one launch for activations + |W| partials, ragged T
+    (129, 2048, 272, "bf16", True),      # longest row of the shared launch (256 vectors)
+    (300, 1024, 400, "f32", False),
+    (33, 4096, 160, "bf16", False),      # rows too long for the shared launch: two launches
+])
+def test_forward_qat_matches_separate_calls(bl, T, K, N, dtype, gain):
+    """bitlinear_forward_qat == bitlinear_quant_weight + bitlinear_forward, bit for bit, and
+    its codes / accumulators against the oracle."""
+    li = synth.random_case(T, K, N, seed=300 + T, dtype=dtype, with_gain=gain)
+    X, W = _gpu(li.X), _gpu(li.W)
+    g = None if li.g is None else _gpu(li.g)
+    fq = bl.bitlinear_forward_qat(X, W, g=g, want_acc=True)
+    qw = bl.bitlinear_quant_weight(W)
+    f = bl.bitlinear_forward(X, qw["wq_i8"], qw["gamma"], g=g, want_acc=True)
+    torch.cuda.synchronize()
+    for k in ("gamma", "wq_i8", "wq_bf16", "packed"):
+        assert torch.equal(fq[k], qw[k]), k
+    for k in ("y", "xq", "sx", "rinv", "xdq", "acc"):
+        assert torch.equal(fq[k], f[k]), k
+    g_gpu = float(fq["gamma"].item())
+    ref = oracle.forward(li.X, li.W, g=li.g, rinv=np_(fq["rinv"]), gamma=g_gpu, out_dtype=dtype)
+    assert np.array_equal(np_(fq["wq_i8"]), ref["wq"])
+    assert np.array_equal(np_(fq["xq"]), ref["xq"])
+    assert np.array_equal(np_(fq["acc"]), ref["acc"])
+
+
 @pytest.mark.parametrize("workload,layer", [("square", 0), ("mlp7b", 0), ("mlp7b", 1), ("layer7b", 0)])
 def test_workload_full_size(bl, workload, layer):
     """Full-size layers of the benchmark workloads (square 2048->2048 x 4096 tokens; the
