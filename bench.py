@@ -406,11 +406,13 @@ def main():
 
     dom_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     launches_before_capture = bl.launch_count()
-    graphs, replay = capture(None, dom_ev)
+    graphs, replay = capture(None)                 # the timed step: kernels only
     kernels_per_step = bl.launch_count() - launches_before_capture
-    graphs_pc, replay_pc = capture(gev)
+    graphs_dom, replay_dom = capture(None, dom_ev)  # the same step, events around the grad-input GEMM
+    graphs_pc, replay_pc = capture(gev)            # sequential, events between all calls
     for _ in range(max(3, args.warmup)):
         replay()
+        replay_dom()
         replay_pc()
     sync_all()
     assert bl.check_device_status() == 0
@@ -429,13 +431,20 @@ def main():
     if clk:
         clk.start()
         time.sleep(0.3)
-    dom_ms = []
     for i in range(K):
         flush.zero_()                       # evict L2 (outside the timed events)
         ev_s[i].record()
         replay()
         ev_e[i].record()
-        torch.cuda.synchronize()            # read this replay's grad-input GEMM time
+    sync_all()
+    # roofline: K more timed steps of the same work with two event nodes around the
+    # grad-input GEMM (event nodes cost the step its launch overlap at that point, so they
+    # stay out of the steps that give the value)
+    dom_ms = []
+    for i in range(K):
+        flush.zero_()
+        replay_dom()
+        torch.cuda.synchronize()
         dom_ms.append(dom_ev[0].elapsed_time(dom_ev[1]))
     sync_all()
     clocks = clk.stop() if clk else None
@@ -456,8 +465,29 @@ def main():
             pieces[p].append(gev[j].elapsed_time(gev[j + 1]))
     sync_all()
     piece_ms = {p: statistics.mean(v) for p, v in pieces.items()}
+    # the grad-input GEMM back to back (20 launches per graph, one event pair): its duration
+    # without an event node's lost launch overlap, reported beside the roofline
+    g_b2b = torch.cuda.CUDAGraph()
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        bl.bitlinear_grad_input(dY, bufs["wq_bf16"], bufs["gamma"], dXhat=bufs["dX"])
+    torch.cuda.current_stream(dev).wait_stream(side)
+    with torch.cuda.graph(g_b2b):
+        for _ in range(20):
+            bl.bitlinear_grad_input(dY, bufs["wq_bf16"], bufs["gamma"], dXhat=bufs["dX"])
+    g_b2b.replay()
+    b2b = []
+    for i in range(5):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g_b2b.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        b2b.append(e0.elapsed_time(e1) / 20)
+    b2b_ms = statistics.median(b2b)
     assert bl.check_device_status() == 0
-    del graphs, graphs_pc
+    del graphs, graphs_dom, graphs_pc, g_b2b
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -517,7 +547,10 @@ def main():
                     "grad_weight": "tc_gemm2_kernel<bf16,MN,MN,f32> (2-SM, 256x256)"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": ncu_traffic(dom), "kernel": kernel_names[dom], "peak_kind": peak_note,
-                "launch_ms": dom_ms}
+                "launch_ms": dom_ms,
+                "back_to_back": {"launch_ms": b2b_ms, "achieved": gemm_flops / (b2b_ms * 1e-3) / 1e12,
+                                 "frac": gemm_flops / (b2b_ms * 1e-3) / 1e12 / peak,
+                                 "how": "20 launches of the GEMM in one CUDA graph, one event pair, median of 5"}}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -536,9 +569,10 @@ def main():
         "e2e": e2e,
         "gpu_launches": int(launches),
         "timing": ("each step replays a CUDA graph of the step's library calls (RMSNorm backward and decode "
-                   "GEMV on a second stream beside the weight-gradient GEMM), event nodes only around the "
-                   "grad-input GEMM for the roofline; pieces_ms from a second, sequential graph with events "
-                   "between all calls, replayed after the timed steps; gpu_launches = kernels per step x steps"),
+                   "GEMV on a second stream beside the weight-gradient GEMM) with no event node inside; the "
+                   "roofline's grad-input GEMM time comes from K further timed steps of the same graph with "
+                   "two event nodes around that GEMM, and pieces_ms from a sequential graph with events "
+                   "between all calls; gpu_launches = kernels per step x steps"),
         "clocks": clocks,
         "pieces_ms": {k: round(v, 5) for k, v in piece_ms.items()},
         "gemm_tflops": {p: gemm_flops / (piece_ms[p] * 1e-3) / 1e12 for p in gemm_pieces},
