@@ -314,8 +314,7 @@ def main():
         b = bufs
         Wi, Xi, dYi = inputs if inputs is not None else (W, X, dY)
         main = torch.cuda.current_stream(dev)
-        # weight + activation quantisation and the forward GEMM (one shared launch for the
-        # activations and the |W| partial sums)
+        # weight + activation quantisation and the forward GEMM in one call
         bl.bitlinear_forward_qat(Xi, Wi, ws=b["ws"], out=b)
         if dom_ev is not None:
             dom_ev[0].record()

@@ -21,7 +21,6 @@
 #include "gemm_simt.cuh"
 #include "rmsnorm_bwd.cuh"
 #include "gemv.cuh"
-#include "fused_quant.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -392,28 +391,6 @@ bl_status run_quant_weight(const float* W, int64_t n, void* scratch, int8_t* Wq_
     return run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
 }
 
-// Activation quantisation and the |W| partial sums in one launch (rows of <= 256 vectors).
-template <bool kBf16, int VPL>
-void launch_act_absmean(const void* X, int64_t T, int64_t K, const float* g, float eps, int8_t* Xq, float* sx,
-                        float* rinv, void* Xdq, const float* W, int64_t n, int parts, double* partials,
-                        cudaStream_t st) {
-    const unsigned grid = (unsigned)(parts + (T + 7) / 8);
-    pdl_launch(bl::act_quant_absmean_kernel<kBf16, VPL>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, 1, g, eps,
-               Xq, sx, rinv, Xdq, W, n, parts, partials);
-}
-
-template <bool kBf16>
-bool try_act_absmean(const void* X, int64_t T, int64_t K, const float* g, float eps, int8_t* Xq, float* sx,
-                     float* rinv, void* Xdq, const float* W, int64_t n, int parts, double* partials,
-                     cudaStream_t st) {
-    const int64_t nvec = K / (kBf16 ? 8 : 4);
-    if (nvec <= 32) launch_act_absmean<kBf16, 1>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
-    else if (nvec <= 64) launch_act_absmean<kBf16, 2>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
-    else if (nvec <= 128) launch_act_absmean<kBf16, 4>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
-    else if (nvec <= 256) launch_act_absmean<kBf16, 8>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
-    else return false;
-    return true;
-}
 size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
 
 template <bool kBf16X, int VPT>
@@ -626,19 +603,15 @@ bl_status bitlinear_forward_qat(const void* X, bl_dtype x_dt, int64_t T, int64_t
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the |W| partial sums, the activation quantiser, then the ternary codes and the GEMM
+    // (a single launch for the first two measured no faster: the quantiser's occupancy
+    // limit throttled the partial-sum blocks)
     const int64_t n = N * K;
     const int parts = bl::wq_num_partials(n);
     double* partials = static_cast<double*>(ws);
-    const bool fused = x_dt == BL_BF16
-                           ? try_act_absmean<true>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st)
-                           : try_act_absmean<false>(X, T, K, g, eps, Xq, sx, rinv, Xdq, W, n, parts, partials, st);
-    if (fused) {
-        BL_TRY(launched("act_quant_absmean"));
-    } else {
-        pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
-        BL_TRY(launched("absmean_partial"));
-        BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
-    }
+    pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
+    BL_TRY(launched("absmean_partial"));
+    BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
     BL_TRY(run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev));
     return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, x_dt, acc, st, dev);
 }

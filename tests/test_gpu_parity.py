@@ -224,10 +224,10 @@ def test_layer_parity(bl, T, K, N, dtype, gain):
 
 
 @pytest.mark.parametrize("T,K,N,dtype,gain", [
-    (7, 256, 144, "bf16", False),        # one launch for activations + |W| partials, ragged T
-    (129, 2048, 272, "bf16", True),      # longest row of the shared launch (256 vectors)
+    (7, 256, 144, "bf16", False),        # ragged T
+    (129, 2048, 272, "bf16", True),      # longest row of the warp-per-row quantiser (256 vectors)
     (300, 1024, 400, "f32", False),
-    (33, 4096, 160, "bf16", False),      # rows too long for the shared launch: two launches
+    (33, 4096, 160, "bf16", False),      # block-per-row quantiser
 ])
 def test_forward_qat_matches_separate_calls(bl, T, K, N, dtype, gain):
     """bitlinear_forward_qat == bitlinear_quant_weight + bitlinear_forward, bit for bit, and
