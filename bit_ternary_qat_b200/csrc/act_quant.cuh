@@ -78,38 +78,41 @@ struct DqLut<false> {
 };
 
 // Quantise one vector of E values of x_hat with scale s and store its codes (E int8) and,
-// when wanted, its dequantised values from the row's table; elements are handled in pairs
-// so few values are live at once.
-__device__ __forceinline__ int quant_code(float h, float s) {
-    const float tq = __fadd_rn(__fmul_rn(h, s), kRoundMagic);   // 1.5*2^23 + rint(x_hat*s)
-    return max(-128, min(127, __float_as_int(tq) - kRoundMagicBits));
+// when wanted, its dequantised values from the row's table.  With tq = fl(fl(x_hat s) +
+// 1.5*2^23) = 1.5*2^23 + q (q = rint(x_hat s), |q| <= 127 for finite inputs), the low byte
+// of tq's bits is q mod 256 -- the int8 code itself -- because 1.5*2^23's low byte is zero;
+// the table index is that byte with its top bit flipped (q + 128).  So codes need no
+// integer conversion, no clamp and no shift: three byte permutes gather four codes.
+__device__ __forceinline__ uint32_t quant_bits(float h, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(h, s), kRoundMagic));   // 1.5*2^23 + rint(x_hat*s)
+}
+__device__ __forceinline__ uint32_t lut_index(uint32_t tq_bits) { return (tq_bits & 0xFFu) ^ 0x80u; }
+__device__ __forceinline__ uint32_t gather_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 template <bool kBf16, int E>
 __device__ __forceinline__ void quant_store_vec(const float (&h)[E], float s, int8_t* Xq, void* Xdq, int64_t vec,
                                                 const typename DqLut<kBf16>::T* lut) {
-    uint32_t cw[E / 4];
-    uint32_t o[E / 2];
+    uint32_t tb[E];
 #pragma unroll
-    for (int w = 0; w < E / 4; ++w) cw[w] = 0u;
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i) {
-        const int q0 = quant_code(h[2 * i], s), q1 = quant_code(h[2 * i + 1], s);
-        cw[i >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
-                      << (16 * (i & 1));
-        if (Xdq != nullptr) {
-            if constexpr (kBf16)
-                o[i] = static_cast<uint32_t>(lut[q0 + 128]) | (static_cast<uint32_t>(lut[q1 + 128]) << 16);
-            else
-                o[i] = 0u, reinterpret_cast<float*>(Xdq)[vec * E + 2 * i] = lut[q0 + 128],
-                reinterpret_cast<float*>(Xdq)[vec * E + 2 * i + 1] = lut[q1 + 128];
-        }
-    }
+    for (int e = 0; e < E; ++e) tb[e] = quant_bits(h[e], s);
     if constexpr (kBf16) {
-        reinterpret_cast<uint2*>(Xq)[vec] = make_uint2(cw[0], cw[1]);
-        if (Xdq != nullptr) reinterpret_cast<uint4*>(Xdq)[vec] = make_uint4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<uint2*>(Xq)[vec] =
+            make_uint2(gather_low_bytes(tb[0], tb[1], tb[2], tb[3]), gather_low_bytes(tb[4], tb[5], tb[6], tb[7]));
+        if (Xdq != nullptr) {
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                o[i] = static_cast<uint32_t>(lut[lut_index(tb[2 * i])]) |
+                       (static_cast<uint32_t>(lut[lut_index(tb[2 * i + 1])]) << 16);
+            reinterpret_cast<uint4*>(Xdq)[vec] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     } else {
-        reinterpret_cast<uint32_t*>(Xq)[vec] = cw[0];
+        reinterpret_cast<uint32_t*>(Xq)[vec] = gather_low_bytes(tb[0], tb[1], tb[2], tb[3]);
+        if (Xdq != nullptr)
+            reinterpret_cast<float4*>(Xdq)[vec] = make_float4(lut[lut_index(tb[0])], lut[lut_index(tb[1])],
+                                                              lut[lut_index(tb[2])], lut[lut_index(tb[3])]);
     }
 }
 
@@ -248,7 +251,8 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
         }
         const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
         // codes and dequantised values.  |x_hat * s| <= 127 * (1 + 2^-23) for finite inputs,
-        // so rint(x_hat * s) is in [-127, 127]; the integer clamp is kept for robustness.
+        // so rint(x_hat * s) is in [-127, 127] (no clamp needed; a non-finite input still
+        // gives an in-range table index).
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
             const int v = threadIdx.x + j * NT;

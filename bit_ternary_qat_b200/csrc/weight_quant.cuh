@@ -145,7 +145,7 @@ __device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int6
 // grid * kWqThreads * kTqGroups groups are handled in further rounds of the same kind.
 constexpr int kTqGroups = 2;
 
-__global__ void __launch_bounds__(kWqThreads) ternary_quant_kernel(
+__global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     const float* __restrict__ W, int64_t n, const double* __restrict__ partials, int nparts,
     int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
     float* __restrict__ gamma_out) {

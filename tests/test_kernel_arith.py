@@ -152,3 +152,30 @@ def test_gemv_field_identity():
         assert all(D[j] % (4 ** j) == 0 for j in range(4))
         got = sum(D[j] >> (2 * j) for j in range(4)) - 2 * int(np.sum(x))
         assert got == ref
+
+
+def _byte_perm(a: int, b: int, sel: int) -> int:
+    """CUDA __byte_perm: byte i of the result is byte (sel >> 4i) & 7 of the 8-byte value b:a."""
+    x = (b << 32) | a
+    out = 0
+    for i in range(4):
+        k = (sel >> (4 * i)) & 7
+        out |= ((x >> (8 * k)) & 0xFF) << (8 * i)
+    return out
+
+
+def test_codes_from_rounding_sum_bits():
+    """The activation quantiser reads the int8 code off the low byte of
+    fl(v + 1.5*2^23) and the table index off that byte with bit 7 flipped."""
+    magic = np.float32(1.5 * 2 ** 23)
+    for q in range(-127, 128):
+        for frac in (0.0, 0.25, -0.25, 0.5 if q % 2 == 0 else 0.0):
+            v = np.float32(q + frac)
+            t = np.float32(v + magic)                   # fp32 addition, round to nearest even
+            bits = int(np.array([t], dtype=np.float32).view(np.uint32)[0])
+            assert (bits & 0xFF) == (q & 0xFF)
+            assert ((bits & 0xFF) ^ 0x80) == q + 128
+    # gathering the low bytes of four words into one
+    words = [0x4B4000FB, 0x4B400005, 0x4B3FFF80, 0x4B40007F]
+    got = _byte_perm(_byte_perm(words[0], words[1], 0x0040), _byte_perm(words[2], words[3], 0x0040), 0x5410)
+    assert got == 0x7F8005FB
