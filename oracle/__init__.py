@@ -69,6 +69,11 @@ def lib():
             L.ora_grad_weight.argtypes = [P, P, I, I, I, P, I, P]
             L.ora_rmsnorm_backward.argtypes = [P, P, P, P, I, I, P, I, P, P]
             L.ora_gemv.argtypes = [P, F, I, I, P, P, I, P, P]
+            L.ora_absmean_gamma_rows.argtypes = [P, I, I, P]
+            L.ora_ternary_round_rows.argtypes = [P, I, I, P, P]
+            L.ora_ternary_tau.argtypes = [P, I, F, F, P]
+            L.ora_act_quant_tensor.argtypes = [P, I, I, P, P, P, P, P]
+            L.ora_linear_epilogue_rows.argtypes = [P, I, I, P, P, P]
             _lib = L
     return _lib
 
@@ -260,6 +265,66 @@ def gemv(packed, gamma: float, K: int, xq, s):
     y = np.empty((B, N), dtype=np.float32)
     lib().ora_gemv(_p(packed), float(gamma), N, K, _p(xq), _p(s), B, _p(acc), _p(y))
     return acc, y
+
+
+# ----------------------------------------------------------------------------------
+# page variants of the quantisers (P4 §9 per-row scale, P2 tau = 0.7 scale, P5 §5.1
+# per-tensor activation scale)
+# ----------------------------------------------------------------------------------
+
+def absmean_gamma_rows(W) -> np.ndarray:
+    """gamma_n = max(mean_k |W[n, k]|, 1e-5), fp64 sum per row."""
+    W = _f32(W)
+    N, K = W.shape
+    g = np.empty(N, dtype=np.float32)
+    lib().ora_absmean_gamma_rows(_p(W), N, K, _p(g))
+    return g
+
+
+def ternary_round_rows(W, gamma_rows) -> np.ndarray:
+    W = _f32(W)
+    N, K = W.shape
+    g = _f32(gamma_rows)
+    out = np.empty((N, K), dtype=np.int8)
+    lib().ora_ternary_round_rows(_p(W), N, K, _p(g), _p(out))
+    return out
+
+
+def quant_weight_rows(W):
+    """(gamma_rows fp32 [N], W_q int8 [N, K])."""
+    g = absmean_gamma_rows(W)
+    return g, ternary_round_rows(W, g)
+
+
+def ternary_tau(W, gamma: float, tau_factor: float) -> np.ndarray:
+    """W_q = 0 where |W| < fl32(tau_factor * gamma), sign(W) elsewhere."""
+    W = _f32(W)
+    out = np.empty(W.shape, dtype=np.int8)
+    lib().ora_ternary_tau(_p(W), W.size, float(gamma), float(tau_factor), _p(out))
+    return out
+
+
+def act_quant_tensor(X, rinv=None, g=None):
+    """Per-tensor scale: (x_q int8 [T,K], s fp32 [T] (one value repeated), x_dq fp32 [T,K])."""
+    X = _f32(X)
+    T, K = X.shape
+    r = None if rinv is None else _f32(rinv)
+    gg = None if g is None else _f32(g)
+    xq = np.empty((T, K), dtype=np.int8)
+    s = np.empty(T, dtype=np.float32)
+    xdq = np.empty((T, K), dtype=np.float32)
+    lib().ora_act_quant_tensor(_p(X), T, K, _p(r), _p(gg), _p(xq), _p(s), _p(xdq))
+    return xq, s, xdq
+
+
+def linear_epilogue_rows(acc, gamma_rows, s_rows) -> np.ndarray:
+    acc = _arr(acc, np.int32)
+    g = _f32(gamma_rows)
+    s_rows = _f32(s_rows)
+    R, N = acc.shape
+    y = np.empty((R, N), dtype=np.float32)
+    lib().ora_linear_epilogue_rows(_p(acc), R, N, _p(g), _p(s_rows), _p(y))
+    return y
 
 
 # ----------------------------------------------------------------------------------

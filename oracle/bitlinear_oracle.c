@@ -348,3 +348,92 @@ void ora_gemv(const uint8_t* packed, float gamma, int64_t N, int64_t K, const in
 void ora_bf16_to_f32(const uint16_t* in, int64_t n, float* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = bf16_bits_to_f32(in[i]);
 }
+
+/* =================================================================================
+ * Variants the pages print beside the b1.58 defaults (cheap parameterisations of the
+ * two quantisers).  Same arithmetic conventions as above.
+ * ================================================================================= */
+
+/* Per-row weight scale (P4 §9 "Quantizer": scale = mean(|x|, dim=1, keepdim=True), one
+ * scale per output row), combined with the b1.58 round/clamp of P3 §2.1 / P5 §2.2:
+ *   gamma_n   = max( (float)( sum_k |W[n,k]| / K ), 1e-5 )      fp64 sum, index order
+ *   W_q[n,k]  = clamp(round(fl32(W[n,k] / gamma_n)), -1, 1). */
+void ora_absmean_gamma_rows(const float* W, int64_t N, int64_t K, float* gamma) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        double S = 0.0;
+        for (int64_t k = 0; k < K; ++k) S += (double)fabsf(W[n * K + k]);
+        float mean = (float)(S / (double)K);
+        gamma[n] = fmaxf(mean, 1e-5f);
+    }
+}
+
+void ora_ternary_round_rows(const float* W, int64_t N, int64_t K, const float* gamma, int8_t* wq) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float v = nearbyintf(W[n * K + k] / gamma[n]);
+            if (v < -1.0f) v = -1.0f;
+            if (v > 1.0f) v = 1.0f;
+            wq[n * K + k] = (int8_t)v;
+        }
+}
+
+/* Zero threshold (P2 "直通估计器在三元权重量化中的作用": tau = 0.7 * scale, |W| < tau
+ * quantises to 0; the other weights keep their sign), with the per-tensor gamma:
+ *   tau = fl32(tau_factor * gamma);   W_q = 0 if |W| < tau, else sign(W) (sign(0) = 0). */
+void ora_ternary_tau(const float* W, int64_t n, float gamma, float tau_factor, int8_t* wq) {
+    float tau = tau_factor * gamma;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(W[i]);
+        wq[i] = (int8_t)(a < tau ? 0 : (W[i] > 0.0f) - (W[i] < 0.0f));
+    }
+}
+
+/* Per-tensor activation scale (P5 §5.1 quantize_activation: scale = 127 / max|x| over the
+ * whole tensor), applied to x_hat as in ora_act_quant, with the same 1e-5 floor and clamp:
+ *   s = fl32(127 / max(max_{t,k} |x_hat|, 1e-5)),  q = clamp(round(fl32(x_hat s)), -128, 127),
+ *   X_dq = fl32(q / s).  s_out receives s for every token (one value repeated). */
+void ora_act_quant_tensor(const float* X, int64_t T, int64_t K, const float* rinv, const float* g,
+                          int8_t* xq, float* s_out, float* xdq) {
+    float m = 0.0f;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t k = 0; k < K; ++k) {
+            float v = X[t * K + k];
+            if (rinv) {
+                v = v * rinv[t];
+                if (g) v = v * g[k];
+            }
+            float a = fabsf(v);
+            if (a > m) m = a;
+        }
+    float s = 127.0f / fmaxf(m, 1e-5f);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        s_out[t] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = X[t * K + k];
+            if (rinv) {
+                v = v * rinv[t];
+                if (g) v = v * g[k];
+            }
+            float r = nearbyintf(v * s);
+            if (r < -128.0f) r = -128.0f;
+            if (r > 127.0f) r = 127.0f;
+            int8_t q = (int8_t)r;
+            xq[t * K + k] = q;
+            if (xdq) xdq[t * K + k] = (float)q / s;
+        }
+    }
+}
+
+/* Output rescale with a per-row weight scale: y[t, n] = fl32( (float)acc[t, n] * fl32(gamma_n / s_t) ). */
+void ora_linear_epilogue_rows(const int32_t* acc, int64_t R, int64_t N, const float* gamma,
+                              const float* s_rows, float* y) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t n = 0; n < N; ++n) {
+            float c = gamma[n] / s_rows[r];
+            y[r * N + n] = (float)acc[r * N + n] * c;
+        }
+}
