@@ -74,6 +74,9 @@ def lib():
             L.ora_ternary_tau.argtypes = [P, I, F, F, P]
             L.ora_act_quant_tensor.argtypes = [P, I, I, P, P, P, P, P]
             L.ora_linear_epilogue_rows.argtypes = [P, I, I, P, P, P]
+            D = ctypes.c_double
+            L.ora_optimizer_step.argtypes = [P, P, P, P, I, D, D, D, D, D, D, I]
+            L.ora_optimizer_step.restype = D
             _lib = L
     return _lib
 
@@ -325,6 +328,23 @@ def linear_epilogue_rows(acc, gamma_rows, s_rows) -> np.ndarray:
     y = np.empty((R, N), dtype=np.float32)
     lib().ora_linear_epilogue_rows(_p(acc), R, N, _p(g), _p(s_rows), _p(y))
     return y
+
+
+# ----------------------------------------------------------------------------------
+# optimizer step: clip -> AdamW -> clamp (returns new arrays; the inputs are untouched)
+# ----------------------------------------------------------------------------------
+
+def optimizer_step(W, dW, m, v, t: int, lr: float = 1e-3, betas=(0.9, 0.95), eps: float = 1e-6,
+                   weight_decay: float = 0.01, max_norm: float = 1.0):
+    """(W', m', v', c) after step t (1-based); c is the clip coefficient applied to dW."""
+    W2 = _f32(W).copy()
+    m2 = _f32(m).copy()
+    v2 = _f32(v).copy()
+    g = _f32(dW)
+    assert W2.shape == g.shape == m2.shape == v2.shape
+    c = lib().ora_optimizer_step(_p(W2), _p(g), _p(m2), _p(v2), W2.size, float(lr), float(betas[0]),
+                                 float(betas[1]), float(eps), float(weight_decay), float(max_norm), int(t))
+    return W2, m2, v2, float(c)
 
 
 # ----------------------------------------------------------------------------------

@@ -437,3 +437,47 @@ void ora_linear_epilogue_rows(const int32_t* acc, int64_t R, int64_t N, const fl
             y[r * N + n] = (float)acc[r * N + n] * c;
         }
 }
+
+/* =================================================================================
+ * Optimizer step of the latent weight, in the order the pages give it: gradient
+ * clipping to a maximum L2 norm (P5 §6.2: clip_grad_norm_ per weight matrix with
+ * max_norm 1.0; P3 §6 and P4 §4.1 the same threshold over the model), then AdamW
+ * (P2 training pipeline: AdamW; hyper-parameters lr 1e-3, betas (0.9, 0.95), weight decay
+ * 0.01, eps 1e-6 from the optimizer configuration of the 1-bit training guide), then
+ * the clamp of the latent weight to [-1, 1] (same guide, section on gradient clipping
+ * and weight constraints).  AdamW is the decoupled-weight-decay algorithm of Loshchilov
+ * and Hutter with bias-corrected moments:
+ *   norm = sqrt(sum_i dW_i^2);  c = min(1, max_norm / (norm + 1e-6))   (c = 1 if max_norm <= 0)
+ *   g = c dW;  W <- W - lr wd W;  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
+ *   W <- W - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps);  W <- clamp(W, -1, 1)
+ * All arithmetic in fp64 from the fp32 inputs; W, m, v are stored back rounded to fp32.
+ * t is the 1-based index of this step.  Returns c.
+ * --------------------------------------------------------------------------------- */
+double ora_optimizer_step(float* W, const float* dW, float* m, float* v, int64_t n, double lr, double beta1,
+                          double beta2, double eps, double wd, double max_norm, int64_t t) {
+    double S = 0.0;
+    for (int64_t i = 0; i < n; ++i) S += (double)dW[i] * (double)dW[i];
+    double norm = sqrt(S);
+    double c = 1.0;
+    if (max_norm > 0.0) {
+        c = max_norm / (norm + 1e-6);
+        if (c > 1.0) c = 1.0;
+    }
+    double bc1 = 1.0 - pow(beta1, (double)t);
+    double bc2 = 1.0 - pow(beta2, (double)t);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double g = c * (double)dW[i];
+        double w = (double)W[i];
+        w = w - lr * wd * w;
+        double mi = beta1 * (double)m[i] + (1.0 - beta1) * g;
+        double vi = beta2 * (double)v[i] + (1.0 - beta2) * g * g;
+        w = w - lr * (mi / bc1) / (sqrt(vi / bc2) + eps);
+        if (w < -1.0) w = -1.0;
+        if (w > 1.0) w = 1.0;
+        W[i] = (float)w;
+        m[i] = (float)mi;
+        v[i] = (float)vi;
+    }
+    return c;
+}
