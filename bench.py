@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
+    ap.add_argument("--next", action="store_true",
+                    help="time the fused optimizer step and the quantiser variants back to back; one JSON object, "
+                         "not the bench line")
     ap.add_argument("--table", action="store_true",
                     help="time every configuration's full step (single, square, mlp7b, layer7b, decode) and the "
                          "oracle on a bounded sample of each; one JSON object, not the bench line")
@@ -234,11 +237,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if args.only_gemv or args.table:
+    if args.only_gemv or args.table or args.next:
         blbuild.build()
         bl.load()
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        if args.table:
+        if args.next:
+            print(json.dumps({"next": next_measure(bl, torch, dev, flush, peaks())}), flush=True)
+        elif args.table:
             print(json.dumps({"table": table_measure(bl, torch, dev, flush, peaks())}), flush=True)
         else:
             print(json.dumps({"decode_gemv": gemv_measure(bl, torch, dev, flush, peaks())}), flush=True)
@@ -631,6 +636,115 @@ def gemv_measure(bl, torch, dev, flush, pk):
     out["hbm_peak_GBs"] = pk["hbm"]
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
                        "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5")
+    return out
+
+
+def next_measure(bl, torch, dev, flush, pk):
+    """The fused optimizer step and the quantiser variants, each launched `reps` times back to
+    back in one CUDA graph between one pair of CUDA events (median of 5, L2 flushed before each
+    replay).  Every input set is larger than the 126 MB L2 or cycled over copies that are.
+    Bytes are algorithmic: each tensor read once and each output written once."""
+    from bit_ternary_qat_b200 import synth
+    out = {}
+
+    def timed(calls, reps):
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(reps):
+                calls[i % len(calls)]()
+        graph.replay()
+        torch.cuda.synchronize()
+        samples = []
+        for _ in range(5):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            samples.append(a.elapsed_time(b) / reps)
+        del graph
+        assert bl.check_device_status() == 0
+        return statistics.median(samples) * 1e3
+
+    def hbm_row(us, nbytes, note):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": us, "GB/s": gbs, "frac_hbm": gbs / pk["hbm"], "bytes": nbytes, "note": note}
+
+    gen = synth.generator(77)
+    # optimizer step: 7B-MLP-shaped weight (4 x 180 MB of fp32 state), and the square weight
+    # cycled over 4 copies (4 x 67 MB)
+    for name, (N, K), copies in (("optimizer_11008x4096", (11008, 4096), 1), ("optimizer_2048x2048", (2048, 2048), 4)):
+        n = N * K
+        sets = []
+        for _ in range(copies):
+            W = synth.normal((N, K), 0.3, gen).clamp_(-1, 1).to(dev)
+            sets.append(dict(W=W, dW=synth.normal((N, K), 1e-3, gen).to(dev), m=torch.zeros_like(W),
+                             v=torch.zeros_like(W), step=torch.zeros(1, dtype=torch.int32, device=dev),
+                             q=dict(gamma=torch.empty(1, dtype=torch.float32, device=dev),
+                                    wq_i8=torch.empty(N, K, dtype=torch.int8, device=dev),
+                                    wq_bf16=torch.empty(N, K, dtype=torch.bfloat16, device=dev),
+                                    packed=torch.empty(N, K // 4, dtype=torch.uint8, device=dev))))
+        ws = bl.workspace(1, N, K, dev)
+        for requant in (True, False):
+            calls = [(lambda S=S, rq=requant: bl.bitlinear_optimizer_step(
+                S["W"], S["dW"], S["m"], S["v"], S["step"], requantize=rq, ws=ws, out=S["q"] if rq else None))
+                for S in sets]
+            us = timed(calls, 8)
+            per = 31.25 if requant else 28.0
+            out[name + ("_requantize" if requant else "")] = hbm_row(
+                us, n * per, f"reads dW, W, m, v; writes W, m, v{', int8 + bf16 + 2-bit codes' if requant else ''} "
+                             f"({per} B per weight); {copies} state cop{'ies' if copies > 1 else 'y'}")
+        del sets, ws
+        torch.cuda.empty_cache()
+
+    # weight quantisers on the 11008 x 4096 fp32 weight (180 MB): default, per-row, tau = 0.7
+    N, K = 11008, 4096
+    W = synth.student_t3((N, K), 0.02, gen).to(dev)
+    ws = bl.workspace(1, N, K, dev)
+    q = dict(gamma=torch.empty(1, dtype=torch.float32, device=dev),
+             wq_i8=torch.empty(N, K, dtype=torch.int8, device=dev),
+             wq_bf16=torch.empty(N, K, dtype=torch.bfloat16, device=dev),
+             packed=torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    qr = dict(q, gamma_rows=torch.empty(N, dtype=torch.float32, device=dev))
+    nb = N * K * 7.25
+    out["quant_weight_11008x4096"] = hbm_row(timed([lambda: bl.bitlinear_quant_weight(W, ws=ws, out=q)], 8), nb,
+                                             "per-tensor gamma (two launches)")
+    out["quant_weight_rows_11008x4096"] = hbm_row(timed([lambda: bl.bitlinear_quant_weight_rows(W, out=qr)], 8), nb,
+                                                  "per-row gamma (one launch)")
+    out["quant_weight_tau_11008x4096"] = hbm_row(
+        timed([lambda: bl.bitlinear_quant_weight_tau(W, 0.7, ws=ws, out=q)], 8), nb, "tau = 0.7 gamma (two launches)")
+    wq_i8 = q["wq_i8"]
+    del W
+    # activation quantisers on X [8192 x 11008] bf16 (180 MB), RMSNorm fused, X_dq written
+    T = 8192
+    X = synth.normal((T, 11008), 1.0, gen).to(torch.bfloat16).to(dev)
+    a = dict(xq=torch.empty(T, 11008, dtype=torch.int8, device=dev), sx=torch.empty(T, device=dev),
+             rinv=torch.empty(T, device=dev), xdq=torch.empty(T, 11008, dtype=torch.bfloat16, device=dev))
+    wsa = bl.workspace(T, 16, 11008, dev)
+    nb = T * 11008 * 5 + T * 8
+    out["act_quant_8192x11008"] = hbm_row(timed([lambda: bl.bitlinear_act_quant(X, out=a)], 8), nb,
+                                          "per-token scale (one launch)")
+    out["act_quant_tensor_8192x11008"] = hbm_row(
+        timed([lambda: bl.bitlinear_act_quant_tensor(X, ws=wsa, out=a)], 8), nb,
+        "per-tensor scale (two launches; X read twice)")
+    del X, a
+    # int8 GEMM with the per-tensor and the per-row epilogue: 8192 tokens, 4096 -> 11008
+    xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev)
+    sx = torch.full((T,), 50.0, device=dev)
+    gr = torch.rand(N, device=dev) * 0.02 + 0.01
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    ops = 2.0 * T * N * K
+    us_t = timed([lambda: bl.bitlinear_linear(xq, sx, wq_i8, q["gamma"], y=y)], 10)
+    us_r = timed([lambda: bl.bitlinear_linear_rows(xq, sx, wq_i8, gr, y=y)], 10)
+    out["linear_8192x4096x11008"] = {"us": us_t, "TOPS": ops / (us_t * 1e-6) / 1e12, "note": "gamma / s_t epilogue"}
+    out["linear_rows_8192x4096x11008"] = {"us": us_r, "TOPS": ops / (us_r * 1e-6) / 1e12,
+                                          "note": "fl(gamma_n / s_t) per element epilogue"}
+    out["hbm_peak_GBs"] = pk["hbm"]
     return out
 
 

@@ -378,6 +378,115 @@ __global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __re
     act_quant_warp_rows<kBf16, VPL>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, blockIdx.x, lut_all);
 }
 
+// ------------------------------------------------------------------------------------
+// Per-tensor activation scale (P5 §5.1 quantize_activation: one scale 127 / max|x| over the
+// whole tensor), applied to x_hat with the same 1e-5 floor, rounding and clamp as above.
+// Two launches over one warp per row, 8 rows per block, a grid of at most kActMaxPartials
+// blocks looping over row groups:
+//   pass 1  r_t and max |x_hat| of every row; block maxima -> partials[blockIdx];
+//   pass 2  every block takes the max of the partials (max is exact in any order), builds
+//           one table of fl(q / s) and quantises its rows again with the shared s.
+// X is read twice (the second read hits L2 when X fits there).
+// ------------------------------------------------------------------------------------
+constexpr int kActMaxPartials = 1184;
+
+template <bool kBf16>
+__device__ __forceinline__ float act_xhat(const uint4& raw, int e, int v, float r, int apply_norm,
+                                          const float* __restrict__ g) {
+    float h = ActVec<kBf16>::elem(raw, e);
+    if (apply_norm) {
+        h = __fmul_rn(h, r);
+        if (g != nullptr) h = __fmul_rn(h, __ldg(g + v * ActVec<kBf16>::kElems + e));
+    }
+    return h;
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) act_tensor_max_kernel(const void* __restrict__ X, int T, int K, int apply_norm,
+                                                             const float* __restrict__ g, float eps,
+                                                             float* __restrict__ rinv, float* __restrict__ partials) {
+    constexpr int E = ActVec<kBf16>::kElems;
+    __shared__ float red[8];
+    pdl_trigger_and_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = K / E;
+    float m = 0.0f;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp; t < T; t += static_cast<int64_t>(gridDim.x) * 8) {
+        const uint4* xrow = reinterpret_cast<const uint4*>(X) + t * nvec;
+        float r = 1.0f;
+        if (apply_norm) {
+            double ss = 0.0;
+            for (int v = lane; v < nvec; v += 32) {
+                const uint4 raw = __ldg(xrow + v);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const double xd = static_cast<double>(ActVec<kBf16>::elem(raw, e));
+                    ss = fma(xd, xd, ss);
+                }
+            }
+            ss = warp_sum(ss);
+            r = static_cast<float>(1.0 / sqrt(ss / static_cast<double>(K) + static_cast<double>(eps)));
+            if (lane == 0) rinv[t] = r;
+        }
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 raw = __ldg(xrow + v);
+#pragma unroll
+            for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(act_xhat<kBf16>(raw, e, v, r, apply_norm, g)));
+        }
+    }
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) b = fmaxf(b, red[w]);
+        partials[blockIdx.x] = b;
+    }
+}
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256) act_tensor_quant_kernel(const void* __restrict__ X, int T, int K,
+                                                               int apply_norm, const float* __restrict__ g,
+                                                               const float* __restrict__ partials, int nparts,
+                                                               int8_t* __restrict__ Xq, float* __restrict__ sx,
+                                                               const float* __restrict__ rinv,
+                                                               void* __restrict__ Xdq) {
+    constexpr int E = ActVec<kBf16>::kElems;
+    using LutT = typename DqLut<kBf16>::T;
+    __shared__ float red[8];
+    __shared__ LutT lut[256];
+    pdl_trigger_and_wait();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < nparts; i += 256) m = fmaxf(m, partials[i]);
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+    const float s = __fdiv_rn(127.0f, fmaxf(m, 1e-5f));
+    if (Xdq != nullptr) {
+        const float c = __frcp_rn(s);
+        lut[threadIdx.x] = DqLut<kBf16>::make(div_by_scale(static_cast<float>(static_cast<int>(threadIdx.x) - 128), s, c));
+        __syncthreads();
+    }
+    const int nvec = K / E;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp; t < T; t += static_cast<int64_t>(gridDim.x) * 8) {
+        const uint4* xrow = reinterpret_cast<const uint4*>(X) + t * nvec;
+        const float r = apply_norm ? __ldg(rinv + t) : 1.0f;
+        if (lane == 0) sx[t] = s;
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 raw = __ldg(xrow + v);
+            float h[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) h[e] = act_xhat<kBf16>(raw, e, v, r, apply_norm, g);
+            quant_store_vec<kBf16, E>(h, s, Xq, Xdq, t * nvec + v, lut);
+        }
+    }
+}
+
 // Largest row (elements) the register-resident kernel handles: 16 vectors per thread.
 constexpr int kActMaxVpt = 16;
 template <bool kBf16>

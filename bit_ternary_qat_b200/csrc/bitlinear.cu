@@ -21,6 +21,7 @@
 #include "gemm_simt.cuh"
 #include "rmsnorm_bwd.cuh"
 #include "gemv.cuh"
+#include "optim.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -326,6 +327,25 @@ bl_status run_linear(const int8_t* Xq, const float* sx, int64_t T, int64_t K, co
     return launch_tc<true, false, false, bl::kEpiLinearF32>(ta, tb, td, a, st, dev);
 }
 
+// Per-column scales gamma_n: the 2-SM kernel at every T (its rows past T are zero-filled
+// loads and clipped stores).
+bl_status run_linear_rows(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq,
+                          const float* gamma_rows, int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, cudaStream_t st,
+                          const DeviceInfo& dev) {
+    CUtensorMap ta, tb, td;
+    BL_TRY(make_tmap(&ta, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, 128));
+    BL_TRY(make_tmap(&tb, Wq, kTmU8, (uint64_t)K, (uint64_t)N, 128, 128));
+    bl::TcGemmArgs a{};
+    a.M = (int)T; a.N = (int)N; a.K = (int)K;
+    a.acc_out = acc; a.row_scale = sx; a.gamma = gamma_rows;
+    if (y_dt == BL_BF16) {
+        BL_TRY(make_tmap(&td, Y, kTmBf16, (uint64_t)N, (uint64_t)T, 64, 32));
+        return launch_tc2<true, false, false, bl::kEpiLinearColBf16>(ta, tb, td, a, st, dev);
+    }
+    BL_TRY(make_tmap(&td, Y, kTmF32, (uint64_t)N, (uint64_t)T, 32, 32));
+    return launch_tc2<true, false, false, bl::kEpiLinearColF32>(ta, tb, td, a, st, dev);
+}
+
 bl_status run_grad_input_gemm(const void* dY, bl_dtype dt, const uint16_t* Wq_bf16, const float* gamma, int64_t T,
                               int64_t K, int64_t N, float* dXhat, cudaStream_t st, const DeviceInfo& dev) {
     if (dt == BL_BF16) {
@@ -369,27 +389,40 @@ size_t quant_ws_bytes() { return sizeof(double) * bl::kWqMaxPartials; }
 
 // Weight quantiser pass 2: gamma, threshold and codes (one round of kTqGroups groups per
 // thread when the grid covers W).
+// tau_factor < 0: the round/clamp threshold; else the zero threshold fl32(tau_factor * gamma).
 bl_status run_ternary(const float* W, int64_t n, const double* partials, int parts, int8_t* Wq_i8, uint16_t* Wq_bf16,
-                      uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev) {
+                      uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev,
+                      float tau_factor = -1.0f) {
     const int64_t groups = n / 16;
     const int64_t per_block = (int64_t)bl::kWqThreads * bl::kTqGroups;
     int64_t blocks = (groups + per_block - 1) / per_block;
     const int64_t cap = (int64_t)dev.sms * 4;
     if (blocks > cap) blocks = cap;
-    pdl_launch(bl::ternary_quant_kernel, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n, partials, parts,
-               Wq_i8, Wq_bf16, Wpacked, gamma);
+    if (tau_factor >= 0.0f) {
+        pdl_launch(bl::ternary_quant_kernel<true>, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n,
+                   partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, tau_factor);
+        return launched("ternary_quant(tau)");
+    }
+    pdl_launch(bl::ternary_quant_kernel<false>, dim3((unsigned)blocks), dim3(bl::kWqThreads), 0, st, W, n, partials,
+               parts, Wq_i8, Wq_bf16, Wpacked, gamma, 0.0f);
     return launched("ternary_quant");
 }
 
 // Weight quantiser: fp64 partial sums of |W| (pass 1), then pass 2.
 bl_status run_quant_weight(const float* W, int64_t n, void* scratch, int8_t* Wq_i8, uint16_t* Wq_bf16,
-                           uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev) {
+                           uint8_t* Wpacked, float* gamma, cudaStream_t st, const DeviceInfo& dev,
+                           float tau_factor = -1.0f) {
     double* partials = static_cast<double*>(scratch);
     const int parts = bl::wq_num_partials(n);
     pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
     BL_TRY(launched("absmean_partial"));
-    return run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
+    return run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev, tau_factor);
 }
+
+// Optimizer scratch: dW^2 partials, |W_new| partials, the published step index.
+constexpr size_t kOptWpartOffset = sizeof(double) * bl::kWqMaxPartials;
+constexpr size_t kOptStepOffset = 2 * sizeof(double) * bl::kWqMaxPartials;
+size_t opt_ws_bytes() { return kOptStepOffset + 16; }
 
 size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
 
@@ -438,8 +471,9 @@ constexpr int64_t kMaxRowK = 16384;
 // One block per SM (at most one per row group) of 16 warps (12 for two n-tiles, whose
 // accumulators need more registers).
 template <int NTILES>
-bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
-                      const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st, const DeviceInfo& dev) {
+bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int gamma_stride, int64_t N, int64_t K,
+                      const int8_t* xq, const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st,
+                      const DeviceInfo& dev) {
     constexpr int WB = NTILES == 1 ? 16 : 12;
     const int64_t n_rg = N / 16;
     const int64_t nb = n_rg < dev.sms ? n_rg : dev.sms;
@@ -458,8 +492,8 @@ bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int
         if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         attr_set.fetch_or(1ull << dev_id);
     }
-    pdl_launch(kern, dim3((unsigned)nb), dim3(WB * 32), smem, st, Wpacked, gamma, (int)N, (int)K, xq, sx, (int)B, y,
-               acc, g_wait_ns.load());
+    pdl_launch(kern, dim3((unsigned)nb), dim3(WB * 32), smem, st, Wpacked, gamma, gamma_stride, (int)N, (int)K, xq,
+               sx, (int)B, y, acc, g_wait_ns.load());
     return launched("ternary_gemv");
 }
 
@@ -481,6 +515,7 @@ size_t bitlinear_workspace_bytes(int64_t T, int64_t N, int64_t K) {
     size_t a = quant_ws_bytes();
     size_t b = dg_ws_bytes(K);
     size_t m = a > b ? a : b;
+    if (opt_ws_bytes() > m) m = opt_ws_bytes();
     return (m + 255) & ~size_t(255);
 }
 
@@ -711,8 +746,21 @@ bl_status ternary_pack(const int8_t* Wq_i8, int64_t N, int64_t K, uint8_t* Wpack
     return launched("ternary_pack");
 }
 
+bl_status gemv_entry(const uint8_t* Wpacked, const float* gamma, int gamma_stride, int64_t N, int64_t K,
+                     const int8_t* xq, const float* sx, int64_t B, float* y, int32_t* acc, void* stream);
+
 bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
                        const float* sx, int64_t B, float* y, int32_t* acc, void* stream) {
+    return gemv_entry(Wpacked, gamma, 0, N, K, xq, sx, B, y, acc, stream);
+}
+
+bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_rows, int64_t N, int64_t K, const int8_t* xq,
+                            const float* sx, int64_t B, float* y, int32_t* acc, void* stream) {
+    return gemv_entry(Wpacked, gamma_rows, 1, N, K, xq, sx, B, y, acc, stream);
+}
+
+bl_status gemv_entry(const uint8_t* Wpacked, const float* gamma, int gamma_stride, int64_t N, int64_t K,
+                     const int8_t* xq, const float* sx, int64_t B, float* y, int32_t* acc, void* stream) {
     BL_TRY(check_ptr(Wpacked, "Wpacked", true));
     BL_TRY(check_ptr(gamma, "gamma", true));
     BL_TRY(check_ptr(xq, "xq", true));
@@ -727,8 +775,8 @@ bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_t N, in
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (B <= 8) return launch_gemv<1>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
-    return launch_gemv<2>(Wpacked, gamma, N, K, xq, sx, B, y, acc, st, dev);
+    if (B <= 8) return launch_gemv<1>(Wpacked, gamma, gamma_stride, N, K, xq, sx, B, y, acc, st, dev);
+    return launch_gemv<2>(Wpacked, gamma, gamma_stride, N, K, xq, sx, B, y, acc, st, dev);
 }
 
 bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
@@ -764,6 +812,158 @@ bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, i
     }
     // pass 1 writes every partial that pass 2 reads, so nothing in the scratch needs clearing
     return run_quant_weight(W, n, scratch, Wq_i8, Wq_bf16, Wpacked, gamma, static_cast<cudaStream_t>(stream), dev);
+}
+
+// ------------------------------------------------------------------------------------
+// quantiser variants
+// ------------------------------------------------------------------------------------
+bl_status bitlinear_quant_weight_rows(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
+                                      uint8_t* Wpacked, float* gamma_rows, void* stream) {
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(gamma_rows, "gamma_rows", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", false));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_dims(1, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    pdl_launch(bl::ternary_quant_rows_kernel, dim3((unsigned)((N + 7) / 8)), dim3(256), 0,
+               static_cast<cudaStream_t>(stream), W, (int)N, (int)K, Wq_i8, Wq_bf16, Wpacked, gamma_rows);
+    return launched("ternary_quant_rows");
+}
+
+bl_status bitlinear_quant_weight_tau(const float* W, int64_t N, int64_t K, float tau_factor, int8_t* Wq_i8,
+                                     uint16_t* Wq_bf16, uint8_t* Wpacked, float* gamma, void* ws, size_t ws_bytes,
+                                     void* stream) {
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", false));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_ptr(ws, "ws", true));
+    BL_TRY(check_dims(1, N, K));
+    BL_REQUIRE(tau_factor >= 0.0f && tau_factor <= 1e30f, BL_ERR_INVALID_ARG,
+               "tau_factor must be finite and >= 0, got %g", (double)tau_factor);
+    BL_REQUIRE(ws_bytes >= quant_ws_bytes(), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu",
+               quant_ws_bytes(), ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_quant_weight(W, N * K, ws, Wq_i8, Wq_bf16, Wpacked, gamma, static_cast<cudaStream_t>(stream), dev,
+                            tau_factor);
+}
+
+bl_status bitlinear_act_quant_tensor(const void* X, bl_dtype x_dt, int64_t T, int64_t K, int apply_rmsnorm,
+                                     const float* g, float eps, int8_t* Xq, float* sx, float* rinv, void* Xdq,
+                                     void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_dtype(x_dt));
+    BL_TRY(check_ptr(X, "X", true));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(rinv, "rinv", apply_rmsnorm != 0));
+    BL_TRY(check_ptr(g, "g", false));
+    BL_TRY(check_ptr(Xdq, "Xdq", false));
+    BL_TRY(check_ptr(ws, "ws", true));
+    BL_TRY(check_dims(T, 16, K));
+    BL_REQUIRE(K <= kMaxRowK, BL_ERR_UNSUPPORTED_SHAPE, "d_in must be <= %lld for the row kernels, got %lld",
+               (long long)kMaxRowK, (long long)K);
+    BL_REQUIRE(!(eps < 0.0f) && eps == eps, BL_ERR_INVALID_ARG, "eps must be >= 0");
+    BL_REQUIRE(ws_bytes >= sizeof(float) * bl::kActMaxPartials, BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu",
+               sizeof(float) * bl::kActMaxPartials, ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t row_blocks = (T + 7) / 8;
+    const int grid = (int)(row_blocks < bl::kActMaxPartials ? row_blocks : bl::kActMaxPartials);
+    float* partials = static_cast<float*>(ws);
+    if (x_dt == BL_BF16) {
+        pdl_launch(bl::act_tensor_max_kernel<true>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, apply_rmsnorm, g,
+                   eps, rinv, partials);
+        BL_TRY(launched("act_tensor_max"));
+        pdl_launch(bl::act_tensor_quant_kernel<true>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, apply_rmsnorm,
+                   g, static_cast<const float*>(partials), grid, Xq, sx, static_cast<const float*>(rinv), Xdq);
+    } else {
+        pdl_launch(bl::act_tensor_max_kernel<false>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, apply_rmsnorm,
+                   g, eps, rinv, partials);
+        BL_TRY(launched("act_tensor_max"));
+        pdl_launch(bl::act_tensor_quant_kernel<false>, dim3(grid), dim3(256), 0, st, X, (int)T, (int)K, apply_rmsnorm,
+                   g, static_cast<const float*>(partials), grid, Xq, sx, static_cast<const float*>(rinv), Xdq);
+    }
+    return launched("act_tensor_quant");
+}
+
+bl_status bitlinear_linear_rows(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const int8_t* Wq_i8,
+                                const float* gamma_rows, int64_t N, void* Y, bl_dtype y_dt, int32_t* acc,
+                                void* stream) {
+    BL_TRY(check_dtype(y_dt));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", true));
+    BL_TRY(check_ptr(gamma_rows, "gamma_rows", true));
+    BL_TRY(check_ptr(Y, "Y", true));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_dims(T, N, K));
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    return run_linear_rows(Xq, sx, T, K, Wq_i8, gamma_rows, N, Y, y_dt, acc, static_cast<cudaStream_t>(stream), dev);
+}
+
+// ------------------------------------------------------------------------------------
+// optimizer step
+// ------------------------------------------------------------------------------------
+bl_status bitlinear_optimizer_step(float* W, const float* dW, float* m, float* v, int64_t N, int64_t K, float lr,
+                                   float beta1, float beta2, float eps, float weight_decay, float max_norm,
+                                   int32_t* step, int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked, float* gamma,
+                                   void* ws, size_t ws_bytes, void* stream) {
+    BL_TRY(check_ptr(W, "W", true));
+    BL_TRY(check_ptr(dW, "dW", true));
+    BL_TRY(check_ptr(m, "m", true));
+    BL_TRY(check_ptr(v, "v", true));
+    BL_TRY(check_ptr(step, "step", true));
+    BL_TRY(check_ptr(gamma, "gamma", false));
+    BL_TRY(check_ptr(Wq_i8, "Wq_i8", false));
+    BL_TRY(check_ptr(Wq_bf16, "Wq_bf16", false));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", false));
+    BL_TRY(check_ptr(ws, "ws", true));
+    BL_TRY(check_dims(1, N, K));
+    BL_REQUIRE(gamma != nullptr || (Wq_i8 == nullptr && Wq_bf16 == nullptr && Wpacked == nullptr), BL_ERR_INVALID_ARG,
+               "the next step's codes need gamma");
+    BL_REQUIRE(lr >= 0.0f && lr <= 1e30f, BL_ERR_INVALID_ARG, "lr must be finite and >= 0");
+    BL_REQUIRE(beta1 >= 0.0f && beta1 < 1.0f && beta2 >= 0.0f && beta2 < 1.0f, BL_ERR_INVALID_ARG,
+               "betas must be in [0, 1)");
+    BL_REQUIRE(eps > 0.0f && eps <= 1e30f, BL_ERR_INVALID_ARG, "eps must be finite and > 0");
+    BL_REQUIRE(weight_decay >= 0.0f && weight_decay <= 1e30f, BL_ERR_INVALID_ARG,
+               "weight_decay must be finite and >= 0");
+    BL_REQUIRE(max_norm == max_norm && max_norm <= 1e30f, BL_ERR_INVALID_ARG, "max_norm must be finite");
+    BL_REQUIRE(ws_bytes >= opt_ws_bytes(), BL_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", opt_ws_bytes(),
+               ws_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n = N * K;
+    const int parts = bl::wq_num_partials(n);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    double* gpart = reinterpret_cast<double*>(wsb);
+    double* wpart = reinterpret_cast<double*>(wsb + kOptWpartOffset);
+    int32_t* step_next = reinterpret_cast<int32_t*>(wsb + kOptStepOffset);
+    bl::AdamwArgs a{};
+    a.lr = lr;
+    a.beta1 = beta1;
+    a.beta2 = beta2;
+    a.eps = eps;
+    a.decay = (float)(1.0 - (double)lr * (double)weight_decay);
+    a.omb1 = (float)(1.0 - (double)beta1);
+    a.omb2 = (float)(1.0 - (double)beta2);
+    a.max_norm = max_norm;
+    pdl_launch(bl::grad_sumsq_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, dW, n, gpart,
+               static_cast<const int32_t*>(step), step_next);
+    BL_TRY(launched("grad_sumsq_partial"));
+    pdl_launch(bl::adamw_clamp_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, dW, m, v, n,
+               static_cast<const double*>(gpart), parts, a, static_cast<const int32_t*>(step_next), step,
+               gamma != nullptr ? wpart : static_cast<double*>(nullptr));
+    BL_TRY(launched("adamw_clamp"));
+    if (gamma == nullptr) return BL_OK;
+    // the next step's codes from the |W_new| partials written above (the quantiser's pass 2)
+    return run_ternary(W, n, wpart, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
 }
 
 bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

@@ -39,6 +39,8 @@ enum TcEpilogue : int {
     kEpiScaleF32 = 1,     // gamma * acc -> fp32
     kEpiF32 = 2,          // acc -> fp32
     kEpiLinearF32 = 3,    // y = acc * (gamma / s_t) -> fp32
+    kEpiLinearColBf16 = 4,  // y = acc * (gamma_n / s_t) -> bf16 (one scale per output column; 2-SM kernel only)
+    kEpiLinearColF32 = 5,   // y = acc * (gamma_n / s_t) -> fp32 (2-SM kernel only)
 };
 
 constexpr int kTcStages = 4;
@@ -66,9 +68,13 @@ __host__ __device__ constexpr size_t tc_smem_bytes() {
            (2 * kTcStages + 4) * sizeof(uint64_t) + 16;
 }
 
-__host__ __device__ constexpr bool epi_is_linear(int e) { return e == kEpiLinearBf16 || e == kEpiLinearF32; }
+__host__ __device__ constexpr bool epi_is_col(int e) { return e == kEpiLinearColBf16 || e == kEpiLinearColF32; }
+__host__ __device__ constexpr bool epi_is_linear(int e) {
+    return e == kEpiLinearBf16 || e == kEpiLinearF32 || epi_is_col(e);
+}
+__host__ __device__ constexpr bool epi_is_bf16(int e) { return e == kEpiLinearBf16 || e == kEpiLinearColBf16; }
 // Output columns per 128-byte chunk.
-__host__ __device__ constexpr int epi_chunk_cols(int e) { return e == kEpiLinearBf16 ? 64 : 32; }
+__host__ __device__ constexpr int epi_chunk_cols(int e) { return epi_is_bf16(e) ? 64 : 32; }
 
 template <bool kInt8, bool kAMN, bool kBMN, int kBN, int kEpi>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -76,6 +82,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tmD, const TcGemmArgs args) {
     static_assert(kBN % 64 == 0 && kBN <= 256, "kBN");
     static_assert(!kInt8 || (!kAMN && !kBMN), "int8 operands are K-major here");
+    static_assert(!epi_is_col(kEpi), "per-column scales are in the 2-SM kernel only");
     constexpr int kBBytes = tc_b_bytes<kBN>();
     constexpr uint32_t kStageTx = kTcABytes + kBBytes;
     constexpr int kKbElems = kInt8 ? 128 : 64;           // elements of K per stage
@@ -495,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         int buf = 0;
         int tcount = 0;
         float gm = 1.0f;
-        if constexpr (kEpi != kEpiF32) gm = __ldg(args.gamma);
+        if constexpr (kEpi != kEpiF32 && !epi_is_col(kEpi)) gm = __ldg(args.gamma);
         for (int tile = pair; tile < num_tiles; tile += npairs, ++tcount) {
             const int b = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
@@ -507,7 +514,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             const int row = row0 + lane;
             const bool row_ok = row < args.M;
             float cs = 1.0f;
-            if constexpr (epi_is_linear(kEpi)) cs = row_ok ? __fdiv_rn(gm, __ldg(args.row_scale + row)) : 0.0f;
+            if constexpr (epi_is_col(kEpi)) cs = row_ok ? __ldg(args.row_scale + row) : 1.0f;   // s_t
+            else if constexpr (epi_is_linear(kEpi)) cs = row_ok ? __fdiv_rn(gm, __ldg(args.row_scale + row)) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(b * kBN);
 #pragma unroll 1
@@ -525,15 +533,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
                 }
                 tmem_ld_wait();
                 auto r = [&](int i) -> uint32_t { return i < 32 ? ra[i] : rb[i - 32]; };
+                // the factor of chunk column i: gamma / s_t, or fl(gamma_n / s_t) per column
+                auto fac = [&](int i) -> float {
+                    if constexpr (epi_is_col(kEpi)) {
+                        const int c = col0 + i < args.N ? col0 + i : args.N - 1;
+                        return row_ok ? __fdiv_rn(__ldg(args.gamma + c), cs) : 0.0f;
+                    } else {
+                        return cs;
+                    }
+                };
                 uint4 v[8];
-                if constexpr (kEpi == kEpiLinearBf16) {
+                if constexpr (epi_is_bf16(kEpi)) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         uint32_t w[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float lo = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e))), cs);
-                            const float hi = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e + 1))), cs);
+                            const float lo = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e))), fac(8 * j + 2 * e));
+                            const float hi = __fmul_rn(static_cast<float>(static_cast<int32_t>(r(8 * j + 2 * e + 1))), fac(8 * j + 2 * e + 1));
                             w[e] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
                         }
                         v[j] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -545,8 +562,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const uint32_t raw = r(4 * j + e);
-                            if constexpr (kEpi == kEpiLinearF32)
-                                f[e] = __fmul_rn(static_cast<float>(static_cast<int32_t>(raw)), cs);
+                            if constexpr (kEpi == kEpiLinearF32 || kEpi == kEpiLinearColF32)
+                                f[e] = __fmul_rn(static_cast<float>(static_cast<int32_t>(raw)), fac(4 * j + e));
                             else if constexpr (kEpi == kEpiScaleF32)
                                 f[e] = __fmul_rn(gm, __uint_as_float(raw));
                             else

@@ -72,7 +72,7 @@ __host__ __device__ inline size_t gemv_smem_bytes(int B, int K, int max_rgs) {
 // ------------------------------------------------------------------------------------
 template <int NTILES, int WB>
 __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
-    const uint8_t* __restrict__ W, const float* __restrict__ gamma, int N, int K,
+    const uint8_t* __restrict__ W, const float* __restrict__ gamma, int gamma_stride, int N, int K,
     const int8_t* __restrict__ xq, const float* __restrict__ sx, int B, float* __restrict__ y,
     int32_t* __restrict__ acc_out, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
@@ -246,13 +246,15 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     }
     __syncthreads();
 
-    // y[b][n] = (acc - 2 sum x_b) * fl(gamma / s_b) for this block's rows, row-fastest
-    const float gm = __ldg(gamma);
+    // y[b][n] = (acc - 2 sum x_b) * fl(gamma_n / s_b) for this block's rows, row-fastest
+    // (gamma_n = gamma[n * gamma_stride]: one scale, or one per weight row)
     const int rows = nrg * 16;
     for (int idx = threadIdx.x; idx < rows * B; idx += WB * 32) {
         const int b = idx / rows, r = idx - b * rows;
         const int acc = accs[r * B + b] - 2 * xsum[b];
-        const int64_t o = static_cast<int64_t>(b) * N + rg0 * 16 + r;
+        const int n = rg0 * 16 + r;
+        const int64_t o = static_cast<int64_t>(b) * N + n;
+        const float gm = __ldg(gamma + static_cast<int64_t>(n) * gamma_stride);
         y[o] = __fmul_rn(static_cast<float>(acc), __fdiv_rn(gm, __ldg(sx + b)));
         if (acc_out != nullptr) acc_out[o] = acc;
     }

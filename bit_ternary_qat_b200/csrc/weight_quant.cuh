@@ -106,11 +106,23 @@ __device__ __forceinline__ float ternary_threshold_warp(float gamma) {
     return __uint_as_float(thr);
 }
 
+constexpr uint32_t kBf16One = 0x3F80u;   // bf16 bits of +1.0
+
+// Codes of 16 consecutive weights (group gi).  thr > 0: W_q = sign(w) [|w| >= thr].  With
+// kNonzero the rule also holds for thr = 0 (a zero weight keeps code 0).  The bf16 output
+// holds W_q times the magnitude whose bf16 bits are mag_bits (the codes themselves for +1).
+template <bool kNonzero = false>
 __device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int64_t gi, int8_t* __restrict__ wq_i8,
-                                           uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed) {
+                                           uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
+                                           uint32_t mag_bits = kBf16One) {
     int q[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) q[e] = (w[e] >= thr) ? 1 : ((w[e] <= -thr) ? -1 : 0);
+    for (int e = 0; e < 16; ++e) {
+        if constexpr (kNonzero)
+            q[e] = (w[e] >= thr && w[e] > 0.0f) ? 1 : ((w[e] <= -thr && w[e] < 0.0f) ? -1 : 0);
+        else
+            q[e] = (w[e] >= thr) ? 1 : ((w[e] <= -thr) ? -1 : 0);
+    }
     if (wq_i8 != nullptr) {
         uint32_t b[4];
 #pragma unroll
@@ -120,12 +132,13 @@ __device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int6
         reinterpret_cast<uint4*>(wq_i8)[gi] = make_uint4(b[0], b[1], b[2], b[3]);
     }
     if (wq_bf16 != nullptr) {
-        // bf16 bits of -1, 0, +1
+        // bf16 bits of -m, 0, +m
+        const uint32_t neg = mag_bits | 0x8000u;
         uint32_t h[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const uint32_t lo = q[2 * j] == 0 ? 0u : (q[2 * j] > 0 ? 0x3F80u : 0xBF80u);
-            const uint32_t hi = q[2 * j + 1] == 0 ? 0u : (q[2 * j + 1] > 0 ? 0x3F80u : 0xBF80u);
+            const uint32_t lo = q[2 * j] == 0 ? 0u : (q[2 * j] > 0 ? mag_bits : neg);
+            const uint32_t hi = q[2 * j + 1] == 0 ? 0u : (q[2 * j + 1] > 0 ? mag_bits : neg);
             h[j] = lo | (hi << 16);
         }
         uint4* dst = reinterpret_cast<uint4*>(wq_bf16) + gi * 2;
@@ -143,12 +156,15 @@ __device__ __forceinline__ void quantise16(const float (&w)[16], float thr, int6
 // n % 32 == 0.  Each thread loads kTqGroups groups of 16 weights (all loads in flight)
 // before the block waits for gamma and the threshold, then quantises them; weights beyond
 // grid * kWqThreads * kTqGroups groups are handled in further rounds of the same kind.
+// kTau: the zero threshold is tau = fl32(tau_factor * gamma) (P2, "直通估计器在三元权重量化
+// 中的作用": tau = 0.7 scale, |W| < tau -> 0) instead of the round/clamp threshold.
 constexpr int kTqGroups = 2;
 
+template <bool kTau>
 __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     const float* __restrict__ W, int64_t n, const double* __restrict__ partials, int nparts,
     int8_t* __restrict__ wq_i8, uint16_t* __restrict__ wq_bf16, uint8_t* __restrict__ packed,
-    float* __restrict__ gamma_out) {
+    float* __restrict__ gamma_out, float tau_factor) {
     __shared__ float s_thr;
     __shared__ double s_red[kWqThreads / 32];
     pdl_trigger_and_wait();
@@ -192,7 +208,11 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
 #pragma unroll
         for (int wi = 0; wi < kWqThreads / 32; ++wi) sum += s_red[wi];
         const float gamma = fmaxf(static_cast<float>(sum / static_cast<double>(n)), 1e-5f);
-        const float thr = ternary_threshold_warp(gamma);
+        float thr;
+        if constexpr (kTau)
+            thr = __fmul_rn(tau_factor, gamma);
+        else
+            thr = ternary_threshold_warp(gamma);
         if (threadIdx.x == 0) {
             s_thr = thr;
             if (blockIdx.x == 0) *gamma_out = gamma;
@@ -203,10 +223,52 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     for (int64_t r0 = 0;;) {
 #pragma unroll
         for (int q = 0; q < kTqGroups; ++q)
-            if (gi[q] < ngroups) quantise16(w[q], thr, gi[q], wq_i8, wq_bf16, packed);
+            if (gi[q] < ngroups) quantise16<kTau>(w[q], thr, gi[q], wq_i8, wq_bf16, packed);
         r0 += round_groups;
         if (r0 >= ngroups) break;
         load(r0, w, gi);
+    }
+}
+
+// Per-row scale (P4 §9 "Quantizer": scale = mean |W| over each output row), with the b1.58
+// round/clamp: gamma_n = max(mean_k |W[n, k]|, 1e-5), W_q = clamp(round(fl32(W / gamma_n)), -1, 1).
+// One warp per row, 8 rows per block: fp64 sum of |W| over the row, the row's threshold
+// (as above), then the row again (an L1/L2 hit) in groups of 16.  The bf16 output holds
+// W_q * bf16(gamma_n), the dequantised weight that the backward contraction uses.  K % 16 == 0.
+__global__ void __launch_bounds__(256) ternary_quant_rows_kernel(const float* __restrict__ W, int N, int K,
+                                                                 int8_t* __restrict__ wq_i8,
+                                                                 uint16_t* __restrict__ wq_bf16,
+                                                                 uint8_t* __restrict__ packed,
+                                                                 float* __restrict__ gamma_rows) {
+    pdl_trigger_and_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (n >= N) return;
+    const float4* row = reinterpret_cast<const float4*>(W + n * K);
+    const int nvec = K / 4;
+    double acc = 0.0;
+    for (int v = lane; v < nvec; v += 32) {
+        const float4 x = __ldg(row + v);
+        acc += (double)fabsf(x.x);
+        acc += (double)fabsf(x.y);
+        acc += (double)fabsf(x.z);
+        acc += (double)fabsf(x.w);
+    }
+    acc = warp_sum(acc);
+    const float gamma = fmaxf(static_cast<float>(acc / static_cast<double>(K)), 1e-5f);
+    const float thr = ternary_threshold_warp(gamma);
+    if (lane == 0) gamma_rows[n] = gamma;
+    const uint32_t mag = float_to_bf16_bits(gamma);
+    const int groups = K / 16;
+    const int64_t g0 = n * groups;
+    for (int q = lane; q < groups; q += 32) {
+        float w[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = __ldg(row + 4 * q + j);
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        }
+        quantise16(w, thr, g0 + q, wq_i8, wq_bf16, packed, mag);
     }
 }
 

@@ -284,6 +284,140 @@ def ternary_gemv(packed: torch.Tensor, gamma: torch.Tensor, K: int, xq: torch.Te
     return y, acc
 
 
+# ----------------------------------------------------------------------------------
+# quantiser variants (per-row weight scale, zero threshold, per-tensor activation scale)
+# ----------------------------------------------------------------------------------
+
+def bitlinear_quant_weight_rows(W: torch.Tensor, want_i8: bool = True, want_bf16: bool = True,
+                                want_packed: bool = True, out=None):
+    """Per-row scale. Returns dict(gamma_rows [N] f32, wq_i8 [N,K] i8, wq_bf16 [N,K] bf16
+    (= W_q * bf16(gamma_n)), packed [N,K/4] u8)."""
+    _cuda(W, "W", torch.float32)
+    N, K = W.shape
+    dev = W.device
+    o = dict(out or {})
+    o.setdefault("gamma_rows", torch.empty(N, dtype=torch.float32, device=dev))
+    if want_i8:
+        o.setdefault("wq_i8", torch.empty(N, K, dtype=torch.int8, device=dev))
+    if want_bf16:
+        o.setdefault("wq_bf16", torch.empty(N, K, dtype=torch.bfloat16, device=dev))
+    if want_packed:
+        o.setdefault("packed", torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    _lib.call("bitlinear_quant_weight_rows", W.data_ptr(), N, K, _ptr(o.get("wq_i8")), _ptr(o.get("wq_bf16")),
+              _ptr(o.get("packed")), o["gamma_rows"].data_ptr(), _stream(dev))
+    return o
+
+
+def bitlinear_quant_weight_tau(W: torch.Tensor, tau_factor: float = 0.7, want_i8: bool = True,
+                               want_bf16: bool = True, want_packed: bool = True,
+                               ws: Optional[torch.Tensor] = None, out=None):
+    """Zero threshold tau = tau_factor * gamma; outputs as bitlinear_quant_weight."""
+    _cuda(W, "W", torch.float32)
+    N, K = W.shape
+    dev = W.device
+    o = dict(out or {})
+    o.setdefault("gamma", torch.empty(1, dtype=torch.float32, device=dev))
+    if want_i8:
+        o.setdefault("wq_i8", torch.empty(N, K, dtype=torch.int8, device=dev))
+    if want_bf16:
+        o.setdefault("wq_bf16", torch.empty(N, K, dtype=torch.bfloat16, device=dev))
+    if want_packed:
+        o.setdefault("packed", torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    if ws is None:
+        ws = workspace(1, N, K, dev)
+    _lib.call("bitlinear_quant_weight_tau", W.data_ptr(), N, K, float(tau_factor), _ptr(o.get("wq_i8")),
+              _ptr(o.get("wq_bf16")), _ptr(o.get("packed")), o["gamma"].data_ptr(), ws.data_ptr(), ws.numel(),
+              _stream(dev))
+    return o
+
+
+def bitlinear_act_quant_tensor(X: torch.Tensor, apply_rmsnorm: bool = True, g: Optional[torch.Tensor] = None,
+                               eps: float = 1e-6, want_xdq: bool = True, ws: Optional[torch.Tensor] = None,
+                               out=None):
+    """Per-tensor scale; returns as bitlinear_act_quant (sx holds the one scale T times)."""
+    _cuda(X, "X")
+    T, K = X.shape
+    dev = X.device
+    if g is not None:
+        _cuda(g, "g", torch.float32)
+    o = dict(out or {})
+    o.setdefault("xq", torch.empty(T, K, dtype=torch.int8, device=dev))
+    o.setdefault("sx", torch.empty(T, dtype=torch.float32, device=dev))
+    if apply_rmsnorm:
+        o.setdefault("rinv", torch.empty(T, dtype=torch.float32, device=dev))
+    if want_xdq:
+        o.setdefault("xdq", torch.empty(T, K, dtype=X.dtype, device=dev))
+    if ws is None:
+        ws = workspace(T, 16, K, dev)
+    _lib.call("bitlinear_act_quant_tensor", X.data_ptr(), _dt(X), T, K, 1 if apply_rmsnorm else 0, _ptr(g),
+              float(eps), o["xq"].data_ptr(), o["sx"].data_ptr(), _ptr(o.get("rinv")), _ptr(o.get("xdq")),
+              ws.data_ptr(), ws.numel(), _stream(dev))
+    return o
+
+
+def bitlinear_linear_rows(xq: torch.Tensor, sx: torch.Tensor, wq_i8: torch.Tensor, gamma_rows: torch.Tensor,
+                          out_dtype=torch.bfloat16, want_acc: bool = False, y: Optional[torch.Tensor] = None,
+                          acc: Optional[torch.Tensor] = None):
+    _cuda(xq, "xq", torch.int8)
+    _cuda(wq_i8, "wq_i8", torch.int8)
+    T, K = xq.shape
+    N = wq_i8.shape[0]
+    dev = xq.device
+    if y is None:
+        y = torch.empty(T, N, dtype=out_dtype, device=dev)
+    if want_acc and acc is None:
+        acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    _lib.call("bitlinear_linear_rows", xq.data_ptr(), sx.data_ptr(), T, K, wq_i8.data_ptr(), gamma_rows.data_ptr(),
+              N, y.data_ptr(), _dt(y), _ptr(acc), _stream(dev))
+    return y, acc
+
+
+def ternary_gemv_rows(packed: torch.Tensor, gamma_rows: torch.Tensor, K: int, xq: torch.Tensor, sx: torch.Tensor,
+                      want_acc: bool = False, y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None):
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(xq, "xq", torch.int8)
+    N = packed.shape[0]
+    B = xq.shape[0]
+    dev = packed.device
+    if y is None:
+        y = torch.empty(B, N, dtype=torch.float32, device=dev)
+    if want_acc and acc is None:
+        acc = torch.empty(B, N, dtype=torch.int32, device=dev)
+    _lib.call("ternary_gemv_rows", packed.data_ptr(), gamma_rows.data_ptr(), N, K, xq.data_ptr(), sx.data_ptr(), B,
+              y.data_ptr(), _ptr(acc), _stream(dev))
+    return y, acc
+
+
+# ----------------------------------------------------------------------------------
+# optimizer step (clip -> AdamW -> clamp), optionally re-quantising W for the next step
+# ----------------------------------------------------------------------------------
+
+def bitlinear_optimizer_step(W: torch.Tensor, dW: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                             step: torch.Tensor, lr: float = 1e-3, betas=(0.9, 0.95), eps: float = 1e-6,
+                             weight_decay: float = 0.01, max_norm: float = 1.0, requantize: bool = False,
+                             ws: Optional[torch.Tensor] = None, out=None):
+    """Updates W, m, v (fp32) and step (int32 [1]) in place.  With requantize, returns
+    dict(gamma, wq_i8, wq_bf16, packed) of the updated W (keys from ``out`` are reused)."""
+    for t, name in ((W, "W"), (dW, "dW"), (m, "m"), (v, "v")):
+        _cuda(t, name, torch.float32)
+    _cuda(step, "step", torch.int32)
+    N, K = W.shape
+    dev = W.device
+    o = dict(out or {})
+    if requantize:
+        o.setdefault("gamma", torch.empty(1, dtype=torch.float32, device=dev))
+        o.setdefault("wq_i8", torch.empty(N, K, dtype=torch.int8, device=dev))
+        o.setdefault("wq_bf16", torch.empty(N, K, dtype=torch.bfloat16, device=dev))
+        o.setdefault("packed", torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+    if ws is None:
+        ws = workspace(1, N, K, dev)
+    _lib.call("bitlinear_optimizer_step", W.data_ptr(), dW.data_ptr(), m.data_ptr(), v.data_ptr(), N, K,
+              float(lr), float(betas[0]), float(betas[1]), float(eps), float(weight_decay), float(max_norm),
+              step.data_ptr(), _ptr(o.get("wq_i8")), _ptr(o.get("wq_bf16")), _ptr(o.get("packed")),
+              _ptr(o.get("gamma")), ws.data_ptr(), ws.numel(), _stream(dev))
+    return o
+
+
 def check_device_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     dev = device if device is not None else torch.cuda.current_device()

@@ -248,6 +248,81 @@ BL_API bl_status ternary_gemv(const uint8_t* Wpacked, const float* gamma, int64_
                        const int8_t* xq, const float* sx, int64_t B,
                        float* y, int32_t* acc, void* stream);
 
+/* ==============================================================================
+ * Quantiser variants the pages print beside the b1.58 defaults.  Same conventions,
+ * sizes, rounding and error behaviour as the entry points above.
+ * ============================================================================== */
+
+/* Per-row weight scale (P4 §9 "Quantizer": scale = mean |W| over each output row),
+ * with the b1.58 round/clamp (P3 §2.1, P5 §2.2):
+ *   gamma_rows[n] = max( (float)(sum_k |W[n,k]| / K), 1e-5 )   fp64 sum
+ *   W_q[n,k]      = clamp(round(fl32(W[n,k] / gamma_rows[n])), -1, 1)
+ * Outputs as bitlinear_quant_weight, except that Wq_bf16 holds the dequantised weight
+ * W_q[n,k] * bf16(gamma_rows[n]) (bf16 bits; the operand of the backward contraction, to
+ * be used with a gamma of 1.0), and gamma_rows is fp32 [N].  No workspace. */
+BL_API bl_status bitlinear_quant_weight_rows(const float* W, int64_t N, int64_t K,
+                                      int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                      float* gamma_rows, void* stream);
+
+/* Zero threshold (P2, "直通估计器在三元权重量化中的作用": tau = 0.7 x scale, |W| < tau
+ * quantises to 0), with the per-tensor gamma of bitlinear_quant_weight:
+ *   tau = fl32(tau_factor * gamma);  W_q = 0 if |W| < tau, else sign(W)  (sign(0) = 0)
+ * tau_factor finite and >= 0 (0.7 on the page; 0.5 reproduces the round rule except at
+ * exact ties), else BL_ERR_INVALID_ARG.  Outputs and workspace as bitlinear_quant_weight. */
+BL_API bl_status bitlinear_quant_weight_tau(const float* W, int64_t N, int64_t K, float tau_factor,
+                                     int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                     float* gamma, void* ws, size_t ws_bytes, void* stream);
+
+/* Per-tensor activation scale (P5 §5.1 quantize_activation: one 127 / max|x| for the
+ * whole tensor), applied to x_hat as in bitlinear_act_quant:
+ *   s    = fl32(127 / max(max_{t,k} |x_hat[t,k]|, 1e-5)),  written to sx[t] for every t
+ *   X_q  = clamp(round(fl32(x_hat * s)), -128, 127),  X_dq = fl32(X_q / s)
+ * Arguments as bitlinear_act_quant plus ws: at least bitlinear_workspace_bytes(T, N, K)
+ * bytes (block maxima).  Two launches; X is read twice. */
+BL_API bl_status bitlinear_act_quant_tensor(const void* X, bl_dtype x_dt, int64_t T, int64_t K,
+                                     int apply_rmsnorm, const float* g, float eps,
+                                     int8_t* Xq, float* sx, float* rinv, void* Xdq,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* The int8 x ternary linear with a per-row weight scale (the weight rows are the output
+ * columns):  y[t,n] = fl32( (float)acc[t,n] * fl32(gamma_rows[n] / sx[t]) ).
+ * Arguments as bitlinear_linear with gamma_rows fp32 [N]. */
+BL_API bl_status bitlinear_linear_rows(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
+                                const int8_t* Wq_i8, const float* gamma_rows, int64_t N,
+                                void* Y, bl_dtype y_dt, int32_t* acc, void* stream);
+
+/* The decode GEMV with a per-row weight scale: y[b,n] = acc[b,n] * fl32(gamma_rows[n] / sx[b]).
+ * Arguments and limits as ternary_gemv with gamma_rows fp32 [N]. */
+BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_rows, int64_t N, int64_t K,
+                            const int8_t* xq, const float* sx, int64_t B,
+                            float* y, int32_t* acc, void* stream);
+
+/* ==============================================================================
+ * Optimizer step of the latent weight, fused with the next step's weight quantiser
+ * (clip -> AdamW -> clamp, in the pages' order):
+ *   gradient clipping per weight matrix (P5 §6.2: clip_grad_norm_(p, 1.0)):
+ *     c = min(1, max_norm / (||dW||_2 + 1e-6)), c = 1 when max_norm <= 0;  g = c dW
+ *   AdamW (the 1-bit training guide's optimizer configuration: lr 1e-3, betas (0.9, 0.95),
+ *   weight decay 0.01, eps 1e-6), decoupled decay, bias-corrected moments, step t:
+ *     m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
+ *     W <- W (1 - lr wd) - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ *   clamp (same guide, weight constraint): W <- clamp(W, -1, 1).
+ * W, m, v fp32 [N x K] are updated in place; dW fp32 [N x K] (after any all-reduce) is
+ * read only.  step: device int32 holding the number of steps taken so far; this call uses
+ * t = *step + 1 and stores t back (so the call can be replayed in a CUDA graph).
+ * Element arithmetic is fp32 (one rounding per operation); the norm is an fp64 sum.
+ * If gamma is not NULL the call also produces the NEXT step's ternary weights from the
+ * updated W exactly as bitlinear_quant_weight would (same partial sums, same gamma, same
+ * codes; Wq_i8 / Wq_bf16 / Wpacked optional), reusing |W| sums taken during the update.
+ * Hyper-parameters must be finite with lr >= 0, 0 <= betas < 1, eps > 0, wd >= 0, else
+ * BL_ERR_INVALID_ARG.  ws: at least bitlinear_workspace_bytes(T, N, K) bytes.
+ * Three launches with gamma, two without; all HBM-bound. */
+BL_API bl_status bitlinear_optimizer_step(float* W, const float* dW, float* m, float* v,
+                                   int64_t N, int64_t K, float lr, float beta1, float beta2,
+                                   float eps, float weight_decay, float max_norm, int32_t* step,
+                                   int8_t* Wq_i8, uint16_t* Wq_bf16, uint8_t* Wpacked,
+                                   float* gamma, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------
  * Self-test of the bounded-wait machinery: launches one block that waits on an
  * mbarrier nothing arrives on, with the given limit (ns), and returns.  Afterwards
