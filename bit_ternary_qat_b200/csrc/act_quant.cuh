@@ -48,16 +48,6 @@ struct ActVec {
 constexpr float kRoundMagic = 12582912.0f;        // 1.5 * 2^23
 constexpr int32_t kRoundMagicBits = 0x4B400000;   // bit pattern of 1.5 * 2^23
 
-// fl(q / s) for integer-valued q in [-128, 127] and s > 0, given c = fl(1/s): two FMA
-// corrections; after the first, y1 is a faithful quotient, so the second residual is
-// exact and the second correction rounds correctly.
-__device__ __forceinline__ float div_by_scale(float q, float s, float c) {
-    const float y0 = __fmul_rn(q, c);
-    const float e0 = __fmaf_rn(-y0, s, q);
-    const float y1 = __fmaf_rn(e0, c, y0);
-    const float e1 = __fmaf_rn(-y1, s, q);
-    return __fmaf_rn(e1, c, y1);
-}
 
 // R independent block sums / maxima with one barrier each (fixed order: per thread, then a
 // fixed butterfly, then the warps in order).

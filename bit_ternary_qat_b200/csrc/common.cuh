@@ -339,6 +339,19 @@ __host__ __device__ constexpr uint32_t umma_idesc(bool int8, bool a_mn, bool b_m
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
     return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
+// fl(a / s) for s > 0, given c = fl(1/s), with two FMA corrections: after the first, y1 is a
+// faithful quotient, so the residual a - s*y1 is exact and the second correction rounds
+// correctly (Markstein's theorem).  Used with a = q in [-128, 127] (X_dq) and with a = a
+// weight scale (the per-column linear epilogue); both are checked in exact rational
+// arithmetic on the host.  No over- or underflow in those ranges.
+__device__ __forceinline__ float div_by_scale(float q, float s, float c) {
+    const float y0 = __fmul_rn(q, c);
+    const float e0 = __fmaf_rn(-y0, s, q);
+    const float y1 = __fmaf_rn(e0, c, y0);
+    const float e1 = __fmaf_rn(-y1, s, q);
+    return __fmaf_rn(e1, c, y1);
+}
+
 __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
     __nv_bfloat16 b = __float2bfloat16_rn(f);
     return *reinterpret_cast<uint16_t*>(&b);

@@ -514,7 +514,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             const int row = row0 + lane;
             const bool row_ok = row < args.M;
             float cs = 1.0f;
-            if constexpr (epi_is_col(kEpi)) cs = row_ok ? __ldg(args.row_scale + row) : 1.0f;   // s_t
+            float cr = 1.0f;   // col epilogues: fl(1 / s_t)
+            if constexpr (epi_is_col(kEpi)) {
+                cs = row_ok ? __ldg(args.row_scale + row) : 1.0f;   // s_t
+                cr = __frcp_rn(cs);
+            }
             else if constexpr (epi_is_linear(kEpi)) cs = row_ok ? __fdiv_rn(gm, __ldg(args.row_scale + row)) : 0.0f;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(b * kBN);
@@ -534,10 +538,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
                 tmem_ld_wait();
                 auto r = [&](int i) -> uint32_t { return i < 32 ? ra[i] : rb[i - 32]; };
                 // the factor of chunk column i: gamma / s_t, or fl(gamma_n / s_t) per column
+                // (correctly rounded from the row's reciprocal with two FMA corrections)
                 auto fac = [&](int i) -> float {
                     if constexpr (epi_is_col(kEpi)) {
                         const int c = col0 + i < args.N ? col0 + i : args.N - 1;
-                        return row_ok ? __fdiv_rn(__ldg(args.gamma + c), cs) : 0.0f;
+                        return row_ok ? div_by_scale(__ldg(args.gamma + c), cs, cr) : 0.0f;
                     } else {
                         return cs;
                     }

@@ -2,9 +2,9 @@
 //
 // Restates, in the order the pages give them: per-matrix gradient clipping to a maximum L2
 // norm (P5 §6.2 clip_grad_norm_(p, 1.0) for weight matrices), AdamW with decoupled weight
-// decay and bias-corrected moments (the 1-bit training guide's optimizer configuration:
-// lr 1e-3, betas (0.9, 0.95), weight decay 0.01, eps 1e-6), then the clamp of the latent
-// weight to [-1, 1] (same guide, "梯度裁剪与权重约束").
+// decay and bias-corrected moments (P1 "BitNet量化感知训练中的梯度传播优化", optimizer
+// configuration: lr 1e-3, betas (0.9, 0.95), weight decay 0.01, eps 1e-6), then the clamp of
+// the latent weight to [-1, 1] (P1 "梯度裁剪与权重约束").
 //
 // Two launches, both HBM-bound:
 //   pass 1  fp64 partial sums of dW^2, one per block, over the slices the weight

@@ -2,6 +2,7 @@
  * bitlinear.h -- C ABI of the B200 (sm_100a) BitNet b1.58 BitLinear hot path.
  *
  * Source pages (titles), cited per entry point below:
+ *   P1 = "BitNet量化感知训练中的梯度传播优化：解决符号函数不可微性的工程实践" (blog.hotdry.top)
  *   P2 = "BitNet 三元权重量化训练工程：直通估计器与梯度裁剪实践" (blog.hotdry.top)
  *   P3 = "BitNet 1.5技术解析：2比特量化在神经网络中的应用与挑战" (intelliparadigm.com)
  *   P4 = "BitNet b1.58：三元权重下的STE设计与优化" (zyxy.net)
@@ -302,11 +303,11 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
  * (clip -> AdamW -> clamp, in the pages' order):
  *   gradient clipping per weight matrix (P5 §6.2: clip_grad_norm_(p, 1.0)):
  *     c = min(1, max_norm / (||dW||_2 + 1e-6)), c = 1 when max_norm <= 0;  g = c dW
- *   AdamW (the 1-bit training guide's optimizer configuration: lr 1e-3, betas (0.9, 0.95),
- *   weight decay 0.01, eps 1e-6), decoupled decay, bias-corrected moments, step t:
+ *   AdamW (P1 optimizer configuration: lr 1e-3, betas (0.9, 0.95), weight decay 0.01,
+ *   eps 1e-6), decoupled decay, bias-corrected moments, step t:
  *     m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2
  *     W <- W (1 - lr wd) - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
- *   clamp (same guide, weight constraint): W <- clamp(W, -1, 1).
+ *   clamp (P1 "梯度裁剪与权重约束"): W <- clamp(W, -1, 1).
  * W, m, v fp32 [N x K] are updated in place; dW fp32 [N x K] (after any all-reduce) is
  * read only.  step: device int32 holding the number of steps taken so far; this call uses
  * t = *step + 1 and stores t back (so the call can be replayed in a CUDA graph).

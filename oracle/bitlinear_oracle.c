@@ -6,6 +6,7 @@
  * shares no code with it (no headers, no helpers, no tables).
  *
  * Pages this restates (titles of the source web pages):
+ *   P1 = "BitNet量化感知训练中的梯度传播优化：解决符号函数不可微性的工程实践" (blog.hotdry.top)
  *   P2 = "BitNet 三元权重量化训练工程：直通估计器与梯度裁剪实践" (blog.hotdry.top)
  *   P3 = "BitNet 1.5技术解析：2比特量化在神经网络中的应用与挑战" (intelliparadigm.com)
  *   P4 = "BitNet b1.58：三元权重下的STE设计与优化" (zyxy.net)
@@ -443,9 +444,8 @@ void ora_linear_epilogue_rows(const int32_t* acc, int64_t R, int64_t N, const fl
  * clipping to a maximum L2 norm (P5 §6.2: clip_grad_norm_ per weight matrix with
  * max_norm 1.0; P3 §6 and P4 §4.1 the same threshold over the model), then AdamW
  * (P2 training pipeline: AdamW; hyper-parameters lr 1e-3, betas (0.9, 0.95), weight decay
- * 0.01, eps 1e-6 from the optimizer configuration of the 1-bit training guide), then
- * the clamp of the latent weight to [-1, 1] (same guide, section on gradient clipping
- * and weight constraints).  AdamW is the decoupled-weight-decay algorithm of Loshchilov
+ * 0.01, eps 1e-6 from P1 "工程实践：可落地参数配置", optimizer configuration), then
+ * the clamp of the latent weight to [-1, 1] (P1 "梯度裁剪与权重约束").  AdamW is the decoupled-weight-decay algorithm of Loshchilov
  * and Hutter with bias-corrected moments:
  *   norm = sqrt(sum_i dW_i^2);  c = min(1, max_norm / (norm + 1e-6))   (c = 1 if max_norm <= 0)
  *   g = c dW;  W <- W - lr wd W;  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2

@@ -8,6 +8,7 @@ are IEEE round-to-nearest-even), independently of any GPU:
 * act quant: fl(q / s) == fl(y1 + fl(q - s*y1) * c) with c = fl(1/s), y0 = fl(q*c),
   y1 = fl(y0 + fl(q - s*y0) * c) (one reciprocal per row, two FMA corrections), for
   every q in [-128, 127];
+* the same two-correction quotient for fl(gamma_n / s_t) (per-column linear epilogue);
 * act quant: round-half-to-even of v via fl(v + 1.5*2^23) for |v| <= 128;
 * weight quant: the ternary code equals sign(w) * [|w| >= w*] with w* found by the
   32-wide window search around gamma/2;
@@ -59,6 +60,24 @@ def test_markstein_quotient_is_correctly_rounded():
                 assert q - s * y1 == e1         # y1 is faithful: the second residual is exact
                 y = rn32(y1 + e1 * c)
                 assert y == rn32(q / s), (float(q), float(s))
+
+
+def test_markstein_weight_scale_quotient_is_correctly_rounded():
+    """The per-column linear epilogue computes fl(gamma_n / s_t) the same way, with the
+    weight scale as the numerator: gamma in [1e-5, 1e2] (the quantiser's floor upwards),
+    s_t over the activation quantiser's whole range."""
+    rng = np.random.default_rng(2)
+    gammas = np.concatenate([10.0 ** rng.uniform(-5, 2, size=400), [1e-5, 0.02, 1.0, 100.0]])
+    ms = np.concatenate([10.0 ** rng.uniform(-5, 4, size=400), [1e-5, 1e-5, 1.0, 1e4]])
+    for gv, m in zip(gammas, ms):
+        a = Fraction(np.float32(max(np.float32(gv), np.float32(1e-5))).item())
+        s = Fraction(np.float32(np.float32(127.0) / np.float32(max(np.float32(m), np.float32(1e-5)))).item())
+        c = rn32(Fraction(1) / s)
+        y0 = rn32(a * c)
+        y1 = rn32(y0 + rn32(a - s * y0) * c)
+        e1 = rn32(a - s * y1)
+        assert a - s * y1 == e1
+        assert rn32(y1 + e1 * c) == rn32(a / s), (float(a), float(s))
 
 
 def test_magic_constant_rounds_half_to_even():

@@ -1,7 +1,8 @@
 """Pins of the oracle's optimizer step (clip -> AdamW -> clamp) to facts outside it.
 
-The pages fix the recipe (clip_grad_norm_ with max_norm 1.0; AdamW with lr 1e-3, betas
-(0.9, 0.95), weight decay 0.01, eps 1e-6; latent weight clamped to [-1, 1]) and call
+The pages fix the recipe (P5 §6.2 clip_grad_norm_ with max_norm 1.0; P1's AdamW with lr
+1e-3, betas (0.9, 0.95), weight decay 0.01, eps 1e-6; P1's clamp of the latent weight to
+[-1, 1]) and call
 torch's routines for it, so torch's own clip_grad_norm_ + AdamW + clamp_ in float64
 is an independent pin; the first step and the clip coefficient also have closed forms.
 """
