@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
+    ap.add_argument("--only-packed", action="store_true",
+                    help="run only the packed-weight linear at 16 tokens on the 28672 x 8192 weight (profiling)")
     ap.add_argument("--next", action="store_true",
                     help="time the fused optimizer step and the quantiser variants back to back; one JSON object, "
                          "not the bench line")
@@ -237,11 +239,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if args.only_gemv or args.table or args.next:
+    if args.only_gemv or args.table or args.next or args.only_packed:
         blbuild.build()
         bl.load()
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        if args.next:
+        if args.only_packed:
+            print(json.dumps({"linear_packed": packed_once(bl, torch, dev)}), flush=True)
+        elif args.next:
             print(json.dumps({"next": next_measure(bl, torch, dev, flush, peaks())}), flush=True)
         elif args.table:
             print(json.dumps({"table": table_measure(bl, torch, dev, flush, peaks())}), flush=True)
@@ -639,6 +643,31 @@ def gemv_measure(bl, torch, dev, flush, pk):
     return out
 
 
+def packed_once(bl, torch, dev):
+    """Three launches of the packed-weight linear, 16 tokens x the 28672 x 8192 decode weight
+    (a small case for a profiler capture); returns the last launch's event time."""
+    from bit_ternary_qat_b200 import synth
+    N, K, T = 28672, 8192, 16
+    W, _ = synth.decode_inputs(1, N, K)
+    q = bl.bitlinear_quant_weight(W.to(dev), want_i8=False, want_bf16=False)
+    del W
+    xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev, generator=torch.Generator(dev).manual_seed(1))
+    sx = torch.full((T,), 50.0, device=dev)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(T * N * 4, dtype=torch.uint8, device=dev)
+    ms = 0.0
+    for _ in range(3):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        bl.bitlinear_linear_packed(xq, sx, q["packed"], q["gamma"], K, y=y, ws=ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+    assert bl.check_device_status() == 0
+    return {"us_last": ms * 1e3, "shape": f"T={T} K={K} N={N}"}
+
+
 def next_measure(bl, torch, dev, flush, pk):
     """The fused optimizer step and the quantiser variants, each launched `reps` times back to
     back in one CUDA graph between one pair of CUDA events (median of 5, L2 flushed before each
@@ -744,6 +773,36 @@ def next_measure(bl, torch, dev, flush, pk):
     out["linear_8192x4096x11008"] = {"us": us_t, "TOPS": ops / (us_t * 1e-6) / 1e12, "note": "gamma / s_t epilogue"}
     out["linear_rows_8192x4096x11008"] = {"us": us_r, "TOPS": ops / (us_r * 1e-6) / 1e12,
                                           "note": "fl(gamma_n / s_t) per element epilogue"}
+    del xq, y
+    # packed-weight tensor-core linear vs the int8-code linear and the decode GEMV, few tokens
+    for (T, N, K) in ((16, 28672, 8192), (64, 11008, 4096), (256, 11008, 4096)):
+        Wd = synth.normal((N, K), 0.02, gen).to(dev)
+        qd = bl.bitlinear_quant_weight(Wd)
+        del Wd
+        # weight copies cycled so that each operand's copies together exceed 3 x L2
+        c8 = max(1, int(-(-3 * 128 * 2 ** 20 // (N * K))))
+        cp = max(1, int(-(-3 * 128 * 2 ** 20 // (N * K // 4))))
+        i8s = [qd["wq_i8"]] + [qd["wq_i8"].clone() for _ in range(c8 - 1)]
+        pks = [qd["packed"]] + [qd["packed"].clone() for _ in range(cp - 1)]
+        xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev)
+        sx = torch.full((T,), 50.0, device=dev)
+        y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+        ws_p = torch.empty(T * N * 4, dtype=torch.uint8, device=dev)
+        us_p = timed([lambda i=i: bl.bitlinear_linear_packed(xq, sx, pks[i], qd["gamma"], K, y=y, ws=ws_p)
+                      for i in range(cp)], 2 * cp)
+        us_8 = timed([lambda i=i: bl.bitlinear_linear(xq, sx, i8s[i], qd["gamma"], y=y) for i in range(c8)], 2 * c8)
+        row = {"packed_us": us_p, "int8_us": us_8,
+               "packed_weight_GBs": N * K / 4 / (us_p * 1e-6) / 1e9,
+               "packed_frac_hbm": (N * K / 4 + T * K + 2 * T * N) / (us_p * 1e-6) / 1e9 / pk["hbm"],
+               "int8_frac_hbm": (N * K + T * K + 2 * T * N) / (us_8 * 1e-6) / 1e9 / pk["hbm"],
+               "weight_copies": {"int8": c8, "packed": cp}}
+        if T <= 16:
+            y32 = torch.empty(T, N, dtype=torch.float32, device=dev)
+            row["gemv_us"] = timed([lambda i=i: bl.ternary_gemv(pks[i], qd["gamma"], K, xq, sx, y=y32)
+                                    for i in range(cp)], 2 * cp)
+        out[f"linear_packed_T{T}_{K}x{N}"] = row
+        del i8s, pks, qd, xq, y, ws_p
+        torch.cuda.empty_cache()
     out["hbm_peak_GBs"] = pk["hbm"]
     return out
 

@@ -55,6 +55,7 @@ SIGNATURES = {
     "bitlinear_act_quant_tensor": (INT, [P, INT, I64, I64, INT, P, F, P, P, P, P, P, SZ, P]),
     "bitlinear_linear_rows": (INT, [P, P, I64, I64, P, P, I64, P, INT, P, P]),
     "ternary_gemv_rows": (INT, [P, P, I64, I64, P, P, I64, P, P, P]),
+    "bitlinear_linear_packed": (INT, [P, P, I64, I64, P, P, I64, P, INT, P, P, SZ, P]),
     "bitlinear_optimizer_step": (INT, [P, P, P, P, I64, I64, F, F, F, F, F, F, P, P, P, P, P, P, SZ, P]),
 }
 

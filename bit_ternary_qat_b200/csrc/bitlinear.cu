@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -22,6 +23,7 @@
 #include "rmsnorm_bwd.cuh"
 #include "gemv.cuh"
 #include "optim.cuh"
+#include "gemm_packed.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -170,7 +172,7 @@ enum TmType { kTmU8 = 0, kTmBf16 = 1, kTmF32 = 2 };
 // 2-D row-major tensor [outer x inner] with 128-byte swizzled boxes [box_outer x box_inner]
 // (box_inner * element size == 128 bytes).
 bl_status make_tmap(CUtensorMap* tm, const void* base, TmType t, uint64_t inner, uint64_t outer,
-                    uint32_t box_inner, uint32_t box_outer) {
+                    uint32_t box_inner, uint32_t box_outer, bool swizzle128 = true) {
     EncodeTiledFn fn = encode_fn();
     BL_REQUIRE(fn != nullptr, BL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const uint64_t esize = t == kTmU8 ? 1 : (t == kTmBf16 ? 2 : 4);
@@ -181,7 +183,8 @@ bl_status make_tmap(CUtensorMap* tm, const void* base, TmType t, uint64_t inner,
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     BL_REQUIRE(r == CUDA_SUCCESS, BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return BL_OK;
 }
@@ -461,6 +464,74 @@ bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const f
         pdl_launch(bl::dg_reduce_kernel, dim3((unsigned)((K + 31) / 32)), dim3(1024), 0, st,
                    static_cast<const float*>(partial), grid, (int)K, dg);
         BL_TRY(launched("dg_reduce"));
+    }
+    return BL_OK;
+}
+
+// ------------------------------------------------------------------------------------
+// packed-weight GEMM: tile shape, K split and launch
+// ------------------------------------------------------------------------------------
+// Work units per wave: the fraction of the last wave's SMs that have work.
+inline double wave_eff(int64_t units, int sms) {
+    const int64_t waves = (units + sms - 1) / sms;
+    return static_cast<double>(units) / static_cast<double>(waves * sms);
+}
+
+template <bool kBf16Out>
+bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
+                        const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch, cudaStream_t st,
+                        const DeviceInfo& dev) {
+    bl::PkArgs a{};
+    a.T = (int)T; a.N = (int)N; a.K = (int)K;
+    int64_t bt = (T + 15) / 16 * 16;
+    if (bt > bl::kPkMaxBT) bt = bl::kPkMaxBT;
+    a.bt = (int)bt;
+    a.t_tiles = (int)((T + bt - 1) / bt);
+    a.n_tiles = (int)((N + bl::kPkBM - 1) / bl::kPkBM);
+    a.k_blocks = (int)((K + 127) / 128);
+    // K split: only with an int32 buffer for the sums, at least two k-blocks per unit; the
+    // smallest split whose last wave is within 3 % of the best
+    int32_t* sums = acc != nullptr ? acc : scratch;
+    const int64_t base = (int64_t)a.n_tiles * a.t_tiles;
+    int splits = 1;
+    if (sums != nullptr) {
+        const int smax = std::min(8, a.k_blocks / 2);
+        double best = wave_eff(base, dev.sms);
+        for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, dev.sms));
+        for (int sp = 1; sp <= std::max(1, smax); ++sp)
+            if (wave_eff(base * sp, dev.sms) >= best - 0.03) { splits = sp; break; }
+    }
+    a.splits = splits;
+    const size_t budget = (size_t)dev.max_smem_optin;
+    int stages = (int)((budget - bl::pk_smem_bytes((int)bt, 0)) / bl::pk_stage_bytes((int)bt));
+    if (stages > bl::kPkMaxStages) stages = bl::kPkMaxStages;
+    BL_REQUIRE(stages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
+    a.stages = stages;
+    a.sx = sx; a.gamma = gamma; a.y = Y;
+    a.acc = splits > 1 ? sums : acc;
+    a.wait_ns = g_wait_ns.load();
+    CUtensorMap tp, tx;
+    BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 32, bl::kPkBM, false));
+    BL_TRY(make_tmap(&tx, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, (uint32_t)bt));
+    auto kern = bl::tc_gemm_packed_kernel<kBf16Out>;
+    const size_t smem = bl::pk_smem_bytes((int)bt, stages);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    const int64_t units = base * splits;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, dev.sms);
+    if (splits > 1) {
+        const int64_t n = T * N;
+        pdl_launch(bl::pk_zero_kernel, dim3((unsigned)std::min<int64_t>((n / 4 + 255) / 256, (int64_t)dev.sms * 4)),
+                   dim3(256), 0, st, sums, n);
+        BL_TRY(launched("pk_zero"));
+    }
+    pdl_launch(kern, dim3(grid), dim3(bl::kPkThreads), smem, st, tp, tx, a);
+    BL_TRY(launched("tc_gemm_packed"));
+    if (splits > 1) {
+        const int64_t nv = T * N / 4;
+        pdl_launch(bl::pk_finalize_kernel<kBf16Out>, dim3((unsigned)std::min<int64_t>((nv + 255) / 256, (int64_t)dev.sms * 8)),
+                   dim3(256), 0, st, static_cast<const int32_t*>(sums), sx, gamma, (int)T, (int)N, Y);
+        BL_TRY(launched("pk_finalize"));
     }
     return BL_OK;
 }
@@ -905,6 +976,32 @@ bl_status bitlinear_linear_rows(const int8_t* Xq, const float* sx, int64_t T, in
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     return run_linear_rows(Xq, sx, T, K, Wq_i8, gamma_rows, N, Y, y_dt, acc, static_cast<cudaStream_t>(stream), dev);
+}
+
+// ------------------------------------------------------------------------------------
+// int8 x packed-ternary GEMM (few tokens)
+// ------------------------------------------------------------------------------------
+bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
+                                  const float* gamma, int64_t N, void* Y, bl_dtype y_dt, int32_t* acc, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    BL_TRY(check_dtype(y_dt));
+    BL_TRY(check_ptr(Xq, "Xq", true));
+    BL_TRY(check_ptr(sx, "sx", true));
+    BL_TRY(check_ptr(Wpacked, "Wpacked", true));
+    BL_TRY(check_ptr(gamma, "gamma", true));
+    BL_TRY(check_ptr(Y, "Y", true));
+    BL_TRY(check_ptr(acc, "acc", false));
+    BL_TRY(check_ptr(ws, "ws", false));
+    BL_TRY(check_dims(T, N, K));
+    BL_REQUIRE(K % 64 == 0, BL_ERR_UNSUPPORTED_SHAPE,
+               "packed rows are read in 16-byte pieces: K must be a multiple of 64, got %lld", (long long)K);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    int32_t* scratch = (ws != nullptr && ws_bytes >= (size_t)(T * N) * sizeof(int32_t)) ? static_cast<int32_t*>(ws)
+                                                                                       : nullptr;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (y_dt == BL_BF16) return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, st, dev);
+    return launch_packed<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, st, dev);
 }
 
 // ------------------------------------------------------------------------------------

@@ -1,0 +1,324 @@
+// gemm_packed.cuh -- int8 x packed-ternary tcgen05 GEMM for few tokens (prefill chunks and
+// batched decode), reading the weight as its 2-bit codes.
+//
+// Restates the linear of P3 §3.1 (y = F.linear(x_q, W_q) * gamma / s_t) on the packed
+// weight of P5 §4.1 (00 -> 0, 01 -> +1, 10 -> -1, 11 reserved -> 0) / §5.1: the weight
+// bytes that cross HBM are a quarter of the int8 codes', which is what bounds a GEMM with
+// few tokens.
+//
+// Operand roles are swapped so that the weight rows fill the 128-row tensor-core tile:
+//   D[n, t] = sum_k W_q[n, k] x_q[t, k]     (UMMA M = 128 weight rows, N = bt tokens)
+// so a batch of 16 tokens costs a 16-column MMA instead of a 128-row one.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over work units):
+//   warp 0     TMA producer: per stage the packed tile (128 rows x 32 bytes = 128 codes,
+//              no swizzle) and the activation tile (bt rows x 128 bytes, 128-byte swizzle);
+//   warps 6-9  decoders: 2-bit codes -> int8 written straight into the 128-byte-swizzled
+//              K-major layout the MMA reads (what TMA would have written for int8 codes);
+//   warp 1     MMA issuer (tcgen05.mma kind::i8, one thread), accumulators in TMEM
+//              (two 256-column buffers: the epilogue of one unit overlaps the next);
+//   warps 2-5  epilogue: tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (warp-wide
+//              coalesced stores along n), or -- when K is split across units -- exact int32
+//              sums added with red.global.add (integer addition: the result does not depend
+//              on the order), finished by pk_finalize_kernel.
+// Decode of one 32-bit word (16 codes): with a byte table TAB = {0, +1, -1, 0}, a byte
+// permute whose selector nibbles are the codes looks all of them up at once:
+//   even = prmt(TAB, sel = w & 0x33333333), odd = prmt(TAB, sel = (w >> 2) & 0x33333333)
+// (and their upper halves), then two permutes interleave even and odd codes -- 13 integer
+// operations per 16 codes.
+#pragma once
+#include "common.cuh"
+
+namespace bl {
+
+constexpr int kPkThreads = 320;
+constexpr int kPkBM = 128;                    // weight rows per tile (UMMA M)
+constexpr int kPkMaxBT = 256;                 // tokens per tile (UMMA N)
+constexpr int kPkMaxStages = 12;
+constexpr int kPkABytes = kPkBM * 128;        // decoded weight tile per stage (int8, SW128 K-major)
+constexpr int kPkPBytes = kPkBM * 32;         // packed weight tile per stage
+constexpr uint32_t kPkTab = 0x00FF0100u;      // byte c = int8 value of code c
+
+struct PkArgs {
+    int T, N, K;
+    int bt;                        // tokens per tile: multiple of 16, <= 256
+    int t_tiles, n_tiles, splits;  // work units = n_tiles * t_tiles * splits
+    int k_blocks;                  // blocks of 128 codes along K
+    int stages;
+    const float* sx;               // s_t [T]
+    const float* gamma;            // [1]
+    void* y;                       // [T x N], written when splits == 1
+    int32_t* acc;                  // [T x N]: splits > 1: summed into (zeroed before); else optional copy
+    uint64_t wait_ns;
+};
+
+__host__ __device__ inline size_t pk_stage_bytes(int bt) {
+    return static_cast<size_t>(kPkABytes) + kPkPBytes + static_cast<size_t>(bt) * 128;
+}
+__host__ __device__ inline size_t pk_smem_bytes(int bt, int stages) {
+    return 1024 + static_cast<size_t>(stages) * pk_stage_bytes(bt) + (3 * kPkMaxStages + 4) * sizeof(uint64_t) + 16;
+}
+
+// 16 codes of one packed word -> 16 int8 values (byte i = code i).
+__device__ __forceinline__ uint4 pk_decode_word(uint32_t w) {
+    const uint32_t se = w & 0x33333333u;
+    const uint32_t so = (w >> 2) & 0x33333333u;
+    const uint32_t e_lo = __byte_perm(kPkTab, 0u, se);          // codes 0, 2, 4, 6
+    const uint32_t e_hi = __byte_perm(kPkTab, 0u, se >> 16);    // codes 8, 10, 12, 14
+    const uint32_t o_lo = __byte_perm(kPkTab, 0u, so);          // codes 1, 3, 5, 7
+    const uint32_t o_hi = __byte_perm(kPkTab, 0u, so >> 16);    // codes 9, 11, 13, 15
+    return make_uint4(__byte_perm(e_lo, o_lo, 0x5140), __byte_perm(e_lo, o_lo, 0x7362),
+                      __byte_perm(e_hi, o_hi, 0x5140), __byte_perm(e_hi, o_hi, 0x7362));
+}
+
+template <bool kBf16Out>
+__global__ void __launch_bounds__(kPkThreads, 1)
+    tc_gemm_packed_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
+                          const PkArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align1024(smem_raw);
+    const int S = args.stages;
+    const int bt = args.bt;
+    const uint32_t x_bytes = static_cast<uint32_t>(bt) * 128u;
+    const size_t stage_bytes = pk_stage_bytes(bt);
+    // stage s: [decoded A 16 KB][activations bt x 128][packed 4 KB]; every piece 1024-aligned
+    auto sA = [&](int s) { return smem + s * stage_bytes; };
+    auto sX = [&](int s) { return smem + s * stage_bytes + kPkABytes; };
+    auto sP = [&](int s) { return smem + s * stage_bytes + kPkABytes + x_bytes; };
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
+    uint64_t* dec = full + kPkMaxStages;
+    uint64_t* empty = dec + kPkMaxStages;
+    uint64_t* tfull = empty + kPkMaxStages;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&dec[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmP);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger_and_wait();
+
+    const int units = args.n_tiles * args.t_tiles * args.splits;
+    const uint64_t lim = args.wait_ns;
+    // unit u -> (weight tile nt, token tile tt, K split sp) and its k-block range
+    auto unit_of = [&](int u, int& nt, int& tt, int& kb0, int& kb1) {
+        const int sp = u % args.splits;
+        const int rest = u / args.splits;
+        tt = rest % args.t_tiles;
+        nt = rest / args.t_tiles;
+        kb0 = static_cast<int>(static_cast<int64_t>(sp) * args.k_blocks / args.splits);
+        kb1 = static_cast<int>(static_cast<int64_t>(sp + 1) * args.k_blocks / args.splits);
+    };
+
+    if (warp == 0) {
+        // ----------------------------------------------------------------- producer
+        if (elect_one()) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int nt, tt, kb0, kb1;
+                unit_of(u, nt, tt, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kPkPBytes) + x_bytes);
+                    tma_load_2d(sP(s), &tmP, &full[s], kb * 32, nt * kPkBM);
+                    tma_load_2d(sX(s), &tmX, &full[s], kb * 128, tt * bt);
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                }
+            }
+            if (!ok) {
+                for (int i = 0; i < S; ++i) {
+                    const int ss = (s - 1 - i + 2 * S) % S;
+                    const uint32_t pp = (s - 1 - i < 0) ? (ph ^ 1u) : ph;
+                    mbar_wait(&full[ss], pp, 100000000ull, nullptr);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ----------------------------------------------------------------- decoders
+        const int dt = threadIdx.x - 192;          // 0..127
+        const int c = dt & 7;                      // word (16 codes) within the 128-code row piece
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            int nt, tt, kb0, kb1;
+            unit_of(u, nt, tt, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(&full[s], ph, lim, abort_flag)) { ok = false; break; }
+                const uint8_t* p = sP(s);
+                uint8_t* a = sA(s);
+#pragma unroll
+                for (int i = 0; i < kPkBM / 16; ++i) {
+                    const int r = (dt >> 3) + 16 * i;
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(p + r * 32 + c * 4);
+                    *reinterpret_cast<uint4*>(a + r * 128 + ((c ^ (r & 7)) << 4)) = pk_decode_word(w);
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dec[s]);
+                if (++s == S) { s = 0; ph ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------------------- MMA issuer
+        if (elect_one()) {
+            const uint32_t idesc = umma_idesc(true, false, false, kPkBM, bt);
+            int s = 0;
+            uint32_t ph = 0;
+            int tcount = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
+                int nt, tt, kb0, kb1;
+                unit_of(u, nt, tt, kb0, kb1);
+                const int b = tcount & 1;
+                const uint32_t tph = (tcount >> 1) & 1;
+                if (!mbar_wait(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kPkMaxBT);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(&full[s], ph, lim, abort_flag) || !mbar_wait(&dec[s], ph, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA(s));
+                    const uint32_t x_base = smem_u32(sX(s));
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma<true>(d_tmem, umma_desc_sw128(a_base + kk * 32, 16, 1024),
+                                     umma_desc_sw128(x_base + kk * 32, 16, 1024), idesc,
+                                     (kb != kb0 || kk != 0) ? 1u : 0u);
+                    tc_commit(&empty[s]);
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(&tfull[b]);
+            }
+            if (!ok) {
+                tc_commit(&tfull[tcount & 1]);
+                mbar_wait(&tfull[tcount & 1], ((tcount >> 1) & 1), 100000000ull, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------------------- epilogue
+        const int quad = warp & 3;                 // TMEM lanes [32 quad, 32 quad + 32)
+        const float gm = __ldg(args.gamma);
+        int tcount = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++tcount) {
+            int nt, tt, kb0, kb1;
+            unit_of(u, nt, tt, kb0, kb1);
+            const int b = tcount & 1;
+            const uint32_t tph = (tcount >> 1) & 1;
+            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            tc_fence_after();
+            const int n = nt * kPkBM + quad * 32 + lane;
+            const bool n_ok = n < args.N;
+            const int t0 = tt * bt;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                   static_cast<uint32_t>(b * kPkMaxBT);
+#pragma unroll 1
+            for (int c0 = 0; c0 < bt; c0 += 32) {
+                if (t0 + c0 >= args.T) break;                  // warp-uniform
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + c0, r);
+                tmem_ld_wait();
+                const int nj = min(32, min(bt - c0, args.T - t0 - c0));
+                if (n_ok) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (j >= nj) break;
+                        const int t = t0 + c0 + j;
+                        const int64_t o = static_cast<int64_t>(t) * args.N + n;
+                        const int32_t v = static_cast<int32_t>(r[j]);
+                        if (args.splits > 1) {
+                            atomicAdd(args.acc + o, v);
+                        } else {
+                            const float y = __fmul_rn(static_cast<float>(v), __fdiv_rn(gm, __ldg(args.sx + t)));
+                            if constexpr (kBf16Out)
+                                static_cast<uint16_t*>(args.y)[o] = float_to_bf16_bits(y);
+                            else
+                                static_cast<float*>(args.y)[o] = y;
+                            if (args.acc != nullptr) args.acc[o] = v;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// Zeroes the int32 sums before a split-K launch (n % 4 == 0).
+__global__ void __launch_bounds__(256) pk_zero_kernel(int32_t* __restrict__ acc, int64_t n) {
+    pdl_trigger_and_wait();
+    const int64_t nv = n / 4;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        reinterpret_cast<int4*>(acc)[i] = make_int4(0, 0, 0, 0);
+}
+
+// y = fl(acc * fl(gamma / s_t)) from the split-K sums (N % 4 == 0).
+template <bool kBf16Out>
+__global__ void __launch_bounds__(256) pk_finalize_kernel(const int32_t* __restrict__ acc,
+                                                          const float* __restrict__ sx,
+                                                          const float* __restrict__ gamma, int T, int N,
+                                                          void* __restrict__ y) {
+    pdl_trigger_and_wait();
+    const float gm = __ldg(gamma);
+    const int64_t nv = static_cast<int64_t>(T) * N / 4;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int t = static_cast<int>((i * 4) / N);
+        const float c = __fdiv_rn(gm, __ldg(sx + t));
+        const int4 a = reinterpret_cast<const int4*>(acc)[i];
+        const float v0 = __fmul_rn(static_cast<float>(a.x), c), v1 = __fmul_rn(static_cast<float>(a.y), c);
+        const float v2 = __fmul_rn(static_cast<float>(a.z), c), v3 = __fmul_rn(static_cast<float>(a.w), c);
+        if constexpr (kBf16Out) {
+            reinterpret_cast<uint2*>(y)[i] =
+                make_uint2((uint32_t)float_to_bf16_bits(v0) | ((uint32_t)float_to_bf16_bits(v1) << 16),
+                           (uint32_t)float_to_bf16_bits(v2) | ((uint32_t)float_to_bf16_bits(v3) << 16));
+        } else {
+            reinterpret_cast<float4*>(y)[i] = make_float4(v0, v1, v2, v3);
+        }
+    }
+}
+
+}  // namespace bl

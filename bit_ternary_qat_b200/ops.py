@@ -372,6 +372,26 @@ def bitlinear_linear_rows(xq: torch.Tensor, sx: torch.Tensor, wq_i8: torch.Tenso
     return y, acc
 
 
+def bitlinear_linear_packed(xq: torch.Tensor, sx: torch.Tensor, packed: torch.Tensor, gamma: torch.Tensor,
+                            K: int, out_dtype=torch.bfloat16, want_acc: bool = False,
+                            y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None,
+                            ws: Optional[torch.Tensor] = None):
+    """int8 x packed-ternary linear (few tokens); ws (>= 4*T*N bytes) lets K be split."""
+    _cuda(xq, "xq", torch.int8)
+    _cuda(packed, "packed", torch.uint8)
+    T = xq.shape[0]
+    N = packed.shape[0]
+    dev = xq.device
+    if y is None:
+        y = torch.empty(T, N, dtype=out_dtype, device=dev)
+    if want_acc and acc is None:
+        acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    _lib.call("bitlinear_linear_packed", xq.data_ptr(), sx.data_ptr(), T, K, packed.data_ptr(), gamma.data_ptr(),
+              N, y.data_ptr(), _dt(y), _ptr(acc), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+              _stream(dev))
+    return y, acc
+
+
 def ternary_gemv_rows(packed: torch.Tensor, gamma_rows: torch.Tensor, K: int, xq: torch.Tensor, sx: torch.Tensor,
                       want_acc: bool = False, y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None):
     _cuda(packed, "packed", torch.uint8)

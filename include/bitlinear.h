@@ -299,6 +299,25 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
                             float* y, int32_t* acc, void* stream);
 
 /* ==============================================================================
+ * int8 x packed-ternary linear for few tokens (prefill chunks, batched decode): the
+ * linear of bitlinear_linear computed from the 2-bit packed weight (P5 §4.1 codes, §5.1
+ * packing; a quarter of the int8 weight bytes cross HBM), decoded to int8 in shared
+ * memory and multiplied on the tensor cores (P3 §3.1):
+ *   acc[t,n] = sum_k decode(Wpacked[n,k]) * Xq[t,k]     exact int32 (reserved 11 -> 0)
+ *   Y[t,n]   = fl32(acc[t,n] * fl32(gamma / sx[t]))     in y_dt
+ * Xq int8 [T x K]; sx fp32 [T]; Wpacked uint8 [N x K/4]; gamma fp32 [1]; Y [T x N];
+ * acc int32 [T x N] optional.  K % 64 == 0.  Meant for T up to a few hundred tokens
+ * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).  When the
+ * weight tiles alone cannot fill the GPU, K is split across CTAs and the exact int32
+ * partial sums are added with atomics (order-free), which needs an int32 [T x N] buffer:
+ * acc if given, else ws if ws_bytes >= 4*T*N; with neither, K is not split.  One to three
+ * launches. */
+BL_API bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
+                                  const uint8_t* Wpacked, const float* gamma, int64_t N,
+                                  void* Y, bl_dtype y_dt, int32_t* acc, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* ==============================================================================
  * Optimizer step of the latent weight, fused with the next step's weight quantiser
  * (clip -> AdamW -> clamp, in the pages' order):
  *   gradient clipping per weight matrix (P5 §6.2: clip_grad_norm_(p, 1.0)):

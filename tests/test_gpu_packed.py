@@ -1,0 +1,82 @@
+"""GPU parity of the int8 x packed-ternary tensor-core linear (few tokens) against the oracle.
+
+The accumulators are exact int32 and compared bit for bit with the oracle's contraction of
+the unpacked codes (reserved code 11 decodes to 0); Y = fl(acc * fl(gamma / s_t)) is
+compared bit for bit with the oracle's epilogue (rounded to bf16 for a bf16 output), with
+and without the K split (whose int32 partial sums are added in any order, exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_ternary_qat_b200 import synth
+from parity_util import np_, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _gpu(a):
+    if isinstance(a, np.ndarray):
+        a = torch.from_numpy(a)
+    return a.to(DEV).contiguous()
+
+
+def _case(T, K, N, seed, raw_bytes=False):
+    rng = np.random.default_rng(seed)
+    xq = rng.integers(-128, 128, size=(T, K)).astype(np.int8)
+    if raw_bytes:
+        packed = rng.integers(0, 256, size=(N, K // 4)).astype(np.uint8)     # includes reserved 11 codes
+    else:
+        packed = oracle.pack(rng.integers(-1, 2, size=(N, K)).astype(np.int8))
+    s = rng.uniform(5, 300, size=T).astype(np.float32)
+    return xq, packed, s
+
+
+def _check(bl, xq, packed, s, gamma, out, split):
+    T, K = xq.shape
+    N = packed.shape[0]
+    ws = torch.empty(T * N * 4, dtype=torch.uint8, device=DEV) if split else None
+    y, acc = bl.bitlinear_linear_packed(_gpu(xq), _gpu(s), _gpu(packed), _gpu(torch.tensor([gamma])), K,
+                                        out_dtype=torch.bfloat16 if out == "bf16" else torch.float32,
+                                        want_acc=True, ws=ws)
+    torch.cuda.synchronize()
+    assert bl.check_device_status() == 0
+    wq = oracle.unpack(packed, K)
+    rows = None if T * N * K <= 2 ** 31 else sample_rows(T, 6, seed=T)
+    acc_o = oracle.int_gemm(xq, wq, rows=rows)
+    acc_g = np_(acc) if rows is None else np_(acc)[rows]
+    assert np.array_equal(acc_g, acc_o)
+    y_o = oracle.linear_epilogue(acc_o, gamma, s if rows is None else s[rows])
+    y_g = np_(y) if rows is None else np_(y)[rows]
+    assert np.array_equal(y_g, oracle.round_bf16(y_o) if out == "bf16" else y_o)
+    return y, acc
+
+
+@pytest.mark.parametrize("T,K,N", [(1, 64, 16), (7, 4096, 11008), (16, 8192, 28672), (64, 2048, 2048),
+                                   (129, 1024, 400), (300, 512, 1040), (33, 192, 2064)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+@pytest.mark.parametrize("split", [False, True])
+def test_linear_packed_parity(bl, T, K, N, out, split):
+    xq, packed, s = _case(T, K, N, seed=T + K + N)
+    _check(bl, xq, packed, s, 0.0173, out, split)
+
+
+def test_linear_packed_reserved_codes_decode_to_zero(bl):
+    xq, packed, s = _case(24, 512, 272, seed=5, raw_bytes=True)
+    assert np.any(((packed[:, :, None] >> np.array([0, 2, 4, 6])) & 3) == 3)
+    _check(bl, xq, packed, s, 0.02, "f32", False)
+    _check(bl, xq, packed, s, 0.02, "bf16", True)
+
+
+def test_linear_packed_matches_int8_linear(bl):
+    """Same layer through the quantisers: the packed path gives the int8 path's Y bit for bit."""
+    li = synth.random_case(48, 4096, 4096, seed=17, dtype="bf16")
+    qw = bl.bitlinear_quant_weight(_gpu(li.W))
+    aq = bl.bitlinear_act_quant(_gpu(li.X))
+    y8, acc8 = bl.bitlinear_linear(aq["xq"], aq["sx"], qw["wq_i8"], qw["gamma"], want_acc=True)
+    yp, accp = bl.bitlinear_linear_packed(aq["xq"], aq["sx"], qw["packed"], qw["gamma"], 4096, want_acc=True)
+    torch.cuda.synchronize()
+    assert torch.equal(acc8, accp)
+    assert torch.equal(y8.view(torch.int16), yp.view(torch.int16))

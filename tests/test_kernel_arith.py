@@ -198,3 +198,36 @@ def test_codes_from_rounding_sum_bits():
     words = [0x4B4000FB, 0x4B400005, 0x4B3FFF80, 0x4B40007F]
     got = _byte_perm(_byte_perm(words[0], words[1], 0x0040), _byte_perm(words[2], words[3], 0x0040), 0x5410)
     assert got == 0x7F8005FB
+
+
+def _pk_decode_word(w: int):
+    """Emulation of the packed GEMM's decoder: byte-permute lookups of the codes in the table
+    {0, +1, -1, 0}, then two permutes that interleave even and odd codes."""
+    tab = 0x00FF0100
+    se = w & 0x33333333
+    so = (w >> 2) & 0x33333333
+    e_lo = _byte_perm(tab, 0, se & 0xFFFF)
+    e_hi = _byte_perm(tab, 0, (se >> 16) & 0xFFFF)
+    o_lo = _byte_perm(tab, 0, so & 0xFFFF)
+    o_hi = _byte_perm(tab, 0, (so >> 16) & 0xFFFF)
+    words = [_byte_perm(e_lo, o_lo, 0x5140), _byte_perm(e_lo, o_lo, 0x7362),
+             _byte_perm(e_hi, o_hi, 0x5140), _byte_perm(e_hi, o_hi, 0x7362)]
+    out = []
+    for x in words:
+        for i in range(4):
+            b = (x >> (8 * i)) & 0xFF
+            out.append(b - 256 if b >= 128 else b)
+    return out
+
+
+def test_packed_gemm_decoder_matches_code_table():
+    """16 codes per word, code i in bits 2i..2i+1: 00 -> 0, 01 -> +1, 10 -> -1, 11 -> 0."""
+    rng = np.random.default_rng(9)
+    words = [0, 0xFFFFFFFF, 0x55555555, 0xAAAAAAAA, 0x1B1B1B1B] + rng.integers(0, 2 ** 32, 3000).tolist()
+    for w in words:
+        w = int(w)
+        ref = []
+        for i in range(16):
+            c = (w >> (2 * i)) & 3
+            ref.append((c & 1) - (c >> 1) if c != 3 else 0)
+        assert _pk_decode_word(w) == ref, hex(w)
