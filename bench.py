@@ -654,7 +654,7 @@ def packed_once(bl, torch, dev):
     xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev, generator=torch.Generator(dev).manual_seed(1))
     sx = torch.full((T,), 50.0, device=dev)
     y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(T * N * 4, dtype=torch.uint8, device=dev)
+    ws = torch.empty(8 * T * N * 4, dtype=torch.uint8, device=dev)
     ms = 0.0
     for _ in range(3):
         a = torch.cuda.Event(enable_timing=True)
@@ -787,7 +787,7 @@ def next_measure(bl, torch, dev, flush, pk):
         xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev)
         sx = torch.full((T,), 50.0, device=dev)
         y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
-        ws_p = torch.empty(T * N * 4, dtype=torch.uint8, device=dev)
+        ws_p = torch.empty(8 * T * N * 4, dtype=torch.uint8, device=dev)
         us_p = timed([lambda i=i: bl.bitlinear_linear_packed(xq, sx, pks[i], qd["gamma"], K, y=y, ws=ws_p)
                       for i in range(cp)], 2 * cp)
         us_8 = timed([lambda i=i: bl.bitlinear_linear(xq, sx, i8s[i], qd["gamma"], y=y) for i in range(c8)], 2 * c8)

@@ -479,8 +479,8 @@ inline double wave_eff(int64_t units, int sms) {
 
 template <bool kBf16Out>
 bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
-                        const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch, cudaStream_t st,
-                        const DeviceInfo& dev) {
+                        const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch, size_t scratch_bytes,
+                        cudaStream_t st, const DeviceInfo& dev) {
     bl::PkArgs a{};
     a.T = (int)T; a.N = (int)N; a.K = (int)K;
     int64_t bt = (T + 15) / 16 * 16;
@@ -489,13 +489,16 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     a.t_tiles = (int)((T + bt - 1) / bt);
     a.n_tiles = (int)((N + bl::kPkBM - 1) / bl::kPkBM);
     a.k_blocks = (int)((K + 127) / 128);
-    // K split: only with an int32 buffer for the sums, at least two k-blocks per unit; the
-    // smallest split whose last wave is within 3 % of the best
-    int32_t* sums = acc != nullptr ? acc : scratch;
+    // K split: only for a narrow token tile (bt <= 64), with a workspace for the int32 partial
+    // sums (splits x T x N), at least two k-blocks per unit, and partial-sum bytes at most a
+    // quarter of the packed weight bytes (splits <= K / (64 T)); the smallest split whose last
+    // wave is within 3 % of the best
     const int64_t base = (int64_t)a.n_tiles * a.t_tiles;
     int splits = 1;
-    if (sums != nullptr) {
-        const int smax = std::min(8, a.k_blocks / 2);
+    if (bt <= 64) {
+        int smax = std::min<int64_t>(8, a.k_blocks / 2);
+        smax = (int)std::min<int64_t>(smax, K / (64 * T));
+        smax = (int)std::min<int64_t>(smax, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));
         double best = wave_eff(base, dev.sms);
         for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, dev.sms));
         for (int sp = 1; sp <= std::max(1, smax); ++sp)
@@ -508,7 +511,7 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     BL_REQUIRE(stages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
     a.stages = stages;
     a.sx = sx; a.gamma = gamma; a.y = Y;
-    a.acc = splits > 1 ? sums : acc;
+    a.acc = splits > 1 ? scratch : acc;
     a.wait_ns = g_wait_ns.load();
     CUtensorMap tp, tx;
     BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 32, bl::kPkBM, false));
@@ -519,18 +522,12 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int64_t units = base * splits;
     const unsigned grid = (unsigned)std::min<int64_t>(units, dev.sms);
-    if (splits > 1) {
-        const int64_t n = T * N;
-        pdl_launch(bl::pk_zero_kernel, dim3((unsigned)std::min<int64_t>((n / 4 + 255) / 256, (int64_t)dev.sms * 4)),
-                   dim3(256), 0, st, sums, n);
-        BL_TRY(launched("pk_zero"));
-    }
     pdl_launch(kern, dim3(grid), dim3(bl::kPkThreads), smem, st, tp, tx, a);
     BL_TRY(launched("tc_gemm_packed"));
     if (splits > 1) {
         const int64_t nv = T * N / 4;
         pdl_launch(bl::pk_finalize_kernel<kBf16Out>, dim3((unsigned)std::min<int64_t>((nv + 255) / 256, (int64_t)dev.sms * 8)),
-                   dim3(256), 0, st, static_cast<const int32_t*>(sums), sx, gamma, (int)T, (int)N, Y);
+                   dim3(256), 0, st, static_cast<const int32_t*>(scratch), splits, sx, gamma, (int)T, (int)N, Y, acc);
         BL_TRY(launched("pk_finalize"));
     }
     return BL_OK;
@@ -997,11 +994,12 @@ bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, 
                "packed rows are read in 16-byte pieces: K must be a multiple of 64, got %lld", (long long)K);
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
-    int32_t* scratch = (ws != nullptr && ws_bytes >= (size_t)(T * N) * sizeof(int32_t)) ? static_cast<int32_t*>(ws)
-                                                                                       : nullptr;
+    int32_t* scratch = static_cast<int32_t*>(ws);
+    const size_t scratch_bytes = ws != nullptr ? ws_bytes : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (y_dt == BL_BF16) return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, st, dev);
-    return launch_packed<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, st, dev);
+    if (y_dt == BL_BF16)
+        return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
+    return launch_packed<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
 }
 
 // ------------------------------------------------------------------------------------

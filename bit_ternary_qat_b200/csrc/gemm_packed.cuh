@@ -10,17 +10,20 @@
 //   D[n, t] = sum_k W_q[n, k] x_q[t, k]     (UMMA M = 128 weight rows, N = bt tokens)
 // so a batch of 16 tokens costs a 16-column MMA instead of a 128-row one.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over work units):
+// Warp roles (704 threads, one CTA per SM, persistent over work units):
 //   warp 0     TMA producer: per stage the packed tile (128 rows x 32 bytes = 128 codes,
 //              no swizzle) and the activation tile (bt rows x 128 bytes, 128-byte swizzle);
-//   warps 6-9  decoders: 2-bit codes -> int8 written straight into the 128-byte-swizzled
-//              K-major layout the MMA reads (what TMA would have written for int8 codes);
+//   warps 6-21 decoders, four groups of four warps taking turns by stage (one stage's
+//              decode is a latency chain -- shared loads, 13 ops per word, shared stores,
+//              proxy fence, barrier arrive -- so four stages are decoded at once): 2-bit
+//              codes -> int8 written straight into the 128-byte-swizzled K-major layout the
+//              MMA reads (what TMA would have written for int8 codes);
 //   warp 1     MMA issuer (tcgen05.mma kind::i8, one thread), accumulators in TMEM
 //              (two 256-column buffers: the epilogue of one unit overlaps the next);
 //   warps 2-5  epilogue: tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (warp-wide
-//              coalesced stores along n), or -- when K is split across units -- exact int32
-//              sums added with red.global.add (integer addition: the result does not depend
-//              on the order), finished by pk_finalize_kernel.
+//              coalesced stores along n), or -- when K is split across units -- the exact
+//              int32 partial sums of split sp stored to slice sp of a workspace, which
+//              pk_finalize_kernel adds in split order (exact) before the same epilogue.
 // Decode of one 32-bit word (16 codes): with a byte table TAB = {0, +1, -1, 0}, a byte
 // permute whose selector nibbles are the codes looks all of them up at once:
 //   even = prmt(TAB, sel = w & 0x33333333), odd = prmt(TAB, sel = (w >> 2) & 0x33333333)
@@ -31,7 +34,8 @@
 
 namespace bl {
 
-constexpr int kPkThreads = 320;
+constexpr int kPkDecGroups = 4;              // decoder groups of 4 warps
+constexpr int kPkThreads = 192 + kPkDecGroups * 128;
 constexpr int kPkBM = 128;                    // weight rows per tile (UMMA M)
 constexpr int kPkMaxBT = 256;                 // tokens per tile (UMMA N)
 constexpr int kPkMaxStages = 12;
@@ -48,7 +52,8 @@ struct PkArgs {
     const float* sx;               // s_t [T]
     const float* gamma;            // [1]
     void* y;                       // [T x N], written when splits == 1
-    int32_t* acc;                  // [T x N]: splits > 1: summed into (zeroed before); else optional copy
+    int32_t* acc;                  // splits == 1: optional int32 copy [T x N]; splits > 1: partial
+                                   // sums [splits x T x N], slice sp written by the units of split sp
     uint64_t wait_ns;
 };
 
@@ -162,15 +167,21 @@ __global__ void __launch_bounds__(kPkThreads, 1)
         __syncwarp();
     } else if (warp >= 6) {
         // ----------------------------------------------------------------- decoders
-        const int dt = threadIdx.x - 192;          // 0..127
+        const int grp = (warp - 6) >> 2;            // this group decodes stages q = grp mod 4
+        const int dt = threadIdx.x - 192 - grp * 128;   // 0..127
         const int c = dt & 7;                      // word (16 codes) within the 128-code row piece
         int s = 0;
         uint32_t ph = 0;
+        int q = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int nt, tt, kb0, kb1;
             unit_of(u, nt, tt, kb0, kb1);
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int kb = kb0; kb < kb1; ++kb, ++q) {
+                if ((q & (kPkDecGroups - 1)) != grp) {
+                    if (++s == S) { s = 0; ph ^= 1u; }
+                    continue;
+                }
                 if (!mbar_wait(&full[s], ph, lim, abort_flag)) { ok = false; break; }
                 const uint8_t* p = sP(s);
                 uint8_t* a = sA(s);
@@ -260,7 +271,8 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                         const int64_t o = static_cast<int64_t>(t) * args.N + n;
                         const int32_t v = static_cast<int32_t>(r[j]);
                         if (args.splits > 1) {
-                            atomicAdd(args.acc + o, v);
+                            const int sp = u % args.splits;
+                            args.acc[static_cast<int64_t>(sp) * args.T * args.N + o] = v;
                         } else {
                             const float y = __fmul_rn(static_cast<float>(v), __fdiv_rn(gm, __ldg(args.sx + t)));
                             if constexpr (kBf16Out)
@@ -286,21 +298,13 @@ __global__ void __launch_bounds__(kPkThreads, 1)
     }
 }
 
-// Zeroes the int32 sums before a split-K launch (n % 4 == 0).
-__global__ void __launch_bounds__(256) pk_zero_kernel(int32_t* __restrict__ acc, int64_t n) {
-    pdl_trigger_and_wait();
-    const int64_t nv = n / 4;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-        reinterpret_cast<int4*>(acc)[i] = make_int4(0, 0, 0, 0);
-}
-
-// y = fl(acc * fl(gamma / s_t)) from the split-K sums (N % 4 == 0).
+// y = fl(acc * fl(gamma / s_t)) with acc = the split-K partial sums added in split order
+// (exact int32); acc_out optional (N % 4 == 0).
 template <bool kBf16Out>
-__global__ void __launch_bounds__(256) pk_finalize_kernel(const int32_t* __restrict__ acc,
+__global__ void __launch_bounds__(256) pk_finalize_kernel(const int32_t* __restrict__ part, int splits,
                                                           const float* __restrict__ sx,
                                                           const float* __restrict__ gamma, int T, int N,
-                                                          void* __restrict__ y) {
+                                                          void* __restrict__ y, int32_t* __restrict__ acc_out) {
     pdl_trigger_and_wait();
     const float gm = __ldg(gamma);
     const int64_t nv = static_cast<int64_t>(T) * N / 4;
@@ -308,7 +312,12 @@ __global__ void __launch_bounds__(256) pk_finalize_kernel(const int32_t* __restr
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>((i * 4) / N);
         const float c = __fdiv_rn(gm, __ldg(sx + t));
-        const int4 a = reinterpret_cast<const int4*>(acc)[i];
+        int4 a = __ldcs(reinterpret_cast<const int4*>(part) + i);
+        for (int sp = 1; sp < splits; ++sp) {
+            const int4 b = __ldcs(reinterpret_cast<const int4*>(part) + sp * nv + i);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        if (acc_out != nullptr) reinterpret_cast<int4*>(acc_out)[i] = a;
         const float v0 = __fmul_rn(static_cast<float>(a.x), c), v1 = __fmul_rn(static_cast<float>(a.y), c);
         const float v2 = __fmul_rn(static_cast<float>(a.z), c), v3 = __fmul_rn(static_cast<float>(a.w), c);
         if constexpr (kBf16Out) {

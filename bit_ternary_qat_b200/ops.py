@@ -376,7 +376,7 @@ def bitlinear_linear_packed(xq: torch.Tensor, sx: torch.Tensor, packed: torch.Te
                             K: int, out_dtype=torch.bfloat16, want_acc: bool = False,
                             y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None,
                             ws: Optional[torch.Tensor] = None):
-    """int8 x packed-ternary linear (few tokens); ws (>= 4*T*N bytes) lets K be split."""
+    """int8 x packed-ternary linear (few tokens); ws (up to 8 x 4*T*N bytes) lets K be split."""
     _cuda(xq, "xq", torch.int8)
     _cuda(packed, "packed", torch.uint8)
     T = xq.shape[0]

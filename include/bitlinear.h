@@ -308,10 +308,11 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
  * Xq int8 [T x K]; sx fp32 [T]; Wpacked uint8 [N x K/4]; gamma fp32 [1]; Y [T x N];
  * acc int32 [T x N] optional.  K % 64 == 0.  Meant for T up to a few hundred tokens
  * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).  When the
- * weight tiles alone cannot fill the GPU, K is split across CTAs and the exact int32
- * partial sums are added with atomics (order-free), which needs an int32 [T x N] buffer:
- * acc if given, else ws if ws_bytes >= 4*T*N; with neither, K is not split.  One to three
- * launches. */
+ * weight tiles alone cannot fill the GPU and at most 64 tokens are given, K may be split
+ * across CTAs: split sp stores its exact int32 partial sums to slice sp of ws (int32
+ * [splits x T x N]) and a second launch adds the slices in split order and applies the
+ * scale.  The split count is limited by ws_bytes / (4 T N) (ws NULL: no split), by 8 and by
+ * K / (64 T).  One or two launches. */
 BL_API bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
                                   const uint8_t* Wpacked, const float* gamma, int64_t N,
                                   void* Y, bl_dtype y_dt, int32_t* acc, void* ws, size_t ws_bytes,

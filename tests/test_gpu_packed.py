@@ -37,7 +37,7 @@ def _case(T, K, N, seed, raw_bytes=False):
 def _check(bl, xq, packed, s, gamma, out, split):
     T, K = xq.shape
     N = packed.shape[0]
-    ws = torch.empty(T * N * 4, dtype=torch.uint8, device=DEV) if split else None
+    ws = torch.empty(8 * T * N * 4, dtype=torch.uint8, device=DEV) if split else None
     y, acc = bl.bitlinear_linear_packed(_gpu(xq), _gpu(s), _gpu(packed), _gpu(torch.tensor([gamma])), K,
                                         out_dtype=torch.bfloat16 if out == "bf16" else torch.float32,
                                         want_acc=True, ws=ws)
@@ -55,7 +55,8 @@ def _check(bl, xq, packed, s, gamma, out, split):
 
 
 @pytest.mark.parametrize("T,K,N", [(1, 64, 16), (7, 4096, 11008), (16, 8192, 28672), (64, 2048, 2048),
-                                   (129, 1024, 400), (300, 512, 1040), (33, 192, 2064)])
+                                   (129, 1024, 400), (300, 512, 1040), (33, 192, 2064), (8, 2048, 400),
+                                   (3, 1024, 272)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 @pytest.mark.parametrize("split", [False, True])
 def test_linear_packed_parity(bl, T, K, N, out, split):
