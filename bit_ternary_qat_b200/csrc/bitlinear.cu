@@ -506,18 +506,20 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     }
     a.splits = splits;
     const size_t budget = (size_t)dev.max_smem_optin;
-    int stages = (int)((budget - bl::pk_smem_bytes((int)bt, 0)) / bl::pk_stage_bytes((int)bt));
-    if (stages > bl::kPkMaxStages) stages = bl::kPkMaxStages;
-    BL_REQUIRE(stages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
-    a.stages = stages;
+    // rings: 4 decoded and 4 activation stages; the packed ring (16 KB stages, 512 codes per
+    // row) takes the rest of shared memory (at most 12 stages)
+    int pstages = (int)((budget - bl::pk_smem_bytes((int)bt, 0)) / bl::kPkPBytes);
+    pstages = std::min(pstages, bl::kPkMaxPStages);
+    BL_REQUIRE(pstages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
+    a.pstages = pstages;
     a.sx = sx; a.gamma = gamma; a.y = Y;
     a.acc = splits > 1 ? scratch : acc;
     a.wait_ns = g_wait_ns.load();
     CUtensorMap tp, tx;
-    BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 32, bl::kPkBM, false));
+    BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, bl::kPkBM));
     BL_TRY(make_tmap(&tx, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, (uint32_t)bt));
     auto kern = bl::tc_gemm_packed_kernel<kBf16Out>;
-    const size_t smem = bl::pk_smem_bytes((int)bt, stages);
+    const size_t smem = bl::pk_smem_bytes((int)bt, pstages);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int64_t units = base * splits;

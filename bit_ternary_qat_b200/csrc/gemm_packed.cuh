@@ -10,20 +10,29 @@
 //   D[n, t] = sum_k W_q[n, k] x_q[t, k]     (UMMA M = 128 weight rows, N = bt tokens)
 // so a batch of 16 tokens costs a 16-column MMA instead of a 128-row one.
 //
-// Warp roles (704 threads, one CTA per SM, persistent over work units):
-//   warp 0     TMA producer: per stage the packed tile (128 rows x 32 bytes = 128 codes,
-//              no swizzle) and the activation tile (bt rows x 128 bytes, 128-byte swizzle);
-//   warps 6-21 decoders, four groups of four warps taking turns by stage (one stage's
-//              decode is a latency chain -- shared loads, 13 ops per word, shared stores,
-//              proxy fence, barrier arrive -- so four stages are decoded at once): 2-bit
-//              codes -> int8 written straight into the 128-byte-swizzled K-major layout the
-//              MMA reads (what TMA would have written for int8 codes);
+// Warp roles (704 threads, one CTA per SM, persistent over work units), three rings:
+//   packed ring (128 rows x 128 bytes = 512 codes per row per stage, 128-byte swizzle) and
+//              activation ring (bt x 128-byte tiles per 128-code k-block, 4 stages in step with
+//              the decoded ring): warp 0 keeps both full with TMA loads.  A packed box moves 128 bytes per
+//              weight row: with 32-byte rows the copy engine's per-row rate, not HBM, was the
+//              limit (measured);
+//   decoded ring (4 stages of 128 rows x 128 int8 codes, 128-byte-swizzled K-major):
+//              warps 6-21, four groups of four warps, group g owning decoded stage g, decode
+//              one k-block of a packed stage into the int8 layout the MMA reads (what TMA
+//              would have written for int8 codes), fence the writes to the async proxy and
+//              arrive;
 //   warp 1     MMA issuer (tcgen05.mma kind::i8, one thread), accumulators in TMEM
 //              (two 256-column buffers: the epilogue of one unit overlaps the next);
 //   warps 2-5  epilogue: tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (warp-wide
-//              coalesced stores along n), or -- when K is split across units -- the exact
-//              int32 partial sums of split sp stored to slice sp of a workspace, which
+//              coalesced stores along n; each lane forms one token's factor and the warp
+//              shares them by shuffle), or -- when K is split across units -- the exact int32
+//              partial sums of split sp stored to slice sp of a workspace, which
 //              pk_finalize_kernel adds in split order (exact) before the same epilogue.
+// Every decoder warp waits on every packed stage and arrives on its empty barrier (16
+// arrivals), and the decoded ring's depth equals the number of groups, so each barrier's
+// phases are waited on strictly in order by each waiter (a parity wait cannot confuse a
+// phase with the one two phases earlier); the producer and the MMA issuer walk all rings in
+// order.
 // Decode of one 32-bit word (16 codes): with a byte table TAB = {0, +1, -1, 0}, a byte
 // permute whose selector nibbles are the codes looks all of them up at once:
 //   even = prmt(TAB, sel = w & 0x33333333), odd = prmt(TAB, sel = (w >> 2) & 0x33333333)
@@ -38,9 +47,13 @@ constexpr int kPkDecGroups = 4;              // decoder groups of 4 warps
 constexpr int kPkThreads = 192 + kPkDecGroups * 128;
 constexpr int kPkBM = 128;                    // weight rows per tile (UMMA M)
 constexpr int kPkMaxBT = 256;                 // tokens per tile (UMMA N)
-constexpr int kPkMaxStages = 12;
+constexpr int kPkDStages = kPkDecGroups;      // decoded ring depth (one stage per group)
+constexpr int kPkXStages = kPkDStages;       // activation ring depth: in step with the decoded
+                                              // ring, so one commit per k-block frees both
+constexpr int kPkMaxPStages = 12;             // packed ring depth
+constexpr int kPkKbPerP = 4;                  // 128-code k-blocks per packed stage
 constexpr int kPkABytes = kPkBM * 128;        // decoded weight tile per stage (int8, SW128 K-major)
-constexpr int kPkPBytes = kPkBM * 32;         // packed weight tile per stage
+constexpr int kPkPBytes = kPkBM * 128;        // packed weight tile per stage (512 codes per row)
 constexpr uint32_t kPkTab = 0x00FF0100u;      // byte c = int8 value of code c
 
 struct PkArgs {
@@ -48,7 +61,7 @@ struct PkArgs {
     int bt;                        // tokens per tile: multiple of 16, <= 256
     int t_tiles, n_tiles, splits;  // work units = n_tiles * t_tiles * splits
     int k_blocks;                  // blocks of 128 codes along K
-    int stages;
+    int pstages;                   // packed ring depth
     const float* sx;               // s_t [T]
     const float* gamma;            // [1]
     void* y;                       // [T x N], written when splits == 1
@@ -57,11 +70,9 @@ struct PkArgs {
     uint64_t wait_ns;
 };
 
-__host__ __device__ inline size_t pk_stage_bytes(int bt) {
-    return static_cast<size_t>(kPkABytes) + kPkPBytes + static_cast<size_t>(bt) * 128;
-}
-__host__ __device__ inline size_t pk_smem_bytes(int bt, int stages) {
-    return 1024 + static_cast<size_t>(stages) * pk_stage_bytes(bt) + (3 * kPkMaxStages + 4) * sizeof(uint64_t) + 16;
+__host__ __device__ inline size_t pk_smem_bytes(int bt, int pstages) {
+    return 1024 + static_cast<size_t>(kPkDStages) * kPkABytes + static_cast<size_t>(kPkXStages) * bt * 128 +
+           static_cast<size_t>(pstages) * kPkPBytes + (2 * kPkMaxPStages + 3 * kPkDStages + 4) * sizeof(uint64_t) + 16;
 }
 
 // 16 codes of one packed word -> 16 int8 values (byte i = code i).
@@ -82,18 +93,22 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                           const PkArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
-    const int S = args.stages;
+    constexpr int XS = kPkXStages;
+    const int PS = args.pstages;
     const int bt = args.bt;
     const uint32_t x_bytes = static_cast<uint32_t>(bt) * 128u;
-    const size_t stage_bytes = pk_stage_bytes(bt);
-    // stage s: [decoded A 16 KB][activations bt x 128][packed 4 KB]; every piece 1024-aligned
-    auto sA = [&](int s) { return smem + s * stage_bytes; };
-    auto sX = [&](int s) { return smem + s * stage_bytes + kPkABytes; };
-    auto sP = [&](int s) { return smem + s * stage_bytes + kPkABytes + x_bytes; };
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);
-    uint64_t* dec = full + kPkMaxStages;
-    uint64_t* empty = dec + kPkMaxStages;
-    uint64_t* tfull = empty + kPkMaxStages;
+    // [decoded A: 4 x 16 KB][packed: PS x 16 KB][activations: XS x bt x 128]; all 1024-aligned
+    auto sA = [&](int d) { return smem + d * kPkABytes; };
+    uint8_t* sPbase = smem + kPkDStages * kPkABytes;
+    auto sP = [&](int p) { return sPbase + p * kPkPBytes; };
+    uint8_t* sXbase = sPbase + PS * kPkPBytes;
+    auto sX = [&](int x) { return sXbase + x * x_bytes; };
+    uint64_t* pfull = reinterpret_cast<uint64_t*>(sXbase + XS * x_bytes);
+    uint64_t* pempty = pfull + kPkMaxPStages;
+    uint64_t* xfull = pempty + kPkMaxPStages;
+    uint64_t* dfull = xfull + kPkXStages;
+    uint64_t* dempty = dfull + kPkDStages;     // frees decoded stage d and activation stage d
+    uint64_t* tfull = dempty + kPkDStages;
     uint64_t* tempty = tfull + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -101,10 +116,16 @@ __global__ void __launch_bounds__(kPkThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&dec[s], 4);
-            mbar_init(&empty[s], 1);
+        for (int p = 0; p < PS; ++p) {
+            mbar_init(&pfull[p], 1);
+            mbar_init(&pempty[p], 4 * kPkDecGroups);   // every decoder warp
+        }
+        for (int x = 0; x < XS; ++x) {
+            mbar_init(&xfull[x], 1);
+        }
+        for (int d = 0; d < kPkDStages; ++d) {
+            mbar_init(&dfull[d], 4);     // the 4 decoder warps of the stage's group
+            mbar_init(&dempty[d], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -140,69 +161,88 @@ __global__ void __launch_bounds__(kPkThreads, 1)
     };
 
     if (warp == 0) {
-        // ----------------------------------------------------------------- producer
+        // ----------------------------------------------------------------- producer (both load rings)
         if (elect_one()) {
-            int s = 0;
-            uint32_t ph = 0;
+            int p = 0, x = 0;
+            uint32_t pph = 0, xph = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 int nt, tt, kb0, kb1;
                 unit_of(u, nt, tt, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kPkPBytes) + x_bytes);
-                    tma_load_2d(sP(s), &tmP, &full[s], kb * 32, nt * kPkBM);
-                    tma_load_2d(sX(s), &tmX, &full[s], kb * 128, tt * bt);
-                    if (++s == S) { s = 0; ph ^= 1u; }
+                    if ((kb - kb0) % kPkKbPerP == 0) {
+                        // the unit's next packed stage: k-blocks kb .. kb + 3
+                        if (!mbar_wait(&pempty[p], pph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                        mbar_arrive_expect_tx(&pfull[p], static_cast<uint32_t>(kPkPBytes));
+                        tma_load_2d(sP(p), &tmP, &pfull[p], kb * 32, nt * kPkBM);
+                        if (++p == PS) { p = 0; pph ^= 1u; }
+                    }
+                    if (!mbar_wait(&dempty[x], xph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&xfull[x], x_bytes);
+                    tma_load_2d(sX(x), &tmX, &xfull[x], kb * 128, tt * bt);
+                    if (++x == XS) { x = 0; xph ^= 1u; }
                 }
             }
             if (!ok) {
-                for (int i = 0; i < S; ++i) {
-                    const int ss = (s - 1 - i + 2 * S) % S;
-                    const uint32_t pp = (s - 1 - i < 0) ? (ph ^ 1u) : ph;
-                    mbar_wait(&full[ss], pp, 100000000ull, nullptr);
+                // let the loads issued last land before the block exits (bounded)
+                for (int i = 0; i < PS; ++i) {
+                    const int pp = (p - 1 - i + 2 * PS) % PS;
+                    mbar_wait(&pfull[pp], (p - 1 - i < 0) ? (pph ^ 1u) : pph, 100000000ull, nullptr);
+                }
+                for (int i = 0; i < XS; ++i) {
+                    const int xx = (x - 1 - i + 2 * XS) % XS;
+                    mbar_wait(&xfull[xx], (x - 1 - i < 0) ? (xph ^ 1u) : xph, 100000000ull, nullptr);
                 }
             }
         }
         __syncwarp();
     } else if (warp >= 6) {
         // ----------------------------------------------------------------- decoders
-        const int grp = (warp - 6) >> 2;            // this group decodes stages q = grp mod 4
+        const int grp = (warp - 6) >> 2;           // decodes k-block sequence numbers q = grp mod 4
         const int dt = threadIdx.x - 192 - grp * 128;   // 0..127
-        const int c = dt & 7;                      // word (16 codes) within the 128-code row piece
-        int s = 0;
-        uint32_t ph = 0;
+        const int c = dt & 7;                      // word (16 codes) within a k-block's 32-byte row piece
+        const int r0 = dt >> 3;                    // rows r0 + 16 i; r & 7 == r0 & 7 for all of them
+        int p = 0;
+        uint32_t pph = 0, dph = 0;
         int q = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             int nt, tt, kb0, kb1;
             unit_of(u, nt, tt, kb0, kb1);
-            for (int kb = kb0; kb < kb1; ++kb, ++q) {
-                if ((q & (kPkDecGroups - 1)) != grp) {
-                    if (++s == S) { s = 0; ph ^= 1u; }
-                    continue;
-                }
-                if (!mbar_wait(&full[s], ph, lim, abort_flag)) { ok = false; break; }
-                const uint8_t* p = sP(s);
-                uint8_t* a = sA(s);
+            for (int kb = kb0; kb < kb1 && ok; kb += kPkKbPerP) {
+                if (!mbar_wait(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
+                const uint8_t* src = sP(p);
+                const int nkb = min(kPkKbPerP, kb1 - kb);
+                for (int j = 0; j < nkb; ++j, ++q) {
+                    if ((q & (kPkDecGroups - 1)) != grp) continue;
+                    // the MMA has finished with this group's decoded stage (its previous use)
+                    if (!mbar_wait(&dempty[grp], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    uint8_t* a = sA(grp);
+                    // 16-byte chunk (2 j + c / 4) of row r sits at chunk (2 j + c / 4) ^ (r & 7)
+                    const int src_off = ((((2 * j + (c >> 2)) ^ (r0 & 7)) << 4) | ((c & 3) << 2));
+                    const int dst_off = (c ^ (r0 & 7)) << 4;
 #pragma unroll
-                for (int i = 0; i < kPkBM / 16; ++i) {
-                    const int r = (dt >> 3) + 16 * i;
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(p + r * 32 + c * 4);
-                    *reinterpret_cast<uint4*>(a + r * 128 + ((c ^ (r & 7)) << 4)) = pk_decode_word(w);
+                    for (int i = 0; i < kPkBM / 16; ++i) {
+                        const int r = r0 + 16 * i;
+                        const uint32_t w = *reinterpret_cast<const uint32_t*>(src + r * 128 + src_off);
+                        *reinterpret_cast<uint4*>(a + r * 128 + dst_off) = pk_decode_word(w);
+                    }
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&dfull[grp]);
+                    dph ^= 1u;
                 }
-                fence_proxy_async_shared();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dec[s]);
-                if (++s == S) { s = 0; ph ^= 1u; }
+                if (lane == 0) mbar_arrive(&pempty[p]);
+                if (++p == PS) { p = 0; pph ^= 1u; }
             }
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------------- MMA issuer
         if (elect_one()) {
             const uint32_t idesc = umma_idesc(true, false, false, kPkBM, bt);
-            int s = 0;
-            uint32_t ph = 0;
+            int d = 0, x = 0;
+            uint32_t dph = 0, xph = 0;
             int tcount = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
@@ -214,20 +254,21 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kPkMaxBT);
                 for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!mbar_wait(&full[s], ph, lim, abort_flag) || !mbar_wait(&dec[s], ph, lim, abort_flag)) {
+                    if (!mbar_wait(&xfull[x], xph, lim, abort_flag) || !mbar_wait(&dfull[d], dph, lim, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(sA(s));
-                    const uint32_t x_base = smem_u32(sX(s));
+                    const uint32_t a_base = smem_u32(sA(d));
+                    const uint32_t x_base = smem_u32(sX(x));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma<true>(d_tmem, umma_desc_sw128(a_base + kk * 32, 16, 1024),
                                      umma_desc_sw128(x_base + kk * 32, 16, 1024), idesc,
                                      (kb != kb0 || kk != 0) ? 1u : 0u);
-                    tc_commit(&empty[s]);
-                    if (++s == S) { s = 0; ph ^= 1u; }
+                    tc_commit(&dempty[d]);     // d == x: the rings move in step
+                    if (++d == kPkDStages) { d = 0; dph ^= 1u; }
+                    if (++x == XS) { x = 0; xph ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit(&tfull[b]);
@@ -263,24 +304,26 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                 tmem_ld_32x32b_x32(t_row + c0, r);
                 tmem_ld_wait();
                 const int nj = min(32, min(bt - c0, args.T - t0 - c0));
-                if (n_ok) {
+                // lane l forms the factor of token t0 + c0 + l; the warp shares them by shuffle
+                const float cl = (args.splits == 1 && lane < nj) ? __fdiv_rn(gm, __ldg(args.sx + t0 + c0 + lane)) : 0.0f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (j >= nj) break;
-                        const int t = t0 + c0 + j;
-                        const int64_t o = static_cast<int64_t>(t) * args.N + n;
-                        const int32_t v = static_cast<int32_t>(r[j]);
-                        if (args.splits > 1) {
-                            const int sp = u % args.splits;
-                            args.acc[static_cast<int64_t>(sp) * args.T * args.N + o] = v;
-                        } else {
-                            const float y = __fmul_rn(static_cast<float>(v), __fdiv_rn(gm, __ldg(args.sx + t)));
-                            if constexpr (kBf16Out)
-                                static_cast<uint16_t*>(args.y)[o] = float_to_bf16_bits(y);
-                            else
-                                static_cast<float*>(args.y)[o] = y;
-                            if (args.acc != nullptr) args.acc[o] = v;
-                        }
+                for (int j = 0; j < 32; ++j) {
+                    if (j >= nj) break;                            // warp-uniform
+                    const float cj = __shfl_sync(0xffffffffu, cl, j);
+                    if (!n_ok) continue;
+                    const int t = t0 + c0 + j;
+                    const int64_t o = static_cast<int64_t>(t) * args.N + n;
+                    const int32_t v = static_cast<int32_t>(r[j]);
+                    if (args.splits > 1) {
+                        const int sp = u % args.splits;
+                        args.acc[static_cast<int64_t>(sp) * args.T * args.N + o] = v;
+                    } else {
+                        const float y = __fmul_rn(static_cast<float>(v), cj);
+                        if constexpr (kBf16Out)
+                            static_cast<uint16_t*>(args.y)[o] = float_to_bf16_bits(y);
+                        else
+                            static_cast<float*>(args.y)[o] = y;
+                        if (args.acc != nullptr) args.acc[o] = v;
                     }
                 }
             }
