@@ -463,13 +463,7 @@ __global__ void __launch_bounds__(256) act_tensor_quant_kernel(const void* __res
         __syncthreads();
     }
     const int nvec = K / E;
-    // rows in the reverse of pass 1's order: the rows pass 1 read last are the likeliest to
-    // still be in L2
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * 8;
-    const int64_t first = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-    const int64_t steps = first < T ? (T - 1 - first) / stride : -1;
-    for (int64_t k = steps; k >= 0; --k) {
-        const int64_t t = first + k * stride;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp; t < T; t += static_cast<int64_t>(gridDim.x) * 8) {
         const uint4* xrow = reinterpret_cast<const uint4*>(X) + t * nvec;
         const float r = apply_norm ? __ldg(rinv + t) : 1.0f;
         if (lane == 0) sx[t] = s;

@@ -184,10 +184,7 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     };
     float w[kTqGroups][16];
     int64_t gi[kTqGroups];
-    // rounds run from the end of W to its start: pass 1 read W front to back, so when W is
-    // larger than L2 the part it read last is still there for the first rounds here
-    const int64_t last_round = ((ngroups + round_groups - 1) / round_groups - 1) * round_groups;
-    load(last_round, w, gi);
+    load(0, w, gi);
     {
         // fixed-order sum of the partials by the whole block: thread i adds partials
         // i, i + 256, ... (all loaded at once), then a fixed butterfly per warp and the warp
@@ -223,12 +220,12 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     }
     __syncthreads();
     const float thr = s_thr;
-    for (int64_t r0 = last_round;;) {
+    for (int64_t r0 = 0;;) {
 #pragma unroll
         for (int q = 0; q < kTqGroups; ++q)
             if (gi[q] < ngroups) quantise16<kTau>(w[q], thr, gi[q], wq_i8, wq_bf16, packed);
-        r0 -= round_groups;
-        if (r0 < 0) break;
+        r0 += round_groups;
+        if (r0 >= ngroups) break;
         load(r0, w, gi);
     }
 }
