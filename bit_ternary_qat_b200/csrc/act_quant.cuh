@@ -255,30 +255,32 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
 // Short rows (at most 32 * VPL 16-byte vectors): one warp per row, 8 rows per block, no
 // shared memory and no block barrier -- both reductions are warp butterflies (fixed order).
 // Each lane keeps its VPL raw vectors of the row in registers and widens them on use, so a
-// warp has the whole row in flight at once and many rows fit on an SM.
-template <bool kBf16, int VPL>
-__device__ __forceinline__ void act_quant_warp_rows(const void* __restrict__ X, int T, int K, int apply_norm,
-                                                    const float* __restrict__ g, float eps, int8_t* __restrict__ Xq,
-                                                    float* __restrict__ sx, float* __restrict__ rinv,
-                                                    void* __restrict__ Xdq, int row_block,
-                                                    typename DqLut<kBf16>::T (*lut_all)[256]) {
-    using V = ActVec<kBf16>;
-    using LutT = typename DqLut<kBf16>::T;
-    constexpr int E = V::kElems;
+// warp has the whole row in flight at once.  The kernel is persistent (two blocks per SM,
+// rows strided over the grid) and loads a warp's next row before it quantises the current
+// one, so loads stay in flight through the reductions and there is no partial last wave.
+template <int VPL>
+__device__ __forceinline__ void act_quant_warp_load(const void* __restrict__ X, int64_t t, int nvec,
+                                                    uint4 (&raw)[VPL]) {
     const int lane = threadIdx.x & 31;
-    const int64_t t = static_cast<int64_t>(row_block) * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
-    LutT* lut = lut_all[threadIdx.x >> 5];
-    const int nvec = K / E;
-    const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
-    const uint4* xrow = reinterpret_cast<const uint4*>(X) + row_vec0;
-
-    uint4 raw[VPL];
+    const uint4* xrow = reinterpret_cast<const uint4*>(X) + t * static_cast<int64_t>(nvec);
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
         const int v = lane + 32 * j;
         raw[j] = v < nvec ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
     }
+}
+
+template <bool kBf16, int VPL>
+__device__ __forceinline__ void act_quant_warp_row(const uint4 (&raw)[VPL], int64_t t, int K, int apply_norm,
+                                                   const float* __restrict__ g, float eps, int8_t* __restrict__ Xq,
+                                                   float* __restrict__ sx, float* __restrict__ rinv,
+                                                   void* __restrict__ Xdq, typename DqLut<kBf16>::T* lut) {
+    using V = ActVec<kBf16>;
+    constexpr int E = V::kElems;
+    const int lane = threadIdx.x & 31;
+    const int nvec = K / E;
+    const int64_t row_vec0 = t * static_cast<int64_t>(nvec);
+    __syncwarp();   // every lane is done with the previous row's table
 
     // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order; max |x| on the way
     float r = 1.0f;
@@ -365,7 +367,23 @@ __global__ void __launch_bounds__(256, 2) act_quant_warp_kernel(const void* __re
                                                                 float* __restrict__ rinv, void* __restrict__ Xdq) {
     __shared__ typename DqLut<kBf16>::T lut_all[8][256];
     pdl_trigger_and_wait();
-    act_quant_warp_rows<kBf16, VPL>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, blockIdx.x, lut_all);
+    const int warp = threadIdx.x >> 5;
+    const int nvec = K / ActVec<kBf16>::kElems;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * 8;
+    int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (t >= T) return;
+    uint4 cur[VPL];
+    act_quant_warp_load<VPL>(X, t, nvec, cur);
+    for (;;) {
+        const int64_t tn = t + stride;
+        uint4 nxt[VPL];
+        if (tn < T) act_quant_warp_load<VPL>(X, tn, nvec, nxt);
+        act_quant_warp_row<kBf16, VPL>(cur, t, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, lut_all[warp]);
+        if (tn >= T) break;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) cur[j] = nxt[j];
+        t = tn;
+    }
 }
 
 // ------------------------------------------------------------------------------------

@@ -275,10 +275,26 @@ void launch_act_quant_v(const void* X, int64_t T, int64_t K, int apply_norm, con
                eps, Xq, sx, rinv, Xdq);
 }
 
+// SM count of the current device (cached per device).
+int sm_count() {
+    static std::atomic<int> cache[64] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (dev_id < 0 || dev_id >= 64) return 148;
+    int n = cache[dev_id].load();
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess || n <= 0) n = 148;
+        cache[dev_id].store(n);
+    }
+    return n;
+}
+
+// Persistent: two blocks of 8 row-warps per SM at most.
 template <bool kBf16, int VPL>
 void launch_act_quant_w(const void* X, int64_t T, int64_t K, int apply_norm, const float* g, float eps, int8_t* Xq,
                         float* sx, float* rinv, void* Xdq, cudaStream_t st) {
-    pdl_launch(bl::act_quant_warp_kernel<kBf16, VPL>, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, st, X, (int)T,
+    const int64_t blocks = std::min<int64_t>((T + 7) / 8, 2 * (int64_t)sm_count());
+    pdl_launch(bl::act_quant_warp_kernel<kBf16, VPL>, dim3((unsigned)blocks), dim3(256), 0, st, X, (int)T,
                (int)K, apply_norm, g, eps, Xq, sx, rinv, Xdq);
 }
 
