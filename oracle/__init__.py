@@ -10,7 +10,9 @@ marshals numpy / torch arrays into it.  Every function documents the page sectio
 it restates in the C source.
 
 Functions with no independent pin would be listed here as "parity unpinned";
-every function below is pinned by ``tests/test_oracle_pins.py``.
+every function below is pinned: the layer's steps by ``tests/test_oracle_pins.py``, the
+quantiser variants by ``tests/test_oracle_variants.py`` and the optimizer step by
+``tests/test_oracle_optimizer.py``.
 """
 from __future__ import annotations
 
