@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
+    ap.add_argument("--only-mem", action="store_true",
+                    help="run each HBM-bound kernel of the step (and the optimizer step) once on 7B-MLP-sized "
+                         "inputs larger than L2 (profiling)")
     ap.add_argument("--only-packed", action="store_true",
                     help="run only the packed-weight linear at 16 tokens on the 28672 x 8192 weight (profiling)")
     ap.add_argument("--next", action="store_true",
@@ -239,11 +242,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if args.only_gemv or args.table or args.next or args.only_packed:
+    if args.only_gemv or args.table or args.next or args.only_packed or args.only_mem:
         blbuild.build()
         bl.load()
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        if args.only_packed:
+        if args.only_mem:
+            print(json.dumps({"memory_kernels": mem_once(bl, torch, dev)}), flush=True)
+        elif args.only_packed:
             print(json.dumps({"linear_packed": packed_once(bl, torch, dev)}), flush=True)
         elif args.next:
             print(json.dumps({"next": next_measure(bl, torch, dev, flush, peaks())}), flush=True)
@@ -641,6 +646,32 @@ def gemv_measure(bl, torch, dev, flush, pk):
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
                        "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5")
     return out
+
+
+def mem_once(bl, torch, dev):
+    """One call each of the activation quantiser (8192 x 11008 bf16, RMSNorm fused), the weight
+    quantiser (11008 x 4096 fp32), the RMSNorm backward (8192 x 11008) and the optimizer step
+    with re-quantisation (11008 x 4096): every input is larger than L2 (a small case for a
+    profiler capture; about 2 GB on the device)."""
+    from bit_ternary_qat_b200 import synth
+    gen = synth.generator(5)
+    T, K, N = 8192, 11008, 4096
+    X = synth.normal((T, K), 1.0, gen).to(torch.bfloat16).to(dev)
+    a = bl.bitlinear_act_quant(X)
+    dX = synth.normal((T, K), 1e-2, gen).to(dev)
+    ws = bl.workspace(T, N, K, dev)
+    bl.bitlinear_rmsnorm_backward(X, a["rinv"], dX, ws=ws, dg=torch.empty(K, device=dev))
+    del X, dX, a
+    W = synth.normal((K, N), 0.02, gen).to(dev)
+    q = bl.bitlinear_quant_weight(W, ws=ws)
+    dW = synth.normal((K, N), 1e-3, gen).to(dev)
+    m, v = torch.zeros_like(W), torch.zeros_like(W)
+    step = torch.zeros(1, dtype=torch.int32, device=dev)
+    bl.bitlinear_optimizer_step(W, dW, m, v, step, requantize=True, ws=ws, out=q)
+    torch.cuda.synchronize()
+    assert bl.check_device_status() == 0
+    return {"act_quant": f"{T}x{K} bf16", "rmsnorm_backward": f"{T}x{K}", "quant_weight": f"{K}x{N}",
+            "optimizer_step": f"{K}x{N} with re-quantisation"}
 
 
 def packed_once(bl, torch, dev):
