@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
     const int nvec = K / E;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * R;
 
-    // the rows, widened to fp32, in registers (read from HBM once)
-    float x[R][VPT][E];
+    // the rows' raw 16-byte vectors in registers (read from HBM once, widened on use)
+    uint4 raw[R][VPT];
 #pragma unroll
     for (int q = 0; q < R; ++q) {
         const bool live = t0 + q < T;
@@ -168,17 +168,18 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
             const int v = threadIdx.x + j * NT;
-            const uint4 raw = (live && v < nvec) ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-            for (int e = 0; e < E; ++e) x[q][j][e] = V::elem(raw, e);
+            raw[q][j] = (live && v < nvec) ? __ldcs(xrow + v) : make_uint4(0u, 0u, 0u, 0u);
         }
     }
 
-    // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order
-    float r[R];
+    // r_t = 1 / sqrt(mean x^2 + eps): fp64 sum, fixed order; max |x| on the way
+    float r[R], mx[R];
 #pragma unroll
-    for (int q = 0; q < R; ++q) r[q] = 1.0f;
-    if (apply_norm) {
+    for (int q = 0; q < R; ++q) {
+        r[q] = 1.0f;
+        mx[q] = 0.0f;
+    }
+    {
         double ss[R];
 #pragma unroll
         for (int q = 0; q < R; ++q) {
@@ -187,34 +188,56 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
             for (int j = 0; j < VPT; ++j)
 #pragma unroll
                 for (int e = 0; e < E; ++e) {
-                    const double xd = static_cast<double>(x[q][j][e]);
+                    const float xf = V::elem(raw[q][j], e);
+                    mx[q] = fmaxf(mx[q], fabsf(xf));
+                    const double xd = static_cast<double>(xf);
                     ss[q] = fma(xd, xd, ss[q]);
                 }
         }
-        block_sum_f64<NT, R>(ss, red_d);
+        if (apply_norm) {
+            block_sum_f64<NT, R>(ss, red_d);
 #pragma unroll
-        for (int q = 0; q < R; ++q)
-            r[q] = static_cast<float>(1.0 / sqrt(ss[q] / static_cast<double>(K) + static_cast<double>(eps)));
+            for (int q = 0; q < R; ++q)
+                r[q] = static_cast<float>(1.0 / sqrt(ss[q] / static_cast<double>(K) + static_cast<double>(eps)));
+        }
     }
 
-    // x_hat = fl(fl(x * r) * g) (kept in place of x) and its absmax
+    // x_hat = fl(fl(x * r) * g), recomputed where needed from the raw vector
+    auto xhat = [&](int q, int j, float (&h)[E]) {
+        const int v = threadIdx.x + j * NT;
+        float gk[E];
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+            const float4 gv = (apply_norm && g != nullptr && v < nvec)
+                                  ? __ldg(reinterpret_cast<const float4*>(g + static_cast<int64_t>(v) * E + e))
+                                  : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            gk[e] = gv.x; gk[e + 1] = gv.y; gk[e + 2] = gv.z; gk[e + 3] = gv.w;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            float x = V::elem(raw[q][j], e);
+            if (apply_norm) {
+                x = __fmul_rn(x, r[q]);
+                if (g != nullptr) x = __fmul_rn(x, gk[e]);
+            }
+            h[e] = x;
+        }
+    };
+    // max |x_hat|: without a gain, rounding is monotone, so max |fl(x r)| = fl(max |x| * r)
     float m[R];
 #pragma unroll
     for (int q = 0; q < R; ++q) {
-        m[q] = 0.0f;
+        if (apply_norm && g != nullptr) {
+            m[q] = 0.0f;
 #pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-            const int v = threadIdx.x + j * NT;
+            for (int j = 0; j < VPT; ++j) {
+                float h[E];
+                xhat(q, j, h);
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                float h = x[q][j][e];
-                if (apply_norm) {
-                    h = __fmul_rn(h, r[q]);
-                    if (g != nullptr && v < nvec) h = __fmul_rn(h, __ldg(g + v * E + e));
-                }
-                x[q][j][e] = h;
-                m[q] = fmaxf(m[q], fabsf(h));
+                for (int e = 0; e < E; ++e) m[q] = fmaxf(m[q], fabsf(h[e]));
             }
+        } else {
+            m[q] = apply_norm ? __fmul_rn(mx[q], r[q]) : mx[q];
         }
     }
     block_max_f32<NT, R>(m, red_f);
@@ -247,7 +270,9 @@ __global__ void __launch_bounds__(NT) act_quant_kernel(const void* __restrict__ 
         for (int j = 0; j < VPT; ++j) {
             const int v = threadIdx.x + j * NT;
             if (v >= nvec) continue;
-            quant_store_vec<kBf16, E>(x[q][j], s[q], Xq, Xdq, row_vec0 + v, lut[q]);
+            float h[E];
+            xhat(q, j, h);
+            quant_store_vec<kBf16, E>(h, s[q], Xq, Xdq, row_vec0 + v, lut[q]);
         }
     }
 }
