@@ -171,16 +171,17 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     const int64_t ngroups = n / 16;
     const float4* w4 = reinterpret_cast<const float4*>(W);
     const int64_t round_groups = static_cast<int64_t>(gridDim.x) * kWqThreads * kTqGroups;
+    auto load1 = [&](int64_t r0, int q, float (&wq)[16], int64_t& g) {
+        g = r0 + (static_cast<int64_t>(blockIdx.x) * kTqGroups + q) * kWqThreads + threadIdx.x;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = g < ngroups ? __ldg(w4 + g * 4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            wq[4 * j] = v.x; wq[4 * j + 1] = v.y; wq[4 * j + 2] = v.z; wq[4 * j + 3] = v.w;
+        }
+    };
     auto load = [&](int64_t r0, float (&w)[kTqGroups][16], int64_t (&gi)[kTqGroups]) {
 #pragma unroll
-        for (int q = 0; q < kTqGroups; ++q) {
-            gi[q] = r0 + (static_cast<int64_t>(blockIdx.x) * kTqGroups + q) * kWqThreads + threadIdx.x;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 v = gi[q] < ngroups ? __ldg(w4 + gi[q] * 4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-                w[q][4 * j] = v.x; w[q][4 * j + 1] = v.y; w[q][4 * j + 2] = v.z; w[q][4 * j + 3] = v.w;
-            }
-        }
+        for (int q = 0; q < kTqGroups; ++q) load1(r0, q, w[q], gi[q]);
     };
     float w[kTqGroups][16];
     int64_t gi[kTqGroups];
@@ -220,13 +221,15 @@ __global__ void __launch_bounds__(kWqThreads, 4) ternary_quant_kernel(
     }
     __syncthreads();
     const float thr = s_thr;
-    for (int64_t r0 = 0;;) {
+    // each group's registers are refilled with the next round's group as soon as it is
+    // quantised, so the next round's loads overlap the current round's other group
+    for (int64_t r0 = 0; r0 < ngroups; r0 += round_groups) {
+        const bool more = r0 + round_groups < ngroups;
 #pragma unroll
-        for (int q = 0; q < kTqGroups; ++q)
+        for (int q = 0; q < kTqGroups; ++q) {
             if (gi[q] < ngroups) quantise16<kTau>(w[q], thr, gi[q], wq_i8, wq_bf16, packed);
-        r0 += round_groups;
-        if (r0 >= ngroups) break;
-        load(r0, w, gi);
+            if (more) load1(r0 + round_groups, q, w[q], gi[q]);
+        }
     }
 }
 
