@@ -110,3 +110,60 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "lib_path", lambda: str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_variant_and_optimizer_validation(L):
+    """Host-side rejections of the entry points beyond the step (nothing reaches a device)."""
+    # per-row weight quantiser: (W, N, K, Wq_i8, Wq_bf16, packed, gamma_rows, stream)
+    assert _lib.status("bitlinear_quant_weight_rows", None, 16, 32, None, None, None, FAKE, None) == 1
+    assert _lib.status("bitlinear_quant_weight_rows", FAKE, 16, 32, None, None, None, None, None) == 1
+    assert _lib.status("bitlinear_quant_weight_rows", FAKE, 16, 48, None, None, None, FAKE, None) == 2
+    assert _lib.status("bitlinear_quant_weight_rows", FAKE, 16, 32, ODD, None, None, FAKE, None) == 3
+    # zero threshold: (W, N, K, tau, Wq_i8, Wq_bf16, packed, gamma, ws, ws_bytes, stream)
+    for bad in (-0.5, float("nan"), float("inf")):
+        assert _lib.status("bitlinear_quant_weight_tau", FAKE, 16, 32, bad, None, None, None, FAKE, FAKE, 1 << 20,
+                           None) == 1
+    assert _lib.status("bitlinear_quant_weight_tau", FAKE, 16, 32, 0.7, None, None, None, FAKE, FAKE, 8, None) == 4
+    # per-tensor activation scale: (X, dt, T, K, norm, g, eps, Xq, sx, rinv, Xdq, ws, ws_bytes, stream)
+    assert _lib.status("bitlinear_act_quant_tensor", FAKE, 1, 8, 64, 1, None, 1e-6, FAKE, FAKE, None, None, FAKE,
+                       1 << 20, None) == 1                                      # rinv needed with RMSNorm
+    assert _lib.status("bitlinear_act_quant_tensor", FAKE, 1, 8, 64, 0, None, 1e-6, FAKE, FAKE, None, None, FAKE,
+                       16, None) == 4                                           # block maxima do not fit
+    assert _lib.status("bitlinear_act_quant_tensor", FAKE, 1, 8, 64, 0, None, 1e-6, FAKE, FAKE, None, None, None,
+                       1 << 20, None) == 1
+    assert L.bitlinear_workspace_bytes(8, 16, 64) >= 4 * 1184
+    # per-row linear and GEMV
+    assert _lib.status("bitlinear_linear_rows", FAKE, FAKE, 8, 64, FAKE, None, 32, FAKE, 1, None, None) == 1
+    assert _lib.status("bitlinear_linear_rows", FAKE, FAKE, 8, 40, FAKE, FAKE, 32, FAKE, 1, None, None) == 2
+    assert _lib.status("ternary_gemv_rows", FAKE, FAKE, 32, 64, FAKE, FAKE, 17, FAKE, None, None) == 2
+    assert _lib.status("ternary_gemv_rows", FAKE, FAKE, 32, 96, FAKE, FAKE, 1, FAKE, None, None) == 2
+    # packed-weight linear: (Xq, sx, T, K, packed, gamma, N, Y, y_dt, acc, ws, ws_bytes, stream)
+    assert _lib.status("bitlinear_linear_packed", FAKE, FAKE, 8, 96, FAKE, FAKE, 32, FAKE, 1, None, None, 0,
+                       None) == 2                                               # K % 64
+    assert _lib.status("bitlinear_linear_packed", FAKE, FAKE, 8, 128, None, FAKE, 32, FAKE, 1, None, None, 0,
+                       None) == 1
+    assert _lib.status("bitlinear_linear_packed", FAKE, FAKE, 8, 128, FAKE, FAKE, 32, FAKE, 1, ODD, None, 0,
+                       None) == 3
+    # optimizer: (W, dW, m, v, N, K, lr, b1, b2, eps, wd, max_norm, step, Wq_i8, Wq_bf16, packed, gamma, ws,
+    #             ws_bytes, stream)
+    ok = [FAKE, FAKE, FAKE, FAKE, 16, 32, 1e-3, 0.9, 0.95, 1e-6, 0.01, 1.0, FAKE, None, None, None, None, FAKE,
+          1 << 20, None]
+
+    def opt(**kw):
+        a = list(ok)
+        names = ["W", "dW", "m", "v", "N", "K", "lr", "b1", "b2", "eps", "wd", "mn", "step", "wq", "wbf", "pk",
+                 "gamma", "ws", "ws_bytes", "st"]
+        for k, val in kw.items():
+            a[names.index(k)] = val
+        return _lib.status("bitlinear_optimizer_step", *a)
+    assert opt(step=None) == 1
+    assert opt(m=None) == 1
+    assert opt(lr=-1.0) == 1
+    assert opt(b1=1.0) == 1
+    assert opt(eps=0.0) == 1
+    assert opt(wd=float("nan")) == 1
+    assert opt(wq=FAKE) == 1                       # next codes without gamma
+    assert opt(ws_bytes=64) == 4
+    assert opt(K=48) == 2
+    assert opt(W=ODD) == 3
+    assert L.bitlinear_workspace_bytes(1, 16, 32) >= 2 * 8 * 1184 + 16
