@@ -308,7 +308,12 @@ void launch_act_quant(const void* X, int64_t T, int64_t K, int apply_norm, const
     if (nvec <= 32) return launch_act_quant_w<kBf16, 1>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     if (nvec <= 64) return launch_act_quant_w<kBf16, 2>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     if (nvec <= 128) return launch_act_quant_w<kBf16, 4>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
-    if (nvec <= 256) return launch_act_quant_w<kBf16, 8>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
+    // rows of 129-256 vectors: the warp-per-row kernel, except bf16 rows when there are at
+    // most 8192 of them, where the block-per-row kernel's wider concurrency measured faster
+    // (4096 x 2048 bf16: 10.0 against 11.2 us back to back; 16384 rows: 36.0 against 34.4 us;
+    // fp32 4096 x 1024: 10.9 against 8.0 us)
+    if (nvec <= 256 && (!kBf16 || T > 8192))
+        return launch_act_quant_w<kBf16, 8>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     const int64_t vpt = (nvec + NT - 1) / NT;
     if (vpt <= 1) launch_act_quant_v<kBf16, 1>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
     else if (vpt <= 2) launch_act_quant_v<kBf16, 2>(X, T, K, apply_norm, g, eps, Xq, sx, rinv, Xdq, st);
