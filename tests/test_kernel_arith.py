@@ -231,3 +231,28 @@ def test_packed_gemm_decoder_matches_code_table():
             c = (w >> (2 * i)) & 3
             ref.append((c & 1) - (c >> 1) if c != 3 else 0)
         assert _pk_decode_word(w) == ref, hex(w)
+
+
+def test_packed_gemm_decoder_addresses():
+    """The packed linear's decoder (4 groups x 128 threads; thread dt owns word c = dt % 8 of
+    rows dt / 8 + 16 i) reads each 32-bit word of k-block j of a 128-byte-swizzled packed
+    stage exactly once and writes each 16-byte chunk of the int8 tile exactly once, at the
+    position the 128-byte swizzle gives it (chunk c of row r at chunk c ^ (r % 8))."""
+    for j in range(4):
+        reads, writes = {}, {}
+        for dt in range(128):
+            c, r0 = dt & 7, dt >> 3
+            src_off = ((((2 * j + (c >> 2)) ^ (r0 & 7)) << 4) | ((c & 3) << 2))
+            dst_off = (c ^ (r0 & 7)) << 4
+            for i in range(8):
+                r = r0 + 16 * i
+                assert r & 7 == r0 & 7
+                # logical word c of k-block j of row r: bytes 32 j + 4 c of the 128-byte row,
+                # i.e. chunk 2 j + c // 4, stored at chunk (2 j + c // 4) ^ (r % 8)
+                logical_chunk = 2 * j + (c >> 2)
+                assert src_off == ((logical_chunk ^ (r % 8)) << 4) | ((c & 3) << 2)
+                reads[(r, c)] = reads.get((r, c), 0) + 1
+                assert dst_off == ((c ^ (r % 8)) << 4)
+                writes[(r, dst_off)] = writes.get((r, dst_off), 0) + 1
+        assert len(reads) == 128 * 8 and set(reads.values()) == {1}
+        assert len(writes) == 128 * 8 and set(writes.values()) == {1}
