@@ -327,3 +327,107 @@ def test_oracle_row_sampling_consistency(ora):
     dX_all, _ = ora.rmsnorm_backward(li.X, f["rinv"], None, dxh_all)
     dX_r, _ = ora.rmsnorm_backward(li.X, f["rinv"], None, dxh_all[rows], rows=rows)
     assert np.array_equal(dX_r, dX_all[rows])
+
+
+# ------------------------------------------------------------------------------------
+# the gain vector of the RMSNorm in front of the activation quantiser (P3 §3.1: the
+# layer's RMSNorm(in_features) output feeds activation_quant)
+# ------------------------------------------------------------------------------------
+
+def _gain_case(T=48, K=192, seed=13):
+    """Rows of N(0,1) with a gain vector spread wide enough (0.05 .. 4) that it moves the
+    absmax entry of most rows, so a mishandled gain changes the scale, not just rounding."""
+    gen = torch.Generator().manual_seed(seed)
+    X = torch.randn(T, K, generator=gen, dtype=torch.float32)
+    g = torch.exp(torch.randn(K, generator=gen, dtype=torch.float32) * 0.8).clamp(0.05, 4.0)
+    return X, g
+
+
+def _per_token_f64(X, g, eps):
+    """Library RMSNorm (torch, float64) followed by the per-token absmax quantiser written
+    in float64: s = 127 / max|x_hat|, v = x_hat s, q = clamp(round-half-even(v))."""
+    K = X.shape[1]
+    xh = torch.nn.functional.rms_norm(X.double(), (K,), weight=g.double(), eps=eps).numpy()
+    m = np.max(np.abs(xh), axis=1, keepdims=True)
+    s = 127.0 / np.maximum(m, 1e-5)
+    v = xh * s
+    return np.clip(np.rint(v), -128, 127), s[:, 0], v
+
+
+def _per_tensor_f64(X, g, eps):
+    K = X.shape[1]
+    xh = torch.nn.functional.rms_norm(X.double(), (K,), weight=g.double(), eps=eps).numpy()
+    s = 127.0 / max(float(np.max(np.abs(xh))), 1e-5)
+    v = xh * s
+    return np.clip(np.rint(v), -128, 127), np.full(X.shape[0], s), v
+
+
+def _agrees_f64(xq, s, xdq, ref):
+    """fp32 oracle output vs the float64 restatement.  x_hat in fp32 carries three roundings
+    (r, x r, (x r) g) and s one more, so s agrees to 2^-20 relative and x_hat s to
+    127 * 2^-20 absolute (< 1.3e-4): a code may differ by one only where the float64
+    product lies that close to a .5 tie.  X_dq = q / s to 2^-20 relative."""
+    ref_q, ref_s, ref_v = ref
+    if not np.all(np.abs(s.astype(np.float64) - ref_s) <= 2.0 ** -20 * ref_s):
+        return False
+    d = xq.astype(np.int64) - ref_q.astype(np.int64)
+    near_tie = np.abs(np.abs(ref_v - np.floor(ref_v)) - 0.5) < 1.3e-4
+    if not (np.all(np.abs(d) <= 1) and np.all((d == 0) | near_tie)):
+        return False
+    want = xq.astype(np.float64) / ref_s[:, None]
+    return bool(np.all(np.abs(xdq.astype(np.float64) - want) <= 2.0 ** -20 * np.abs(want)))
+
+
+def test_act_quant_gain_matches_torch_rms_norm(ora):
+    X, g = _gain_case()
+    eps = 1e-6
+    r = ora.rmsnorm_rinv(X, eps)
+    xq, s, xdq = ora.act_quant(X, r, g)
+    ref = _per_token_f64(X, g, eps)
+    assert _agrees_f64(xq, s, xdq, ref)
+    # the case is informative: the gain moved the absmax entry of most rows
+    arg_gain = np.argmax(np.abs(ref[2]), axis=1)
+    arg_raw = np.argmax(np.abs(X.numpy()), axis=1)
+    assert np.mean(arg_gain != arg_raw) > 0.5
+
+
+def test_act_quant_gain_pin_rejects_planted_mistakes(ora):
+    """Each plausible slip in the gain path, planted by feeding the oracle the mistaken
+    operands, must fail the float64 pin above."""
+    X, g = _gain_case()
+    eps = 1e-6
+    Xn, gn = X.numpy(), g.numpy()
+    r = ora.rmsnorm_rinv(X, eps)
+    ref = _per_token_f64(X, g, eps)
+    mistakes = {
+        # gain dropped (x_hat = x r)
+        "dropped": ora.act_quant(X, r, None),
+        # gain applied before the normalisation statistic (r taken over x g)
+        "inside_rms": ora.act_quant((Xn * gn).astype(np.float32), ora.rmsnorm_rinv(Xn * gn, eps), None),
+        # gain indexed in reverse (a transposed / mis-strided gain read)
+        "reversed": ora.act_quant(X, r, gn[::-1].copy()),
+        # gain applied twice
+        "squared": ora.act_quant(X, r, (gn * gn).astype(np.float32)),
+        # gain divided instead of multiplied
+        "inverted": ora.act_quant(X, r, (1.0 / gn).astype(np.float32)),
+    }
+    for name, (q_b, s_b, xdq_b) in mistakes.items():
+        assert not _agrees_f64(q_b, s_b, xdq_b, ref), name
+
+
+def test_act_quant_tensor_gain_matches_torch_rms_norm(ora):
+    X, g = _gain_case(T=40, K=160, seed=17)
+    eps = 1e-6
+    r = ora.rmsnorm_rinv(X, eps)
+    xq, s, xdq = ora.act_quant_tensor(X, r, g)
+    ref = _per_tensor_f64(X, g, eps)
+    assert _agrees_f64(xq, s, xdq, ref)
+    Xn, gn = X.numpy(), g.numpy()
+    mistakes = {
+        "dropped": ora.act_quant_tensor(X, r, None),
+        "inside_rms": ora.act_quant_tensor((Xn * gn).astype(np.float32), ora.rmsnorm_rinv(Xn * gn, eps), None),
+        "reversed": ora.act_quant_tensor(X, r, gn[::-1].copy()),
+        "per_token_scale": ora.act_quant(X, r, g),
+    }
+    for name, (q_b, s_b, xdq_b) in mistakes.items():
+        assert not _agrees_f64(q_b, s_b, xdq_b, ref), name
