@@ -870,6 +870,30 @@ bl_status gemv_entry(const uint8_t* Wpacked, const float* gamma, int gamma_strid
     return launch_gemv<2>(Wpacked, gamma, gamma_stride, N, K, xq, sx, B, y, acc, st, dev);
 }
 
+namespace {
+// cuCtxGetCurrent through the runtime's driver entry point (the library does not link libcuda)
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+constexpr int kScratchDevices = 64;
+struct ScratchAddr {
+    CUcontext ctx;
+    void* addr;
+};
+}  // namespace
+
 bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, int8_t* Wq_i8, uint16_t* Wq_bf16,
                                          uint8_t* Wpacked, float* gamma, void* stream) {
     BL_TRY(check_ptr(W, "W", true));
@@ -884,22 +908,33 @@ bl_status bitlinear_quant_weight_noalloc(const float* W, int64_t N, int64_t K, i
                "the built-in scratch holds %d partial sums, this weight needs %d", bl::kWqMaxPartials, parts);
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
-    // set-up, once per device: the device address of the scratch array
-    static std::mutex mu;
-    static void* addr[64] = {};
-    int dev_id = 0;
+    // set-up, once per device and context: the device address of the scratch array.  The
+    // address belongs to the context that loaded this module, so it is cached together with
+    // that context and looked up again when the current context differs (after a
+    // cudaDeviceReset the device gets a new primary context and the old address is gone).
+    int dev_id = -1;
     cudaError_t e = cudaGetDevice(&dev_id);
     if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    BL_REQUIRE(dev_id >= 0 && dev_id < kScratchDevices, BL_ERR_INVALID_ARG,
+               "device index %d is beyond the %d devices the scratch table covers", dev_id, kScratchDevices);
+    CtxGetCurrentFn ctx_fn = ctx_get_current_fn();
+    BL_REQUIRE(ctx_fn != nullptr, BL_ERR_CUDA, "cuCtxGetCurrent is unavailable");
+    CUcontext ctx = nullptr;
+    CUresult cr = ctx_fn(&ctx);
+    BL_REQUIRE(cr == CUDA_SUCCESS && ctx != nullptr, BL_ERR_CUDA, "cuCtxGetCurrent failed (%d)", (int)cr);
     void* scratch = nullptr;
     {
+        static std::mutex mu;
+        static ScratchAddr cache[kScratchDevices] = {};
         std::lock_guard<std::mutex> lk(mu);
-        if (addr[dev_id] == nullptr) {
+        if (cache[dev_id].addr == nullptr || cache[dev_id].ctx != ctx) {
             void* p = nullptr;
             e = cudaGetSymbolAddress(&p, g_quant_scratch);
             if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-            addr[dev_id] = p;
+            cache[dev_id].addr = p;
+            cache[dev_id].ctx = ctx;
         }
-        scratch = addr[dev_id];
+        scratch = cache[dev_id].addr;
     }
     // pass 1 writes every partial that pass 2 reads, so nothing in the scratch needs clearing
     return run_quant_weight(W, n, scratch, Wq_i8, Wq_bf16, Wpacked, gamma, static_cast<cudaStream_t>(stream), dev);

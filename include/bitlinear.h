@@ -120,8 +120,11 @@ BL_API bl_status bitlinear_quant_weight(const float* W, int64_t N, int64_t K,
  *     sums is capped at 1184); a weight that needed more would be rejected with
  *     BL_ERR_UNSUPPORTED_SHAPE.
  *   - Set-up: the first call on each device looks up the scratch array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with the device's
+ *     current context; a call that finds another context current (after cudaDeviceReset)
+ *     looks it up again.  Make the first call on a device, and the first after a reset,
+ *     before any stream capture.  Device ordinals 0..63 are covered; a call on a device
+ *     beyond them returns BL_ERR_INVALID_ARG.
  *   - Sharing: all calls on a device share the one array and it keeps the last call's
  *     contents.  Nothing in it needs to start at zero (every partial a call reads was
  *     written by that call), but calls that overlap on the GPU (for example on two

@@ -40,3 +40,25 @@ def test_noalloc_matches_workspace_entry_point(bl):
         assert bl.check_device_status() == 0
         for k in ("gamma", "wq_i8", "wq_bf16", "packed"):
             assert torch.equal(out[k], ref[k]), (N, K, k)
+
+
+def test_noalloc_allocates_nothing(bl):
+    """Once the first call has looked up the scratch address, a call changes neither torch's
+    allocator count nor the device's free memory: no allocation happens on its path."""
+    stream = torch.cuda.current_stream().cuda_stream
+    N, K = 1024, 512
+    W = synth.normal((N, K), synth.W_STD, synth.generator(23)).to(DEV)
+    out = _outputs(N, K)
+    args = (W.data_ptr(), N, K, out["wq_i8"].data_ptr(), out["wq_bf16"].data_ptr(), out["packed"].data_ptr(),
+            out["gamma"].data_ptr(), stream)
+    _lib.call("bitlinear_quant_weight_noalloc", *args)          # set-up call
+    torch.cuda.synchronize()
+    torch_before = torch.cuda.memory_allocated()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        _lib.call("bitlinear_quant_weight_noalloc", *args)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == torch_before
+    assert free_after == free_before
+    assert bl.check_device_status() == 0
