@@ -167,3 +167,15 @@ def test_variant_and_optimizer_validation(L):
     assert opt(K=48) == 2
     assert opt(W=ODD) == 3
     assert L.bitlinear_workspace_bytes(1, 16, 32) >= 2 * 8 * 1184 + 16
+
+
+def test_status_values_match_header():
+    """The numeric bl_status values of the header, which differ from a plain
+    OK / invalid / shape / CUDA / timeout list by the misalignment, workspace and device
+    codes, are the ones the binding decodes."""
+    text = open(HEADER).read()
+    body = text[text.index("typedef enum {"):text.index("} bl_status;")]
+    vals = {name: int(v) for name, v in re.findall(r"\b(BL_\w+)\s*=\s*(\d+)", body)}
+    assert vals == {"BL_OK": 0, "BL_ERR_INVALID_ARG": 1, "BL_ERR_UNSUPPORTED_SHAPE": 2, "BL_ERR_MISALIGNED": 3,
+                    "BL_ERR_WORKSPACE": 4, "BL_ERR_CUDA": 5, "BL_ERR_TIMEOUT": 6, "BL_ERR_DEVICE": 7}
+    assert {v: k for k, v in vals.items()} == _lib.STATUS_NAMES
