@@ -3,17 +3,22 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the whole hot path over one batch of the "square" workload
-(one BitLinear 2048 -> 2048, 4096 tokens per GPU, bf16 X / dY, fp32 latent W):
-weight quantisation (absmean + ternary round + 2-bit pack), RMSNorm + int8 activation
-quantisation, the int8 x ternary contraction, the straight-through backward (grad
-input GEMM, RMSNorm backward, grad weight GEMM), and a 16-token decode GEMV over the
-freshly packed weights.  With N > 1 GPUs each rank holds its own 4096 tokens (weak
-scaling) and the weight gradient is summed over ranks with an NCCL all-reduce.
+One step = one pass of the whole hot path over the seven projections of a 7B-shaped
+transformer layer (q, k, v, o 4096 -> 4096; gate, up 4096 -> 11008; down 11008 -> 4096),
+16384 tokens per GPU, bf16 X / dY, fp32 latent W.  For every projection: weight
+quantisation (absmean + ternary round + 2-bit pack), RMSNorm + int8 activation
+quantisation, the int8 x ternary contraction, the straight-through backward (grad-input
+GEMM, RMSNorm backward, weight-gradient GEMM) and a 16-token decode GEMV over the freshly
+packed codes.  With N > 1 GPUs each rank holds its own 16384 tokens (weak scaling) and each
+projection's weight gradient is summed over ranks with an NCCL all-reduce that overlaps
+the next projection's work.
 
-Prints one JSON line (rank 0).  Inputs are synthetic and seeded (bit_ternary_qat_b200.synth).
-L2 is flushed (a 512 MB write) before every timed step; each step is timed with CUDA
-events on the launching stream, the per-rank sum is max-reduced over ranks.
+Prints one JSON line (rank 0).  Inputs are synthetic and seeded (bit_ternary_qat_b200.synth;
+rank 0 draws exactly the parity tests' layer7b inputs).  L2 is flushed (a 512 MB write)
+before every timed step; each step is timed with CUDA events on the launching stream and
+the sum over steps is max-reduced over ranks.  The roofline denominators are the measured
+peaks of MEASURED_PEAKS.json (HBM copy, cuBLAS bf16 burst) and, for int8, the library's own
+tcgen05 kind::i8 peak loop timed at the start of the run.
 """
 from __future__ import annotations
 
@@ -30,10 +35,15 @@ from datetime import timedelta
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-T_TOK, D_IN, D_OUT = 4096, 2048, 2048
+WORKLOAD_NAME = "layer7b"
+T_TOK = 16384
 DECODE_B = 16
 METRIC = "BitLinear fwd+bwd tokens/s & % of TC peak; packed-ternary GEMV HBM GB/s"
-WORKLOAD = "square: BitLinear 2048->2048, 4096 tokens/GPU, bf16 X/dY, fp32 W; quant+fwd+bwd+16-token decode GEMV"
+WORKLOAD = ("layer7b: the 7 projections of a 7B-shaped layer (q,k,v,o 4096->4096; gate,up 4096->11008; "
+            "down 11008->4096), 16384 tokens/GPU, bf16 X/dY, fp32 W; per projection quant+fwd+bwd and a "
+            "16-token decode GEMV")
+PIECES = ["quant_weight", "act_quant", "linear_i8", "grad_input", "rmsnorm_bwd", "grad_weight", "decode_gemv"]
+CPU_SAMPLE_TOKENS = 16
 
 
 def parse():
@@ -43,7 +53,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-gemv", action="store_true", help="skip the decode-GEMV side measurement")
+    ap.add_argument("--no-sub", action="store_true", help="skip the decode-GEMV and other-configuration records")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only-gemv", action="store_true", help="run only the decode-GEMV measurement (profiling)")
     ap.add_argument("--only-mem", action="store_true",
@@ -51,6 +61,10 @@ def parse():
                          "inputs larger than L2 (profiling)")
     ap.add_argument("--only-packed", action="store_true",
                     help="run only the packed-weight linear at 16 tokens on the 28672 x 8192 weight (profiling)")
+    ap.add_argument("--only-gemm", choices=["linear_i8", "grad_input", "grad_weight"], default=None,
+                    help="run three launches of one GEMM of the step on the gate projection's shape "
+                         "(16384 tokens, 4096 -> 11008; profiling)")
+    ap.add_argument("--only-peak", action="store_true", help="run only the tensor-pipe peak probe")
     ap.add_argument("--next", action="store_true",
                     help="time the fused optimizer step and the quantiser variants back to back; one JSON object, "
                          "not the bench line")
@@ -86,15 +100,15 @@ def kernel_src_hash() -> str:
 
 
 def ncu_traffic(kernel_key: str):
-    """DRAM bytes per launch of a kernel from the committed ncu summary, if it was taken on
-    the current kernel sources; otherwise None."""
+    """DRAM bytes per launch of a kernel of the step, from the committed ncu summary, if it
+    was taken on the current kernel sources; otherwise None."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
             d = json.load(f)
-        if d.get("src_sha") != kernel_src_hash():
+        if d.get("src_sha") != kernel_src_hash() or d.get("workload") != WORKLOAD_NAME:
             return None
         v = d.get("kernels", {}).get(kernel_key, {}).get("dram_bytes_per_launch")
         return None if v is None else float(v)
@@ -111,7 +125,6 @@ class ClockSampler:
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
         self.proc = None
-        self.lines = []
 
     def start(self):
         try:
@@ -130,7 +143,7 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out = ""
-        sm, smax, reasons = [], [], set()
+        sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in out.strip().splitlines():
             parts = [p.strip() for p in ln.split(",")]
@@ -141,13 +154,27 @@ class ClockSampler:
                 smax.append(float(parts[2]))
             except ValueError:
                 continue
+            try:
+                power.append(float(parts[3]))
+            except ValueError:
+                pass
             for nm, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+               "samples": len(sm)}
+        if power:
+            out["power_w_max"] = max(power)
+        return out
+
+
+def gpu_id_of(torch, dev) -> str:
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return str(dev.index or 0)
 
 
 # ------------------------------------------------------------------------------------
@@ -155,14 +182,15 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------
 
 def oracle_step(ora, li, t_s: int):
-    """The oracle's pass over the hot path on the first t_s tokens (weight quantisation
-    over the full W).  Returns seconds."""
+    """The oracle's pass over the hot path on the first t_s tokens of one layer (weight
+    quantisation over the full W).  Returns (seconds, seconds of the weight quantisation)."""
     X = li.X[:t_s].float().numpy()
     dY = li.dY[:t_s].float().numpy()
     W = li.W.numpy()
     t0 = time.perf_counter()
     gamma, wq = ora.quant_weight(W)
     packed = ora.pack(wq)
+    t_wq = time.perf_counter() - t0
     r = ora.rmsnorm_rinv(X, 1e-6)
     xq, s, xdq = ora.act_quant(X, r, None)
     acc = ora.int_gemm(xq, wq)
@@ -173,27 +201,40 @@ def oracle_step(ora, li, t_s: int):
     ora.grad_weight(dY, xdq_b)
     b = min(DECODE_B, t_s)
     ora.gemv(packed, gamma, W.shape[1], xq[:b], s[:b])
-    return time.perf_counter() - t0
+    return time.perf_counter() - t0, t_wq
+
+
+def oracle_workload_step(ora, lis, t_s: int):
+    """One oracle step over every layer of the workload on a t_s-token sample.  Returns
+    (measured seconds, seconds extrapolated to the full token count): per layer, the weight
+    quantisation once plus the token-proportional rest scaled by T / t_s."""
+    meas, extra = 0.0, 0.0
+    for li in lis:
+        T = li.X.shape[0]
+        full, wq = oracle_step(ora, li, t_s)
+        meas += full
+        extra += wq + (full - wq) * (T / t_s)
+    return meas, extra
 
 
 def cpu_baseline(target_s: float = 12.0):
-    """The oracle on the square workload, repeated until about `target_s` seconds of CPU work."""
+    """The oracle on the layer7b workload, 16 tokens per projection per step (full weight
+    quantisation), repeated until about `target_s` seconds of CPU work, extrapolated to
+    16384 tokens."""
     import oracle as ora
     from bit_ternary_qat_b200 import synth
     ora.build()
-    li = synth.workload_inputs("square")[0]
-    t_s = 64
-    dt = oracle_step(ora, li, t_s)
-    while dt < target_s / 4 and t_s < T_TOK:
-        t_s = min(T_TOK, t_s * 4)
-        dt = oracle_step(ora, li, t_s)
-    steps, tot = 1, dt
-    while tot < target_s:
-        tot += oracle_step(ora, li, t_s)
+    lis = synth.workload_inputs(WORKLOAD_NAME)
+    steps, meas, extra = 0, 0.0, 0.0
+    while meas < target_s:
+        m, e = oracle_workload_step(ora, lis, CPU_SAMPLE_TOKENS)
+        meas += m
+        extra += e
         steps += 1
-    return {"value": steps * t_s / tot, "unit": "tokens/s", "cores": ora.num_threads(), "kind": "oracle",
-            "sample": f"{steps} oracle step(s) on {t_s} of the {T_TOK} tokens of the square workload "
-                      f"(weight quantisation over the full 2048x2048 W included), {tot:.1f} s"}
+    return {"value": T_TOK * steps / extra, "unit": "tokens/s", "cores": ora.num_threads(), "kind": "oracle",
+            "sample": f"{steps} oracle step(s), each: every projection's full weight quantisation and "
+                      f"{CPU_SAMPLE_TOKENS} of its {T_TOK} tokens (fwd + bwd + decode GEMV), {meas:.1f} s measured; "
+                      f"tokens/s extrapolated linearly in tokens (weight quantisation once per projection)"}
 
 
 def run_reference(args, rank, world):
@@ -202,24 +243,59 @@ def run_reference(args, rank, world):
     import oracle as ora
     from bit_ternary_qat_b200 import synth
     ora.build()
-    li = synth.workload_inputs("square")[0]
-    t_s = 256
+    lis = synth.workload_inputs(WORKLOAD_NAME)
     for _ in range(args.warmup):
-        oracle_step(ora, li, t_s)
-    tot = 0.0
+        oracle_workload_step(ora, lis, CPU_SAMPLE_TOKENS)
+    meas, extra = 0.0, 0.0
     for _ in range(args.steps):
-        tot += oracle_step(ora, li, t_s)
-    value = t_s * args.steps / tot
+        m, e = oracle_workload_step(ora, lis, CPU_SAMPLE_TOKENS)
+        meas += m
+        extra += e
+    value = T_TOK * args.steps / extra
+    sample = (f"each step: every projection's full weight quantisation and {CPU_SAMPLE_TOKENS} of its {T_TOK} "
+              f"tokens (fwd + bwd + decode GEMV), {meas / args.steps:.2f} s measured per step; tokens/s "
+              f"extrapolated linearly in tokens (weight quantisation once per projection)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * extra / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
-        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens_per_step": t_s},
+        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens_per_gpu": T_TOK,
+                                        "sampled_tokens_per_step": CPU_SAMPLE_TOKENS},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "kind": "oracle", "cores": ora.num_threads(),
-                         "sample": f"each step: the oracle on {t_s} of {T_TOK} tokens (full weight quantisation)"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------
+# tensor-pipe peak (the library's own tcgen05 loop; denominator of the int8 GEMMs)
+# ------------------------------------------------------------------------------------
+
+def probe_tensor_peaks(bl, torch, dev, iters: int = 20000, reps: int = 5):
+    """Each of kind::i8 / kind::f16 x cta_group::1 / ::2: one short warm-up launch, then `reps`
+    timed launches (about 5 ms each); the best rate of each is its burst peak in TFLOP/s (or
+    TOPS for int8)."""
+    out = {}
+    for kind in ("int8", "bf16"):
+        for pair in (False, True):
+            bl.mma_peak_probe(kind, pair, max(1, iters // 4))
+            torch.cuda.synchronize()
+            rates = []
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                ops = bl.mma_peak_probe(kind, pair, iters)
+                b.record()
+                torch.cuda.synchronize()
+                rates.append(ops / (a.elapsed_time(b) * 1e-3) / 1e12)
+            out[f"{kind}_{'cta_pair' if pair else 'cta'}"] = max(rates)
+    assert bl.check_device_status() == 0
+    out["int8"] = max(out["int8_cta"], out["int8_cta_pair"])
+    out["bf16"] = max(out["bf16_cta"], out["bf16_cta_pair"])
+    out["how"] = (f"tcgen05.mma loop from fixed pseudo-random shared-memory operands into TMEM, no global "
+                  f"traffic; {iters} x 4 instructions per CTA (or pair) per launch, best of {reps} launches")
+    return out
 
 
 # ------------------------------------------------------------------------------------
@@ -242,9 +318,16 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if args.only_gemv or args.table or args.next or args.only_packed or args.only_mem:
+    if (args.only_gemv or args.table or args.next or args.only_packed or args.only_mem or args.only_gemm
+            or args.only_peak):
         blbuild.build()
         bl.load()
+        if args.only_peak:
+            print(json.dumps({"tensor_peaks": probe_tensor_peaks(bl, torch, dev)}), flush=True)
+            return
+        if args.only_gemm:
+            print(json.dumps({"gemm": gemm_once(bl, torch, dev, args.only_gemm)}), flush=True)
+            return
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
         if args.only_mem:
             print(json.dumps({"memory_kernels": mem_once(bl, torch, dev)}), flush=True)
@@ -264,87 +347,96 @@ def main():
     if world > 1:
         dist.barrier()
     bl.load()
+    pk = peaks()
+    f32, bf16, i8, u8 = torch.float32, torch.bfloat16, torch.int8, torch.uint8
+
+    # ---------------------------------------------------------------- tensor-pipe peaks
+    clk_probe = ClockSampler(gpu_id_of(torch, dev)) if rank == 0 else None
+    if clk_probe:
+        clk_probe.start()
+        time.sleep(0.3)
+    tpk = probe_tensor_peaks(bl, torch, dev)
+    if clk_probe:
+        tpk["clocks"] = clk_probe.stop()
 
     # ---------------------------------------------------------------- inputs (HBM resident)
-    wl = synth.WORKLOADS["square"]
-    gen = synth.generator(wl.seed)
-    W_h = synth.normal((D_OUT, D_IN), synth.W_STD, gen)                  # same W on every rank
-    gen_r = synth.generator(wl.seed * 1000 + rank)                       # rank's own tokens
-    X_h = synth.normal((T_TOK, D_IN), 1.0, gen_r).to(torch.bfloat16)
-    dY_h = synth.normal((T_TOK, D_OUT), synth.DY_STD_BF16, gen_r).to(torch.bfloat16)
-    W, X, dY = W_h.to(dev), X_h.to(dev), dY_h.to(dev)
-
-    f32, bf16, i8, u8 = torch.float32, torch.bfloat16, torch.int8, torch.uint8
-    bufs = dict(
-        gamma=torch.empty(1, dtype=f32, device=dev), wq_i8=torch.empty(D_OUT, D_IN, dtype=i8, device=dev),
-        wq_bf16=torch.empty(D_OUT, D_IN, dtype=bf16, device=dev),
-        packed=torch.empty(D_OUT, D_IN // 4, dtype=u8, device=dev),
-        xq=torch.empty(T_TOK, D_IN, dtype=i8, device=dev), sx=torch.empty(T_TOK, dtype=f32, device=dev),
-        rinv=torch.empty(T_TOK, dtype=f32, device=dev), xdq=torch.empty(T_TOK, D_IN, dtype=bf16, device=dev),
-        y=torch.empty(T_TOK, D_OUT, dtype=bf16, device=dev), dX=torch.empty(T_TOK, D_IN, dtype=f32, device=dev),
-        dW=torch.empty(D_OUT, D_IN, dtype=f32, device=dev), dg=torch.empty(D_IN, dtype=f32, device=dev),
-        ydec=torch.empty(DECODE_B, D_OUT, dtype=f32, device=dev),
-        ws=bl.workspace(T_TOK, D_OUT, D_IN, dev))
+    lis = synth.workload_inputs(WORKLOAD_NAME)          # rank 0: the parity tests' inputs
+    if rank > 0:                                        # same W; the rank's own tokens
+        gen_r = synth.generator(synth.WORKLOADS[WORKLOAD_NAME].seed * 1000 + rank)
+        for li in lis:
+            li.X = synth.normal(tuple(li.X.shape), 1.0, gen_r).to(bf16)
+            li.dY = synth.normal(tuple(li.dY.shape), synth.DY_STD_BF16, gen_r).to(bf16)
+    maxK = max(li.W.shape[1] for li in lis)
+    maxN = max(li.W.shape[0] for li in lis)
+    T = T_TOK
+    shared = dict(
+        gamma=torch.empty(1, dtype=f32, device=dev), wq_i8=torch.empty(maxN * maxK, dtype=i8, device=dev),
+        wq_bf16=torch.empty(maxN * maxK, dtype=bf16, device=dev),
+        packed=torch.empty(maxN * maxK // 4, dtype=u8, device=dev),
+        xq=torch.empty(T * maxK, dtype=i8, device=dev), sx=torch.empty(T, dtype=f32, device=dev),
+        rinv=torch.empty(T, dtype=f32, device=dev), xdq=torch.empty(T * maxK, dtype=bf16, device=dev),
+        y=torch.empty(T * maxN, dtype=bf16, device=dev), dX=torch.empty(T * maxK, dtype=f32, device=dev),
+        dg=torch.empty(maxK, dtype=f32, device=dev), ydec=torch.empty(DECODE_B * maxN, dtype=f32, device=dev))
+    ws = bl.workspace(T, maxN, maxK, dev)
+    layers = []
+    for li in lis:
+        N, K = li.W.shape
+        fo = dict(gamma=shared["gamma"], wq_i8=shared["wq_i8"][:N * K].view(N, K),
+                  wq_bf16=shared["wq_bf16"][:N * K].view(N, K), packed=shared["packed"][:N * K // 4].view(N, K // 4),
+                  y=shared["y"][:T * N].view(T, N), xq=shared["xq"][:T * K].view(T, K), sx=shared["sx"],
+                  rinv=shared["rinv"], xdq=shared["xdq"][:T * K].view(T, K))
+        layers.append(dict(name=li.shape.name, N=N, K=K, W=li.W.to(dev), X=li.X.to(dev), dY=li.dY.to(dev),
+                           dW=torch.empty(N, K, dtype=f32, device=dev), fo=fo,
+                           dX=shared["dX"][:T * K].view(T, K), dg=shared["dg"][:K],
+                           ydec=shared["ydec"][:DECODE_B * N].view(DECODE_B, N)))
     flush = torch.empty(512 * 1024 * 1024, dtype=u8, device=dev)        # > 126 MB L2
-
-    # names of the timed pieces, in step order (each is one public call)
-    PIECES = ["quant_weight", "act_quant", "linear_i8", "grad_input", "rmsnorm_bwd", "grad_weight",
-              "allreduce_dW", "decode_gemv"]
-
-    def step(ev=None, inputs=None, dom_ev=None):
-        b = bufs
-        Wi, Xi, dYi = inputs if inputs is not None else (W, X, dY)
-        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
-        if dom_ev is not None:      # bracket only the dominant kernel (grad-input GEMM)
-            rec = (lambda i: dom_ev[i - 3].record() if i in (3, 4) else None)
-        rec(0)
-        bl.bitlinear_quant_weight(Wi, ws=b["ws"], out=b)
-        rec(1)
-        bl.bitlinear_act_quant(Xi, apply_rmsnorm=True, out=b)
-        rec(2)
-        bl.bitlinear_linear(b["xq"], b["sx"], b["wq_i8"], b["gamma"], y=b["y"])
-        rec(3)
-        bl.bitlinear_grad_input(dYi, b["wq_bf16"], b["gamma"], dXhat=b["dX"])
-        rec(4)
-        bl.bitlinear_rmsnorm_backward(Xi, b["rinv"], b["dX"], ws=b["ws"], dg=b["dg"])
-        rec(5)
-        bl.bitlinear_backward_weight(dYi, b["xdq"], dW=b["dW"])
-        rec(6)
-        dp.allreduce_weight_grad(b["dW"])
-        rec(7)
-        bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B], y=b["ydec"])
-        rec(8)
-
-    # The timed step runs the forward as one call (bitlinear_forward_qat: quantisation of W and
-    # X, then the GEMM) and the backward pieces; after the grad-input GEMM the RMSNorm
-    # backward and the decode GEMV go to a second stream and run beside the weight-gradient
-    # GEMM (its persistent CTAs leave room for the RMSNorm blocks).  Measured against other
-    # orders (weight quantisation beside activation quantisation as well, the weight-gradient
-    # GEMM first): this one is the fastest; the calls before the fork keep their
-    # programmatic-dependent-launch overlap.
     ovs = torch.cuda.Stream(device=dev)
 
-    def step_overlap(dom_ev=None, inputs=None, with_tail=True):
-        b = bufs
-        Wi, Xi, dYi = inputs if inputs is not None else (W, X, dY)
+    # One projection's step.  The forward is one call (bitlinear_forward_qat: the weight
+    # quantiser's |W| sums, the activation quantiser, the ternary codes, the int8 GEMM); after
+    # the grad-input GEMM the RMSNorm backward and the decode GEMV go to a second stream and
+    # run beside the weight-gradient GEMM.  `dom` brackets one GEMM with two events.
+    def layer_step(L, dom=None, inputs=None):
+        fo = L["fo"]
+        Wi, Xi, dYi = inputs if inputs is not None else (L["W"], L["X"], L["dY"])
         main = torch.cuda.current_stream(dev)
-        # weight + activation quantisation and the forward GEMM in one call
-        bl.bitlinear_forward_qat(Xi, Wi, ws=b["ws"], out=b)
-        if dom_ev is not None:
-            dom_ev[0].record()
-        bl.bitlinear_grad_input(dYi, b["wq_bf16"], b["gamma"], dXhat=b["dX"])
-        if dom_ev is not None:
-            dom_ev[1].record()
+        bl.bitlinear_forward_qat(Xi, Wi, ws=ws, out=fo)
+        if dom is not None and dom[0] == "grad_input":
+            dom[1].record()
+        bl.bitlinear_grad_input(dYi, fo["wq_bf16"], fo["gamma"], dXhat=L["dX"])
+        if dom is not None and dom[0] == "grad_input":
+            dom[2].record()
         ovs.wait_stream(main)
         with torch.cuda.stream(ovs):
-            bl.bitlinear_rmsnorm_backward(Xi, b["rinv"], b["dX"], ws=b["ws"], dg=b["dg"])
-            if with_tail:
-                bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B],
-                                y=b["ydec"])
-        bl.bitlinear_backward_weight(dYi, b["xdq"], dW=b["dW"])
-        if with_tail:
-            dp.allreduce_weight_grad(b["dW"])
+            bl.bitlinear_rmsnorm_backward(Xi, fo["rinv"], L["dX"], ws=ws, dg=L["dg"])
+            bl.ternary_gemv(fo["packed"], fo["gamma"], L["K"], fo["xq"][:DECODE_B], fo["sx"][:DECODE_B],
+                            y=L["ydec"])
+        if dom is not None and dom[0] == "grad_weight":
+            dom[1].record()
+        bl.bitlinear_backward_weight(dYi, fo["xdq"], dW=L["dW"])
+        if dom is not None and dom[0] == "grad_weight":
+            dom[2].record()
         main.wait_stream(ovs)
+
+    # The same work as separate sequential calls with an event before each (piece times).
+    def layer_pieces(L, ev):
+        fo = L["fo"]
+        q = dict(gamma=fo["gamma"], wq_i8=fo["wq_i8"], wq_bf16=fo["wq_bf16"], packed=fo["packed"])
+        a = dict(xq=fo["xq"], sx=fo["sx"], rinv=fo["rinv"], xdq=fo["xdq"])
+        ev[0].record()
+        bl.bitlinear_quant_weight(L["W"], ws=ws, out=q)
+        ev[1].record()
+        bl.bitlinear_act_quant(L["X"], apply_rmsnorm=True, out=a)
+        ev[2].record()
+        bl.bitlinear_linear(fo["xq"], fo["sx"], fo["wq_i8"], fo["gamma"], y=fo["y"])
+        ev[3].record()
+        bl.bitlinear_grad_input(L["dY"], fo["wq_bf16"], fo["gamma"], dXhat=L["dX"])
+        ev[4].record()
+        bl.bitlinear_rmsnorm_backward(L["X"], fo["rinv"], L["dX"], ws=ws, dg=L["dg"])
+        ev[5].record()
+        bl.bitlinear_backward_weight(L["dY"], fo["xdq"], dW=L["dW"])
+        ev[6].record()
+        bl.ternary_gemv(fo["packed"], fo["gamma"], L["K"], fo["xq"][:DECODE_B], fo["sx"][:DECODE_B], y=L["ydec"])
 
     def sync_all():
         torch.cuda.synchronize()
@@ -352,81 +444,55 @@ def main():
             dist.barrier()
             torch.cuda.synchronize()
 
-    # ---------------------------------------------------------------- warm-up
+    # ---------------------------------------------------------------- warm-up (eager)
     for _ in range(max(3, args.warmup)):
-        step()
+        for L in layers:
+            layer_step(L)
+        for L in layers:
+            dp.allreduce_weight_grad(L["dW"])
     sync_all()
     assert bl.check_device_status() == 0
 
-    # ---------------------------------------------------------------- CUDA graphs of one step
-    # The step is 9 library calls; replaying it as a captured graph removes the Python /
-    # ctypes launch overhead from the device timeline.  The timed graph holds the kernels
-    # alone (consecutive kernels overlap their launch with the previous kernel's drain); a
-    # second graph with event nodes between the calls times every piece, in a separate loop
-    # whose time does not enter the step time.
-    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(9)]
-    side = torch.cuda.Stream(device=dev)
-    side.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(side):
-        step()
-        step_overlap(with_tail=(world == 1))
-    torch.cuda.current_stream(dev).wait_stream(side)
-    sync_all()
+    # ---------------------------------------------------------------- CUDA graphs
+    # One GPU: the whole step (7 projections) is one graph.  N GPUs: one graph per projection,
+    # and after each replay its dW is all-reduced asynchronously (NCCL stays outside the
+    # graphs) while the next projection's graph runs.
+    launches_before = bl.launch_count()
+    if world == 1:
+        g_all = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_all):
+            for L in layers:
+                layer_step(L)
+        graphs = [g_all]
 
-    def capture(ev, dom_ev=None):
-        if world == 1:
+        def replay():
+            g_all.replay()
+    else:
+        graphs = []
+        for L in layers:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                if ev is None:
-                    step_overlap(dom_ev)
-                else:
-                    step(ev)
-            return [g], (lambda: g.replay())
-        # the NCCL all-reduce stays outside the graphs
-        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
-        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        b = bufs
-        if ev is None:
-            with torch.cuda.graph(g1):
-                step_overlap(dom_ev, with_tail=False)
-            with torch.cuda.graph(g2):
-                bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B],
-                                y=b["ydec"])
+                layer_step(L)
+            graphs.append(g)
 
-            def rp0():
-                g1.replay()
-                dp.allreduce_weight_grad(bufs["dW"])
-                g2.replay()
-            return [g1, g2], rp0
-        with torch.cuda.graph(g1):
-            rec(0)
-            bl.bitlinear_quant_weight(W, ws=b["ws"], out=b); rec(1)
-            bl.bitlinear_act_quant(X, apply_rmsnorm=True, out=b); rec(2)
-            bl.bitlinear_linear(b["xq"], b["sx"], b["wq_i8"], b["gamma"], y=b["y"]); rec(3)
-            bl.bitlinear_grad_input(dY, b["wq_bf16"], b["gamma"], dXhat=b["dX"]); rec(4)
-            bl.bitlinear_rmsnorm_backward(X, b["rinv"], b["dX"], ws=b["ws"], dg=b["dg"]); rec(5)
-            bl.bitlinear_backward_weight(dY, b["xdq"], dW=b["dW"]); rec(6)
-        with torch.cuda.graph(g2):
-            rec(7)
-            bl.ternary_gemv(b["packed"], b["gamma"], D_IN, b["xq"][:DECODE_B], b["sx"][:DECODE_B], y=b["ydec"])
-            rec(8)
-
-        def rp():
-            g1.replay()
-            dp.allreduce_weight_grad(bufs["dW"])
-            g2.replay()
-        return [g1, g2], rp
-
-    dom_ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-    launches_before_capture = bl.launch_count()
-    graphs, replay = capture(None)                 # the timed step: kernels only
-    kernels_per_step = bl.launch_count() - launches_before_capture
-    graphs_dom, replay_dom = capture(None, dom_ev)  # the same step, events around the grad-input GEMM
-    graphs_pc, replay_pc = capture(gev)            # sequential, events between all calls
+        def replay():
+            works = []
+            for g, L in zip(graphs, layers):
+                g.replay()
+                works.append(dist.all_reduce(L["dW"], op=dist.ReduceOp.SUM, async_op=True))
+            for w in works:
+                w.wait()
+    kernels_per_step = bl.launch_count() - launches_before
+    # sequential pieces with events between the calls (piece times; not part of the value)
+    pev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(8)] for _ in layers]
+    g_pc = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_pc):
+        for L, ev in zip(layers, pev):
+            layer_pieces(L, ev)
+        pev[-1][7].record()
     for _ in range(max(3, args.warmup)):
         replay()
-        replay_dom()
-        replay_pc()
+        g_pc.replay()
     sync_all()
     assert bl.check_device_status() == 0
 
@@ -434,12 +500,7 @@ def main():
     K = args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    gpu_uuid = None
-    try:
-        gpu_uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        gpu_uuid = str(local)
-    clk = ClockSampler(gpu_uuid) if rank == 0 else None
+    clk = ClockSampler(gpu_id_of(torch, dev)) if rank == 0 else None
     sync_all()
     if clk:
         clk.start()
@@ -450,91 +511,88 @@ def main():
         replay()
         ev_e[i].record()
     sync_all()
-    # roofline: K more timed steps of the same work with two event nodes around the
-    # grad-input GEMM (event nodes cost the step its launch overlap at that point, so they
-    # stay out of the steps that give the value)
-    dom_ms = []
-    for i in range(K):
-        flush.zero_()
-        replay_dom()
-        torch.cuda.synchronize()
-        dom_ms.append(dom_ev[0].elapsed_time(dom_ev[1]))
-    sync_all()
     clocks = clk.stop() if clk else None
-    launches = kernels_per_step * K
     per_step = [a.elapsed_time(b) for a, b in zip(ev_s, ev_e)]
-    tot_ms = sum(per_step)
-    t = torch.tensor([tot_ms], dtype=torch.float64, device=dev)
+    t = torch.tensor([sum(per_step)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     tot_ms = float(t.item())
-    # piece breakdown (same step with event nodes between the calls; not part of the value)
-    pieces = {p: [] for p in PIECES}
+
+    # ---------------------------------------------------------------- piece times
+    pieces = {p: [[] for _ in layers] for p in PIECES}
     for i in range(K):
         flush.zero_()
-        replay_pc()
+        g_pc.replay()
         torch.cuda.synchronize()
-        for j, p in enumerate(PIECES):
-            pieces[p].append(gev[j].elapsed_time(gev[j + 1]))
+        for li, ev in enumerate(pev):
+            nxt = pev[li + 1][0] if li + 1 < len(pev) else pev[-1][7]
+            for j, p in enumerate(PIECES):
+                end = ev[j + 1] if j + 1 < 7 else nxt
+                pieces[p][li].append(ev[j].elapsed_time(end))
     sync_all()
-    piece_ms = {p: statistics.mean(v) for p, v in pieces.items()}
-    # the grad-input GEMM back to back (20 launches per graph, one event pair): its duration
-    # without an event node's lost launch overlap, reported beside the roofline
-    g_b2b = torch.cuda.CUDAGraph()
+    piece_ms = {p: [statistics.mean(v) for v in per_layer] for p, per_layer in pieces.items()}
+
+    # ---------------------------------------------------------------- dominant kernel, live in the step
+    ops_gemm = [2.0 * T * L["N"] * L["K"] for L in layers]
+    dom = max(("grad_input", "grad_weight"), key=lambda p: sum(piece_ms[p]))
+    dev_ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+              for _ in layers]
+    g_dom = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(side):
-        bl.bitlinear_grad_input(dY, bufs["wq_bf16"], bufs["gamma"], dXhat=bufs["dX"])
-    torch.cuda.current_stream(dev).wait_stream(side)
-    with torch.cuda.graph(g_b2b):
-        for _ in range(20):
-            bl.bitlinear_grad_input(dY, bufs["wq_bf16"], bufs["gamma"], dXhat=bufs["dX"])
-    g_b2b.replay()
-    b2b = []
-    for i in range(5):
+    with torch.cuda.graph(g_dom):
+        for L, (e0, e1) in zip(layers, dev_ev):
+            layer_step(L, dom=(dom, e0, e1))
+    g_dom.replay()
+    torch.cuda.synchronize()
+    dom_ms = [[] for _ in layers]
+    for i in range(K):
         flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g_b2b.replay()
-        e1.record()
+        g_dom.replay()
         torch.cuda.synchronize()
-        b2b.append(e0.elapsed_time(e1) / 20)
-    b2b_ms = statistics.median(b2b)
+        for li, (e0, e1) in enumerate(dev_ev):
+            dom_ms[li].append(e0.elapsed_time(e1))
+    dom_layer_ms = [statistics.mean(v) for v in dom_ms]
     assert bl.check_device_status() == 0
-    del graphs, graphs_dom, graphs_pc, g_b2b
+    del graphs, g_pc, g_dom
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
     if not args.no_e2e:
-        W_p, X_p, dY_p = W_h.pin_memory(), X_h.pin_memory(), dY_h.pin_memory()
-        W_d, X_d, dY_d = torch.empty_like(W), torch.empty_like(X), torch.empty_like(dY)
-        dW_p = torch.empty(D_OUT, D_IN, dtype=f32).pin_memory()
-        g_p = torch.empty(1, dtype=f32).pin_memory()
-        h2d = W_p.numel() * 4 + X_p.numel() * 2 + dY_p.numel() * 2
-        d2h = dW_p.numel() * 4 + 4
-        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-        for i in range(2):
-            W_d.copy_(W_p, non_blocking=True); X_d.copy_(X_p, non_blocking=True); dY_d.copy_(dY_p, non_blocking=True)
-            step_overlap(inputs=(W_d, X_d, dY_d))
-            dW_p.copy_(bufs["dW"], non_blocking=True); g_p.copy_(bufs["gamma"], non_blocking=True)
+        host = [dict(W=li.W.pin_memory(), X=li.X.pin_memory(), dY=li.dY.pin_memory()) for li in lis]
+        dW_h = [torch.empty(L["N"], L["K"], dtype=f32).pin_memory() for L in layers]
+        g_h = torch.empty(len(layers), dtype=f32).pin_memory()
+        h2d = sum(h["W"].numel() * 4 + h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host)
+        d2h = sum(d.numel() * 4 for d in dW_h) + 4 * len(layers)
+
+        def e2e_step():
+            for li, (L, h) in enumerate(zip(layers, host)):
+                L["W"].copy_(h["W"], non_blocking=True)
+                L["X"].copy_(h["X"], non_blocking=True)
+                L["dY"].copy_(h["dY"], non_blocking=True)
+                layer_step(L)
+                g_h[li:li + 1].copy_(L["fo"]["gamma"], non_blocking=True)
+                dp.allreduce_weight_grad(L["dW"])
+                dW_h[li].copy_(L["dW"], non_blocking=True)
+
+        e2e_step()
         sync_all()
-        for i in range(K):
+        ke = max(1, min(K, 10))
+        es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ke)]
+        for i in range(ke):
             flush.zero_()
             es[i][0].record()
-            W_d.copy_(W_p, non_blocking=True); X_d.copy_(X_p, non_blocking=True); dY_d.copy_(dY_p, non_blocking=True)
-            step_overlap(inputs=(W_d, X_d, dY_d))
-            dW_p.copy_(bufs["dW"], non_blocking=True); g_p.copy_(bufs["gamma"], non_blocking=True)
+            e2e_step()
             es[i][1].record()
         sync_all()
         e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in es)], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": T_TOK * world * K / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
-
-    # ---------------------------------------------------------------- decode GEMV (28672 x 8192)
-    gemv = None
-    if not args.no_gemv and rank == 0:
-        gemv = gemv_measure(bl, torch, dev, flush, peaks())
+        e2e = {"value": T * world * ke / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ke,
+               "how": "per projection: pinned host -> device copies of W, X, dY, the eager library calls of the "
+                      "step, device -> host copies of dW and gamma; CUDA events around each step"}
+        del host, dW_h
 
     if world > 1:
         dist.barrier()
@@ -544,56 +602,206 @@ def main():
         return
 
     # ---------------------------------------------------------------- roofline of the dominant kernel
-    pk = peaks()
-    gemm_flops = 2.0 * T_TOK * D_OUT * D_IN
-    gemm_pieces = {"linear_i8": "int8", "grad_input": "bf16", "grad_weight": "bf16"}
-    # the grad-input GEMM, timed by the two event nodes around it inside the timed graph
-    dom = "grad_input"
-    dom_ms = statistics.mean(dom_ms)
-    achieved = gemm_flops / (dom_ms * 1e-3) / 1e12
-    if gemm_pieces[dom] == "bf16":
-        peak, peak_note = pk["bf16_sust"], f"bf16 sustained ({pk['src']})"
-    else:
-        peak, peak_note = 2.0 * pk["bf16_sust"], f"int8 = 2 x bf16 sustained ({pk['src']}; nominal 4.5/2.25 ratio)"
+    bf16_peak = pk["bf16"]
+    int8_peak = tpk["int8"]
+    dom_ms_tot = sum(dom_layer_ms)
+    achieved = sum(ops_gemm) / (dom_ms_tot * 1e-3) / 1e12
     kernel_names = {"linear_i8": "tc_gemm2_kernel<int8,K,K,linear> (2-SM, 256x256)",
                     "grad_input": "tc_gemm2_kernel<bf16,K,MN,scale_f32> (2-SM, 256x256)",
                     "grad_weight": "tc_gemm2_kernel<bf16,MN,MN,f32> (2-SM, 256x256)"}
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": ncu_traffic(dom), "kernel": kernel_names[dom], "peak_kind": peak_note,
-                "launch_ms": dom_ms,
-                "back_to_back": {"launch_ms": b2b_ms, "achieved": gemm_flops / (b2b_ms * 1e-3) / 1e12,
-                                 "frac": gemm_flops / (b2b_ms * 1e-3) / 1e12 / peak,
-                                 "how": "20 launches of the GEMM in one CUDA graph, one event pair, median of 5"}}
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak, "traffic": ncu_traffic(dom), "kernel": kernel_names[dom],
+                "peak_kind": f"bf16 dense, cuBLAS burst ({pk['src']})",
+                "launch_ms": dom_ms_tot / len(layers), "launches_per_step": len(layers),
+                "flop_per_launch": sum(ops_gemm) / len(layers),
+                "per_layer_ms": {L["name"]: round(v, 5) for L, v in zip(layers, dom_layer_ms)},
+                "frac_of_probe_bf16": achieved / tpk["bf16"],
+                "how": "two event nodes around this GEMM of every projection inside K further replays of the "
+                       "timed step's graph (L2 flushed before each); achieved = its FLOPs / its time, summed "
+                       "over the projections"}
+
+    # every kernel of the step against its roofline (sequential piece times)
+    def bytes_of(p, L):
+        N, K = L["N"], L["K"]
+        if p == "act_quant":
+            return T * K * 2 + T * K + T * K * 2 + 8 * T
+        if p == "quant_weight":
+            return N * K * 4 + N * K + N * K * 2 + N * K // 4
+        if p == "rmsnorm_bwd":
+            return T * K * 4 + T * K * 2 + T * K * 4 + 4 * T
+        if p == "decode_gemv":
+            return N * K // 4 + DECODE_B * K + 4 * DECODE_B * N + 4 * DECODE_B
+        return None
+    kernels = {}
+    for p in PIECES:
+        ms = sum(piece_ms[p])
+        rec = {"ms_per_step": ms, "share_of_pieces": ms / sum(sum(v) for v in piece_ms.values())}
+        if p in ("linear_i8", "grad_input", "grad_weight"):
+            rate = sum(ops_gemm) / (ms * 1e-3) / 1e12
+            pkv = int8_peak if p == "linear_i8" else bf16_peak
+            rec.update({"achieved": rate, "unit": "TOPS" if p == "linear_i8" else "TFLOP/s", "peak": pkv,
+                        "frac": rate / pkv,
+                        "peak_kind": "int8 measured (own tcgen05 kind::i8 loop)" if p == "linear_i8"
+                        else f"bf16 dense, cuBLAS burst ({pk['src']})"})
+        else:
+            nb = sum(bytes_of(p, L) for L in layers)
+            rate = nb / (ms * 1e-3) / 1e9
+            rec.update({"achieved": rate, "unit": "GB/s", "peak": pk["hbm"], "frac": rate / pk["hbm"],
+                        "bytes_per_step": nb})
+        rec["per_layer_ms"] = {L["name"]: round(v, 5) for L, v in zip(layers, piece_ms[p])}
+        kernels[p] = rec
+
+    sub = None
+    if not args.no_sub:
+        sub = {"decode_gemv": gemv_measure(bl, torch, dev, flush, pk),
+               "configs": configs_measure(bl, torch, dev, flush)}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu = cpu_baseline()
 
-    value = T_TOK * world * K / (tot_ms * 1e-3)
+    value = T * world * K / (tot_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": tot_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "s8+bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens_per_gpu": T_TOK, "d_in": D_IN, "d_out": D_OUT,
+        "config": {"workload": WORKLOAD, "tokens_per_gpu": T,
+                   "layers": {L["name"]: f"{L['K']}->{L['N']}" for L in layers},
                    "decode_batch": DECODE_B, "parallelism": f"dp{world}",
-                   "l2": "flushed before every timed step (512 MB write)"},
+                   "l2": "flushed before every timed step (512 MB write); every projection's inputs exceed L2"},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": int(launches),
-        "timing": ("each step replays a CUDA graph of the step's library calls (RMSNorm backward and decode "
-                   "GEMV on a second stream beside the weight-gradient GEMM) with no event node inside; the "
-                   "roofline's grad-input GEMM time comes from K further timed steps of the same graph with "
-                   "two event nodes around that GEMM, and pieces_ms from a sequential graph with events "
-                   "between all calls; gpu_launches = kernels per step x steps"),
+        "gpu_launches": int(kernels_per_step * K),
+        "timing": ("each step replays CUDA graph(s) of the step's library calls (per projection: forward_qat, "
+                   "grad-input GEMM, then RMSNorm backward and decode GEMV on a second stream beside the "
+                   "weight-gradient GEMM) with no event node inside; the roofline's GEMM times come from K "
+                   "further replays with event nodes around that GEMM, and `kernels` from a sequential graph "
+                   "with events between all calls; gpu_launches = kernels per step x steps"),
         "clocks": clocks,
-        "pieces_ms": {k: round(v, 5) for k, v in piece_ms.items()},
-        "gemm_tflops": {p: gemm_flops / (piece_ms[p] * 1e-3) / 1e12 for p in gemm_pieces},
-        "decode_gemv": gemv,
+        "tensor_peaks": tpk,
+        "kernels": kernels,
+        "sub": sub,
     }
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def configs_measure(bl, torch, dev, flush, steps: int = 5):
+    """The other training configurations' full steps (single, square, mlp7b): per layer weight
+    quantisation, activation quantisation, forward GEMM, grad-input GEMM, RMSNorm backward,
+    weight-gradient GEMM, all in one CUDA graph; L2 flushed before each replay; median of
+    `steps`."""
+    from bit_ternary_qat_b200 import synth
+    out = {}
+    for name in ("single", "square", "mlp7b"):
+        ms, T, layers = step_graph_ms(bl, torch, dev, flush, name, steps)
+        out[name] = {"ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3), "layers": layers,
+                     "dtype": synth.WORKLOADS[name].dtype}
+    return out
+
+
+def step_graph_ms(bl, torch, dev, flush, name, steps):
+    from bit_ternary_qat_b200 import synth
+    wl = synth.WORKLOADS[name]
+    lis = synth.workload_inputs(name)
+    T = lis[0].X.shape[0]
+    dt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+    maxK = max(li.X.shape[1] for li in lis)
+    maxN = max(li.W.shape[0] for li in lis)
+    ws = bl.workspace(T, maxN, maxK, dev)
+    dev_layers = []
+    for li in lis:
+        N, K = li.W.shape
+        dev_layers.append(dict(
+            W=li.W.to(dev), X=li.X.to(dev), dY=li.dY.to(dev), N=N, K=K,
+            q=dict(gamma=torch.empty(1, dtype=torch.float32, device=dev),
+                   wq_i8=torch.empty(N, K, dtype=torch.int8, device=dev),
+                   wq_bf16=torch.empty(N, K, dtype=torch.bfloat16, device=dev),
+                   packed=torch.empty(N, K // 4, dtype=torch.uint8, device=dev))))
+    shared = dict(xq=torch.empty(T * maxK, dtype=torch.int8, device=dev),
+                  xdq=torch.empty(T * maxK, dtype=dt, device=dev),
+                  sx=torch.empty(T, dtype=torch.float32, device=dev),
+                  rinv=torch.empty(T, dtype=torch.float32, device=dev),
+                  y=torch.empty(T * maxN, dtype=dt, device=dev),
+                  dX=torch.empty(T * maxK, dtype=torch.float32, device=dev),
+                  dW=torch.empty(maxN * maxK, dtype=torch.float32, device=dev),
+                  dg=torch.empty(maxK, dtype=torch.float32, device=dev))
+
+    def step():
+        for L in dev_layers:
+            N, K = L["N"], L["K"]
+            a = dict(xq=shared["xq"][:T * K].view(T, K), xdq=shared["xdq"][:T * K].view(T, K),
+                     sx=shared["sx"], rinv=shared["rinv"])
+            bl.bitlinear_quant_weight(L["W"], ws=ws, out=L["q"])
+            bl.bitlinear_act_quant(L["X"], apply_rmsnorm=True, out=a)
+            bl.bitlinear_linear(a["xq"], a["sx"], L["q"]["wq_i8"], L["q"]["gamma"],
+                                out_dtype=dt, y=shared["y"][:T * N].view(T, N))
+            dX = shared["dX"][:T * K].view(T, K)
+            bl.bitlinear_grad_input(L["dY"], L["q"]["wq_bf16"], L["q"]["gamma"], dXhat=dX)
+            bl.bitlinear_rmsnorm_backward(L["X"], a["rinv"], dX, ws=ws, dg=shared["dg"][:K])
+            bl.bitlinear_backward_weight(L["dY"], a["xdq"], dW=shared["dW"][:N * K].view(N, K))
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush.zero_()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record()
+        graph.replay()
+        b_ev.record()
+        torch.cuda.synchronize()
+        ms.append(a_ev.elapsed_time(b_ev))
+    del graph
+    assert bl.check_device_status() == 0
+    layers = [f"{L['K']}->{L['N']}" for L in dev_layers]
+    del dev_layers, shared, ws
+    torch.cuda.empty_cache()
+    return statistics.median(ms), T, layers
+
+
+def gemm_once(bl, torch, dev, which: str):
+    """Three launches of one GEMM of the step on the gate projection's shape (16384 tokens,
+    4096 -> 11008): a small case for a profiler capture (about 1 GB on the device)."""
+    T, K, N = 16384, 4096, 11008
+    g = torch.Generator(device=dev).manual_seed(1)
+    gamma = torch.full((1,), 0.02, device=dev)
+    if which == "linear_i8":
+        xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev, generator=g)
+        wq = torch.randint(-1, 2, (N, K), dtype=torch.int8, device=dev, generator=g)
+        sx = torch.full((T,), 50.0, device=dev)
+        y = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+        call = lambda: bl.bitlinear_linear(xq, sx, wq, gamma, y=y)  # noqa: E731
+    elif which == "grad_input":
+        dY = (torch.randn(T, N, device=dev, generator=g) * 1e-2).to(torch.bfloat16)
+        wq = torch.randint(-1, 2, (N, K), device=dev, generator=g).to(torch.bfloat16)
+        dX = torch.empty(T, K, dtype=torch.float32, device=dev)
+        call = lambda: bl.bitlinear_grad_input(dY, wq, gamma, dXhat=dX)  # noqa: E731
+    else:
+        dY = (torch.randn(T, N, device=dev, generator=g) * 1e-2).to(torch.bfloat16)
+        xdq = (torch.randn(T, K, device=dev, generator=g)).to(torch.bfloat16)
+        dW = torch.empty(N, K, dtype=torch.float32, device=dev)
+        call = lambda: bl.bitlinear_backward_weight(dY, xdq, dW=dW)  # noqa: E731
+    ms = 0.0
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+    assert bl.check_device_status() == 0
+    return {"which": which, "shape": f"T={T} K={K} N={N}", "ms_last": ms,
+            "tflops_last": 2.0 * T * N * K / (ms * 1e-3) / 1e12}
 
 
 def gemv_measure(bl, torch, dev, flush, pk):
@@ -920,8 +1128,7 @@ def table_measure(bl, torch, dev, flush, pk, steps: int = 5):
         t_s = min(T, 64 if T <= 4096 else 16)
         cpu_s = 0.0
         for li in lis:
-            full = oracle_step(ora, li, t_s)
-            wq_only = oracle_weight_quant_s(ora, li)
+            full, wq_only = oracle_step(ora, li, t_s)
             cpu_s += wq_only + (full - wq_only) * (T / t_s)
         out[name] = {"tokens": T, "layers": [f"{L['K']}->{L['N']}" for L in dev_layers], "dtype": wl.dtype,
                      "ms_per_step": t, "tokens_per_s": T / (t * 1e-3),
@@ -944,14 +1151,6 @@ def table_measure(bl, torch, dev, flush, pk, steps: int = 5):
     out["decode"]["oracle_B1"] = {"us": dt_s * 1e6, "GB/s": (28672 * 8192 // 4) / dt_s / 1e9,
                                   "cores": ora.num_threads()}
     return out
-
-
-def oracle_weight_quant_s(ora, li) -> float:
-    W = li.W.numpy()
-    t0 = time.perf_counter()
-    gamma, wq = ora.quant_weight(W)
-    ora.pack(wq)
-    return time.perf_counter() - t0
 
 
 if __name__ == "__main__":

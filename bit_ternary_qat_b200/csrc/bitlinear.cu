@@ -24,6 +24,7 @@
 #include "gemv.cuh"
 #include "optim.cuh"
 #include "gemm_packed.cuh"
+#include "mma_peak.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -1117,6 +1118,43 @@ bl_status bitlinear_optimizer_step(float* W, const float* dW, float* m, float* v
     if (gamma == nullptr) return BL_OK;
     // the next step's codes from the |W_new| partials written above (the quantiser's pass 2)
     return run_ternary(W, n, wpart, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev);
+}
+
+bl_status bl_mma_peak_probe(int kind, int pair, int iters, double* ops_out, void* stream) {
+    BL_REQUIRE(kind == 0 || kind == 1, BL_ERR_INVALID_ARG, "kind must be 0 (int8) or 1 (bf16), got %d", kind);
+    BL_REQUIRE(pair == 0 || pair == 1, BL_ERR_INVALID_ARG, "pair must be 0 or 1, got %d", pair);
+    BL_REQUIRE(iters >= 1 && iters <= (1 << 20), BL_ERR_INVALID_ARG, "iters must be in [1, 2^20], got %d", iters);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    BL_REQUIRE(bl::kPeakSmemBytes <= dev.max_smem_optin, BL_ERR_DEVICE, "probe needs %d bytes of shared memory",
+               bl::kPeakSmemBytes);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint64_t wait_ns = g_wait_ns.load();
+    int ctas = pair ? 2 * (dev.sms / 2) : dev.sms;
+    void (*kern)(int, uint64_t) = nullptr;
+    if (pair) kern = kind == 0 ? bl::mma_peak2_kernel<true> : bl::mma_peak2_kernel<false>;
+    else kern = kind == 0 ? bl::mma_peak_kernel<true> : bl::mma_peak_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bl::kPeakSmemBytes);
+    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (pair) {
+        // no more clusters than can be resident at once: every pair runs in the same wave
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)ctas);
+        cfg.blockDim = dim3(bl::kPeakThreads);
+        cfg.dynamicSmemBytes = bl::kPeakSmemBytes;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s", cudaGetErrorString(e));
+        if (n < 1) return fail(BL_ERR_DEVICE, "no 2-CTA cluster of the probe fits on the device");
+        ctas = std::min(ctas, 2 * n);
+    }
+    // multiply-adds x 2 of the launch: per instruction M x N x (32 bytes of K)
+    const double k_per_instr = kind == 0 ? 32.0 : 16.0;
+    const double per_instr = 2.0 * (pair ? 256.0 * 256.0 : 128.0 * 256.0) * k_per_instr;
+    const double units = pair ? ctas / 2 : ctas;
+    if (ops_out) *ops_out = units * 4.0 * (double)iters * per_instr;
+    pdl_launch(kern, dim3((unsigned)ctas), dim3(bl::kPeakThreads), (size_t)bl::kPeakSmemBytes, st, iters, wait_ns);
+    return launched("mma_peak");
 }
 
 bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

@@ -455,3 +455,15 @@ def launch_count() -> int:
 def selftest_bounded_wait(limit_ns: int, device=None) -> None:
     dev = device if device is not None else torch.cuda.current_device()
     _lib.call("bl_selftest_bounded_wait", int(limit_ns), _stream(dev))
+
+
+def mma_peak_probe(kind: str = "int8", pair: bool = True, iters: int = 20000, device=None) -> float:
+    """Launch the tensor-pipe peak probe on the current stream (tcgen05.mma from fixed
+    shared-memory operands, no global traffic).  Returns 2 x the multiply-adds of the
+    launch; time the launch with CUDA events for the rate."""
+    import ctypes
+    dev = device if device is not None else torch.cuda.current_device()
+    ops = ctypes.c_double(0.0)
+    _lib.call("bl_mma_peak_probe", {"int8": 0, "bf16": 1}[kind], 1 if pair else 0, int(iters),
+              ctypes.byref(ops), _stream(dev))
+    return float(ops.value)

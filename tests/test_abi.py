@@ -179,3 +179,9 @@ def test_status_values_match_header():
     assert vals == {"BL_OK": 0, "BL_ERR_INVALID_ARG": 1, "BL_ERR_UNSUPPORTED_SHAPE": 2, "BL_ERR_MISALIGNED": 3,
                     "BL_ERR_WORKSPACE": 4, "BL_ERR_CUDA": 5, "BL_ERR_TIMEOUT": 6, "BL_ERR_DEVICE": 7}
     assert {v: k for k, v in vals.items()} == _lib.STATUS_NAMES
+
+
+@pytest.mark.parametrize("kind,pair,iters", [(2, 0, 10), (0, 2, 10), (0, 0, 0), (1, 1, (1 << 20) + 1)])
+def test_peak_probe_validation(L, kind, pair, iters):
+    assert _lib.status("bl_mma_peak_probe", kind, pair, iters, None, None) == 1
+    assert len(_lib.last_error()) > 0

@@ -194,8 +194,24 @@ def _layer_case(bl, li, eps=1e-6):
     return dt, g_gpu, wq, f, dX, dW, dg
 
 
+def test_single_workload_seed0(bl):
+    """The single-layer fp32 workload exactly as specified (X 64x256, W 512x256, dY 64x512,
+    seed 0, gain 1): every code, accumulator and output exact, gradients within 1e-4."""
+    li = synth.workload_inputs("single")[0]
+    assert li.X.dtype == torch.float32 and tuple(li.X.shape) == (64, 256) and tuple(li.W.shape) == (512, 256)
+    dt, g_gpu, wq, f, dX, dW, dg = _layer_case(bl, li)
+    r_gpu = np_(f["rinv"])
+    assert ulp_diff(r_gpu, oracle.rmsnorm_rinv(li.X, 1e-6)).max() <= 1
+    ref = oracle.forward(li.X, li.W, rinv=r_gpu, gamma=g_gpu, out_dtype="f32")
+    for k_gpu, k_ref in (("xq", "xq"), ("sx", "s"), ("acc", "acc"), ("y", "y"), ("xdq", "xdq")):
+        assert np.array_equal(np_(f[k_gpu]), ref[k_ref]), k_gpu
+    dX_o, dW_o, dg_o, _ = oracle.backward(li.X, li.dY, ref)
+    for name, a, b in (("dX", dX, dX_o), ("dW", dW, dW_o), ("dg", dg, dg_o)):
+        assert max_rel_err(np_(a), b) <= TOL["f32"], name
+
+
 @pytest.mark.parametrize("T,K,N,dtype,gain", [
-    (64, 256, 512, "f32", False),        # the single-layer fp32 workload
+    (64, 256, 512, "f32", False),        # the single-layer fp32 shape on another seed
     (300, 160, 400, "bf16", True),
     (257, 512, 144, "f32", True),
     (130, 1024, 784, "bf16", False),
@@ -250,14 +266,28 @@ def test_forward_qat_matches_separate_calls(bl, T, K, N, dtype, gain):
     assert np.array_equal(np_(fq["acc"]), ref["acc"])
 
 
-@pytest.mark.parametrize("workload,layer", [("square", 0), ("mlp7b", 0), ("mlp7b", 1), ("layer7b", 0)])
+_WORKLOAD_CACHE = {}
+
+
+def _workload_layer(workload, layer):
+    """One layer's inputs; a workload's draws are made once per test session (they are
+    sequential, so layer i needs every earlier layer's draws)."""
+    if workload not in _WORKLOAD_CACHE:
+        _WORKLOAD_CACHE.clear()
+        _WORKLOAD_CACHE[workload] = synth.workload_inputs(workload)
+    return _WORKLOAD_CACHE[workload][layer]
+
+
+@pytest.mark.parametrize("workload,layer", [("square", 0), ("mlp7b", 0), ("mlp7b", 1)] +
+                         [("layer7b", i) for i in range(7)])
 def test_workload_full_size(bl, workload, layer):
     """Full-size layers of the benchmark workloads (square 2048->2048 x 4096 tokens; the
-    7B MLP's 4096->11008 and 11008->4096 x 8192 tokens with Student-t weights; the 7B
-    layer's 4096->4096 x 16384 tokens), bf16: every code exact, sampled rows of the
+    7B MLP's 4096->11008 and 11008->4096 x 8192 tokens with Student-t weights; all seven
+    projections of the 7B layer at 16384 tokens: q, k, v, o 4096->4096, gate and up
+    4096->11008, down 11008->4096), bf16: every code exact, sampled rows of the
     accumulators / outputs / gradients against the oracle, the rest through exact
     properties."""
-    li = synth.workload_inputs(workload, first=layer + 1)[layer]
+    li = _workload_layer(workload, layer)
     dt, g_gpu, wq, f, dX, dW, dg = _layer_case(bl, li)
     T, K = li.X.shape
     r_gpu = np_(f["rinv"])
