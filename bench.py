@@ -290,11 +290,24 @@ def probe_tensor_peaks(bl, torch, dev, iters: int = 20000, reps: int = 5):
                 torch.cuda.synchronize()
                 rates.append(ops / (a.elapsed_time(b) * 1e-3) / 1e12)
             out[f"{kind}_{'cta_pair' if pair else 'cta'}"] = max(rates)
+    # the warp-level IMMA of the decode GEMV (mma.sync m16n8k32 int8)
+    bl.mma_peak_probe("imma_sync", False, max(1, iters // 8))
+    torch.cuda.synchronize()
+    rates = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ops = bl.mma_peak_probe("imma_sync", False, iters // 2)
+        b.record()
+        torch.cuda.synchronize()
+        rates.append(ops / (a.elapsed_time(b) * 1e-3) / 1e12)
+    out["imma_sync"] = max(rates)
     assert bl.check_device_status() == 0
     out["int8"] = max(out["int8_cta"], out["int8_cta_pair"])
     out["bf16"] = max(out["bf16_cta"], out["bf16_cta_pair"])
     out["how"] = (f"tcgen05.mma loop from fixed pseudo-random shared-memory operands into TMEM, no global "
-                  f"traffic; {iters} x 4 instructions per CTA (or pair) per launch, best of {reps} launches")
+                  f"traffic; {iters} x 4 instructions per CTA (or pair) per launch, best of {reps} launches; "
+                  f"imma_sync: mma.sync m16n8k32 u8 x s8 from registers, 16 warps x 8 chains per SM")
     return out
 
 
@@ -653,7 +666,7 @@ def main():
 
     sub = None
     if not args.no_sub:
-        sub = {"decode_gemv": gemv_measure(bl, torch, dev, flush, pk),
+        sub = {"decode_gemv": gemv_measure(bl, torch, dev, flush, pk, imma_peak=tpk["imma_sync"]),
                "configs": configs_measure(bl, torch, dev, flush)}
 
     cpu = None
@@ -804,7 +817,7 @@ def gemm_once(bl, torch, dev, which: str):
             "tflops_last": 2.0 * T * N * K / (ms * 1e-3) / 1e12}
 
 
-def gemv_measure(bl, torch, dev, flush, pk):
+def gemv_measure(bl, torch, dev, flush, pk, imma_peak=None):
     """Decode GEMV on the 28672 x 8192 packed weight at batch 1, 4, 16.
 
     Four copies of the packed weight (235 MB, above the 126 MB L2) are cycled, so every launch
@@ -848,9 +861,16 @@ def gemv_measure(bl, torch, dev, flush, pk):
         ms = statistics.median(samples)
         nbytes = N * K // 4 + B * K + 4 * B + 4 * B * N + 4
         gbs = nbytes / (ms * 1e-3) / 1e9
-        out[f"B{B}"] = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / pk["hbm"],
-                        "int_ops_T": 2.0 * B * N * K / (ms * 1e-3) / 1e12}
+        rec = {"us": ms * 1e3, "GB/s": gbs, "frac_hbm": gbs / pk["hbm"],
+               "int_ops_T": 2.0 * B * N * K / (ms * 1e-3) / 1e12}
+        if imma_peak:
+            # the MMAs run 8 batch columns per n-tile (one n-tile up to B = 8, two beyond)
+            mma_ops = 2.0 * (8 if B <= 8 else 16) * N * K
+            rec["imma_bound_us"] = mma_ops / (imma_peak * 1e12) * 1e6
+            rec["frac_imma"] = rec["imma_bound_us"] / rec["us"]
+        out[f"B{B}"] = rec
     out["hbm_peak_GBs"] = pk["hbm"]
+    out["imma_peak_T"] = imma_peak
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
                        "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5")
     return out

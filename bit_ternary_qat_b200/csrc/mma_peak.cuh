@@ -12,6 +12,7 @@
 // signs), so the datapath toggles as it does on real data.  The final wait is bounded.
 #pragma once
 #include "common.cuh"
+#include "gemv.cuh"
 
 namespace bl {
 
@@ -155,6 +156,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPeakThreads, 1) mma
         tc_fence_after();
         tmem_dealloc_pair(tmem, 256);
     }
+}
+
+// The warp-level integer MMA the decode GEMV uses (mma.sync m16n8k32, u8 x s8 -> s32) from
+// register operands: 16 warps per SM, each with 8 independent accumulator chains, so the
+// rate is the IMMA pipe's throughput rather than one chain's latency.
+constexpr int kImmaWarps = 16;
+constexpr int kImmaChains = 8;
+__global__ void __launch_bounds__(kImmaWarps * 32, 1) imma_sync_peak_kernel(int iters) {
+    pdl_trigger_and_wait();
+    const uint32_t h = peak_hash(blockIdx.x * 1024u + threadIdx.x);
+    const uint32_t a[4] = {h & 0x3F3F3F3Fu, (h >> 3) & 0x3F3F3F3Fu, (h >> 5) & 0x3F3F3F3Fu, (h >> 7) & 0x3F3F3F3Fu};
+    const uint32_t b0 = peak_hash(h), b1 = peak_hash(h + 1u);
+    int d[kImmaChains][4] = {};
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int c = 0; c < kImmaChains; ++c) mma_u8s8_16832(d[c], a, b0, b1);
+    }
+    int acc = 0;
+#pragma unroll
+    for (int c = 0; c < kImmaChains; ++c) acc += d[c][0] + d[c][1] + d[c][2] + d[c][3];
+    if (acc == 0x7fffffff) record_status(0);   // keeps the chains live; never true in practice
 }
 
 }  // namespace bl

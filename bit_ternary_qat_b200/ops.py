@@ -464,6 +464,6 @@ def mma_peak_probe(kind: str = "int8", pair: bool = True, iters: int = 20000, de
     import ctypes
     dev = device if device is not None else torch.cuda.current_device()
     ops = ctypes.c_double(0.0)
-    _lib.call("bl_mma_peak_probe", {"int8": 0, "bf16": 1}[kind], 1 if pair else 0, int(iters),
+    _lib.call("bl_mma_peak_probe", {"int8": 0, "bf16": 1, "imma_sync": 2}[kind], 1 if pair else 0, int(iters),
               ctypes.byref(ops), _stream(dev))
     return float(ops.value)

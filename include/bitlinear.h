@@ -354,8 +354,9 @@ BL_API bl_status bitlinear_optimizer_step(float* W, const float* dW, float* m, f
  * traffic, so the achieved rate is the tensor pipe's ceiling for the GEMMs' instruction
  * shapes.  kind 0 = kind::i8 (s8 x s8 -> s32, 32 values of K per instruction), 1 = kind::f16
  * (bf16 x bf16 -> f32, 16 values).  pair 0 = cta_group::1, M = 128 x N = 256 on every SM;
- * pair 1 = cta_group::2, M = 256 x N = 256 on every resident pair of SMs.  iters in
- * [1, 2^20].  ops_out (host pointer, may be NULL) receives 2 x the multiply-adds of the
+ * pair 1 = cta_group::2, M = 256 x N = 256 on every resident pair of SMs.  kind 2 = the
+ * warp-level mma.sync m16n8k32 (u8 x s8 -> s32) of the decode GEMV, from registers, 16 warps
+ * per SM with 8 independent accumulators each (pair ignored).  iters in [1, 2^20].  ops_out (host pointer, may be NULL) receives 2 x the multiply-adds of the
  * launch; divide by the launch's duration (CUDA events on `stream`) for the rate. */
 BL_API bl_status bl_mma_peak_probe(int kind, int pair, int iters, double* ops_out, void* stream);
 

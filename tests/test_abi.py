@@ -181,7 +181,7 @@ def test_status_values_match_header():
     assert {v: k for k, v in vals.items()} == _lib.STATUS_NAMES
 
 
-@pytest.mark.parametrize("kind,pair,iters", [(2, 0, 10), (0, 2, 10), (0, 0, 0), (1, 1, (1 << 20) + 1)])
+@pytest.mark.parametrize("kind,pair,iters", [(3, 0, 10), (-1, 0, 10), (0, 2, 10), (0, 0, 0), (1, 1, (1 << 20) + 1)])
 def test_peak_probe_validation(L, kind, pair, iters):
     assert _lib.status("bl_mma_peak_probe", kind, pair, iters, None, None) == 1
     assert len(_lib.last_error()) > 0
