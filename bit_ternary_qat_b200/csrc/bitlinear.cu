@@ -567,71 +567,25 @@ bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int gamma_stri
                       const int8_t* xq, const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st,
                       const DeviceInfo& dev) {
     constexpr int WB = NTILES == 1 ? 16 : 12;
-    auto kern = bl::ternary_gemv_kernel<NTILES, WB>;
-    int dev_id = 0;
-    cudaGetDevice(&dev_id);
-    if (dev_id < 0 || dev_id >= 64) return fail(BL_ERR_DEVICE, "device ordinal %d out of range", dev_id);
-    // Cluster size (4, else 2, else 1) and how many clusters are resident at once with one
-    // CTA per SM, queried once per device: the largest size whose clusters still cover
-    // (almost) every SM.
-    static std::atomic<int> cfg_c[64] = {}, cfg_n[64] = {};
-    int C = cfg_c[dev_id].load(), ncl_max = cfg_n[dev_id].load();
-    if (C == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
-        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        C = 1;
-        ncl_max = dev.sms;
-        for (int c : {4, 2}) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3((unsigned)(c * (dev.sms / c)));
-            cfg.blockDim = dim3(WB * 32);
-            cfg.dynamicSmemBytes = (size_t)dev.max_smem_optin;
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeClusterDimension;
-            at[0].val.clusterDim.x = (unsigned)c;
-            at[0].val.clusterDim.y = 1;
-            at[0].val.clusterDim.z = 1;
-            cfg.attrs = at;
-            cfg.numAttrs = 1;
-            int n = 0;
-            e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-            if (e != cudaSuccess) {
-                cudaGetLastError();
-                continue;
-            }
-            if (n * c >= dev.sms - 4) {
-                C = c;
-                ncl_max = n;
-                break;
-            }
-        }
-        cfg_n[dev_id].store(ncl_max);
-        cfg_c[dev_id].store(C);
-    }
     const int64_t n_rg = N / 16;
-    const int64_t ncl = n_rg < ncl_max ? n_rg : ncl_max;
-    const int64_t rg_per_cl = (n_rg + ncl - 1) / ncl;
-    const int max_rgs = (int)((rg_per_cl + C - 1) / C + 1);
+    const int64_t nb = n_rg < dev.sms ? n_rg : dev.sms;
+    const int max_rgs = (int)((n_rg + nb - 1) / nb);
     const size_t smem = bl::gemv_smem_bytes((int)B, (int)K, max_rgs);
     BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
                "GEMV needs %zu bytes of shared memory for B = %lld, K = %lld; at most %d fit", smem, (long long)B,
                (long long)K, dev.max_smem_optin);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(ncl * C));
-    cfg.blockDim = dim3(WB * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)C;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    cudaLaunchKernelEx(&cfg, kern, Wpacked, gamma, gamma_stride, (int)N, (int)K, xq, sx, (int)B, y, acc,
-                       g_wait_ns.load());
+    auto kern = bl::ternary_gemv_kernel<NTILES, WB>;
+    static std::atomic<uint64_t> attr_set{0};   // bit d: attribute set on device d
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (dev_id < 0 || dev_id >= 64) return fail(BL_ERR_DEVICE, "device ordinal %d out of range", dev_id);
+    if (!(attr_set.load() & (1ull << dev_id))) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_set.fetch_or(1ull << dev_id);
+    }
+    pdl_launch(kern, dim3((unsigned)nb), dim3(WB * 32), smem, st, Wpacked, gamma, gamma_stride, (int)N, (int)K, xq,
+               sx, (int)B, y, acc, g_wait_ns.load());
     return launched("ternary_gemv");
 }
 

@@ -48,56 +48,28 @@ __host__ __device__ inline size_t gemv_smem_bytes(int B, int K, int max_rgs) {
     const int spr = (K / 16 + 15) / 16;     // steps per row
     const size_t ld = (size_t)spr * 16 + 1;
     const size_t acc_ints = ((size_t)max_rgs * 16 * B + B + 1) & ~(size_t)1;
-    return 16 + (size_t)B * ld * 16 + acc_ints * 4 + sizeof(uint64_t) + 8 * sizeof(int) + 16;
+    return 16 + (size_t)B * ld * 16 + acc_ints * 4 + sizeof(uint64_t) + 16;
 }
 
 // ------------------------------------------------------------------------------------
-// Work split.  The grid is a set of clusters of C CTAs (C = 1, 2 or 4, one CTA per SM);
-// cluster c owns a balanced range [R0, R1) of the N/16 row groups (16 rows each), and the
-// (row group, 64-byte column block) steps of that range, numbered row-group-major, are
-// split into C equal contiguous runs, one per CTA, and each CTA's run into equal runs, one
-// per warp.  So every warp streams the same number of bytes (+-1 step), and the only
-// imbalance left is between clusters (row groups per cluster differ by at most one).
-// A row group belongs to the CTA that holds its first step; a CTA whose run ends inside a
-// row group adds its partial sums for it into the owner's shared accumulators through
-// distributed shared memory (cluster-scope integer reductions: exact and order free).
+// Block b owns the row groups (16 rows each) [rg0, rg1) of a balanced partition of the
+// N/16 row groups; its work is split into steps (row group, 64-byte column block) numbered
+// row-group-major, and warp w takes one contiguous, equally long run of them (+-1), so a
+// warp's run touches one or two row groups and all warps stream the same number of bytes.
 // A warp reads its weights straight from HBM into registers: per step, lane (g = lane/4,
 // t = lane%4) loads words 4t..4t+3 of the step's 64 bytes of rows g and g+8 (one 16-byte
 // load each; 8 rows x 64 contiguous bytes per warp instruction), kGemvU steps per batch,
 // two batches in registers (the next loading while the current one is multiplied), with
 // the load and compute positions advanced incrementally (no division in the loop).
-// Before it waits for the previous kernel in the stream, each warp asks L2 for the lines of
-// its first two batches (a prefetch only moves data into L2, which every SM's later
-// loads see coherently), so the first loads after the wait hit L2 instead of HBM.
 // Words 4t, 4t+1 feed one m16n8k32 k-block and words 4t+2, 4t+3 the next: byte i of word q
-// holds codes 16q + 4i + j, so k-slot 4t + i (16 + 4t + i) of a k-block pairs with
-// activation word x_j of group q = 4t (4t + 1), etc.  When its run leaves a row group the
-// warp folds its accumulators and adds them into the owning CTA's shared int32 sums of
-// that row group; after a cluster barrier every CTA writes y for the rows it owns.
+// holds codes 16q + 4i + j,
+// so k-slot 4t + i (16 + 4t + i) of a k-block pairs with activation word x_j of group q =
+// 4t (4t + 1), etc.  When its run leaves a row group the warp folds its accumulators and
+// adds them into the block's shared int32 sums of that row group (shared-memory integer
+// atomics: exact, order free); after a block barrier the block writes y for its rows.
 // The activation rows reach shared memory by bulk copy (one bounded mbarrier wait) while
-// the first weight batch is in flight, and are interleaved in place.
+// the first weight batch is already in flight, and are interleaved in place.
 // ------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void red_add_shared_cluster(uint32_t cluster_addr, int v) {
-    asm volatile("red.shared::cluster.add.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
-
-// First step (cluster-local) of CTA c's run, and the first row group (cluster-local) that
-// CTA c owns: the one whose first step lies in its run.
-__device__ __forceinline__ int gemv_cta_step0(int S, int c, int C) {
-    return static_cast<int>(static_cast<int64_t>(S) * c / C);
-}
-__device__ __forceinline__ int gemv_own0(int S, int c, int C, int spr) {
-    return (gemv_cta_step0(S, c, C) + spr - 1) / spr;
-}
-
 template <int NTILES, int WB>
 __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     const uint8_t* __restrict__ W, const float* __restrict__ gamma, int gamma_stride, int N, int K,
@@ -111,62 +83,21 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     const int Gp = spr * 16;                     // staged activation groups per row (zero past G)
     const int ld = Gp + 1;
     const int n_rg = N / 16;
-    // cluster partition
-    const int C = static_cast<int>(cluster_nctarank());
-    const int rank = static_cast<int>(cluster_ctarank());
-    const int cl = static_cast<int>(blockIdx.x) / C, ncl = static_cast<int>(gridDim.x) / C;
-    const int R0 = static_cast<int>(static_cast<int64_t>(cl) * n_rg / ncl);
-    const int R1 = static_cast<int>(static_cast<int64_t>(cl + 1) * n_rg / ncl);
-    const int S = (R1 - R0) * spr;
-    const int cs0 = gemv_cta_step0(S, rank, C), cs1 = gemv_cta_step0(S, rank + 1, C);
-    const int own0 = gemv_own0(S, rank, C, spr);
-    const int own1 = rank + 1 < C ? gemv_own0(S, rank + 1, C, spr) : R1 - R0;
-    const int nown = own1 - own0;                 // row groups this CTA owns (may be 0)
+    const int rg0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * n_rg / gridDim.x);
+    const int rg1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * n_rg / gridDim.x);
+    const int nrg = rg1 - rg0;
     int4* xs = reinterpret_cast<int4*>(base);                                  // [B][ld]
-    int* accs = reinterpret_cast<int*>(xs + static_cast<size_t>(B) * ld);      // [nown*16][B]
-    int* xsum = accs + nown * 16 * B;                                         // [B]
-    uint64_t* xbar = reinterpret_cast<uint64_t*>(accs + ((nown * 16 * B + B + 1) & ~1));
-    int* own_b = reinterpret_cast<int*>(xbar + 1);                            // [C + 1] first owned row groups
+    int* accs = reinterpret_cast<int*>(xs + static_cast<size_t>(B) * ld);      // [nrg*16][B]
+    int* xsum = accs + nrg * 16 * B;                                          // [B]
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(accs + ((nrg * 16 * B + B + 1) & ~1));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-
-    // this warp's run of steps [i0, i1) (cluster-local, row-group-major)
-    const int nsteps = cs1 - cs0;
-    const int i0 = cs0 + static_cast<int>(static_cast<int64_t>(warp) * nsteps / WB);
-    const int i1 = cs0 + static_cast<int>(static_cast<int64_t>(warp + 1) * nsteps / WB);
-    // Load cursor: the next step to load, its position in its row, and this lane's address of
-    // its 16-byte slice of row g (row g+8 is 8 rows further).  A slice past the row end (the
-    // last step of a row when K/4 is not a multiple of 64) loads as zeros.
-    const int64_t r8 = 8 * static_cast<int64_t>(row_bytes);
-    const int64_t rg_jump = 16 * static_cast<int64_t>(row_bytes) - static_cast<int64_t>(spr) * kGemvStepBytes;
-    const bool tail_ok = (spr - 1) * kGemvStepBytes + 16 * t < row_bytes;
-    int li = i0, l_s = i0 % spr;
-    const uint8_t* lp = W + (static_cast<int64_t>(R0 + i0 / spr) * 16 + g) * row_bytes +
-                        static_cast<int64_t>(l_s) * kGemvStepBytes + 16 * t;
-    // L2 prefetch of the first two batches (lanes t = 0 cover each 64-byte step slice)
-    if (t == 0) {
-        int pi = li, ps = l_s;
-        const uint8_t* pp = lp;
-        for (int u = 0; u < 2 * kGemvU && pi < i1; ++u) {
-            prefetch_l2(pp);
-            prefetch_l2(pp + r8);
-            ++pi;
-            pp += kGemvStepBytes;
-            if (++ps == spr) {
-                ps = 0;
-                pp += rg_jump;
-            }
-        }
-    }
-
     if (threadIdx.x == 0) {
         mbar_init(xbar, 1);
         fence_mbar_init();
     }
-    if (threadIdx.x <= C) own_b[threadIdx.x] = threadIdx.x < C ? gemv_own0(S, threadIdx.x, C, spr) : R1 - R0;
-    for (int idx = threadIdx.x; idx < nown * 16 * B; idx += WB * 32) accs[idx] = 0;
-    cluster_sync_all();      // every CTA's sums are zero before any remote reduction
+    __syncthreads();
     pdl_trigger_and_wait();
     if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(B * K));
@@ -174,6 +105,19 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
             bulk_load(xs + static_cast<size_t>(b) * ld, xq + static_cast<int64_t>(b) * K, static_cast<uint32_t>(K), xbar);
     }
 
+    // this warp's run of steps [i0, i1) of the block's row-group-major sequence
+    const int nsteps = nrg * spr;
+    const int i0 = static_cast<int>(static_cast<int64_t>(warp) * nsteps / WB);
+    const int i1 = static_cast<int>(static_cast<int64_t>(warp + 1) * nsteps / WB);
+    // Load cursor: the next step to load, its position in its row, and this lane's address of
+    // its 16-byte slice of row g (row g+8 is 8 rows further).  A slice past the row end (the
+    // last step of a row when K/4 is not a multiple of 64) loads as zeros.
+    const int64_t r8 = 8 * static_cast<int64_t>(row_bytes);
+    const int64_t rg_jump = 16 * static_cast<int64_t>(row_bytes) - static_cast<int64_t>(spr) * kGemvStepBytes;
+    const bool tail_ok = (spr - 1) * kGemvStepBytes + 16 * t < row_bytes;
+    int li = i0, l_s = i0 % spr;
+    const uint8_t* lp = W + (static_cast<int64_t>(rg0 + i0 / spr) * 16 + g) * row_bytes +
+                        static_cast<int64_t>(l_s) * kGemvStepBytes + 16 * t;
     auto load_next = [&](uint4& ra, uint4& rb) {
         ra = make_uint4(0u, 0u, 0u, 0u);
         rb = ra;
@@ -193,7 +137,8 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
 #pragma unroll
     for (int u = 0; u < kGemvU; ++u) load_next(Aa[u], Ab[u]);
 
-    // activations: wait for the copies, interleave in place (zero past K)
+    // activations: wait for the copies, interleave in place (zero past K), clear the sums
+    for (int idx = threadIdx.x; idx < nrg * 16 * B; idx += WB * 32) accs[idx] = 0;
     mbar_wait(xbar, 0, wait_ns, nullptr);
     for (int idx = threadIdx.x; idx < B * Gp; idx += WB * 32) {
         const int b = idx / Gp, gg = idx - b * Gp;
@@ -237,12 +182,7 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
         for (int nt = 0; nt < NTILES; ++nt)
 #pragma unroll
             for (int q = 0; q < 4; ++q) d[j][nt][q] = 0;
-    // fold the accumulators of cluster-local row group rgl into its owner's shared sums
     auto flush = [&](int rgl) {
-        int owner = C - 1;
-        while (owner > 0 && own_b[owner] > rgl) --owner;
-        const int slot = rgl - own_b[owner];
-        const bool remote = owner != rank;
 #pragma unroll
         for (int nt = 0; nt < NTILES; ++nt)
 #pragma unroll
@@ -250,11 +190,7 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
                 const int tot = d[0][nt][q] + (d[1][nt][q] >> 2) + (d[2][nt][q] >> 4) + (d[3][nt][q] >> 6);
                 const int b = nt * 8 + 2 * t + (q & 1);
                 const int r = (q < 2) ? g : g + 8;
-                if (b < B) {
-                    int* dst = &accs[(slot * 16 + r) * B + b];
-                    if (!remote) atomicAdd(dst, tot);
-                    else red_add_shared_cluster(mapa_shared(smem_u32(dst), static_cast<uint32_t>(owner)), tot);
-                }
+                if (b < B) atomicAdd(&accs[(rgl * 16 + r) * B + b], tot);
                 d[0][nt][q] = d[1][nt][q] = d[2][nt][q] = d[3][nt][q] = 0;
             }
     };
@@ -308,16 +244,15 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
         for (int u = 0; u < kGemvU; ++u) load_next(Aa[u], Ab[u]);
         process(Ba, Bb);
     }
-    cluster_sync_all();      // every CTA's reductions into this CTA's sums have landed
+    __syncthreads();
 
-    // y[b][n] = (acc - 2 sum x_b) * fl(gamma_n / s_b) for the rows this CTA owns, row-fastest
+    // y[b][n] = (acc - 2 sum x_b) * fl(gamma_n / s_b) for this block's rows, row-fastest
     // (gamma_n = gamma[n * gamma_stride]: one scale, or one per weight row)
-    const int rows = nown * 16;
-    const int n0 = (R0 + own0) * 16;
+    const int rows = nrg * 16;
     for (int idx = threadIdx.x; idx < rows * B; idx += WB * 32) {
         const int b = idx / rows, r = idx - b * rows;
         const int acc = accs[r * B + b] - 2 * xsum[b];
-        const int n = n0 + r;
+        const int n = rg0 * 16 + r;
         const int64_t o = static_cast<int64_t>(b) * N + n;
         const float gm = __ldg(gamma + static_cast<int64_t>(n) * gamma_stride);
         y[o] = __fmul_rn(static_cast<float>(acc), __fdiv_rn(gm, __ldg(sx + b)));
