@@ -451,29 +451,54 @@ size_t opt_ws_bytes() { return kOptStepOffset + 16; }
 
 size_t dg_ws_bytes(int64_t K) { return sizeof(float) * (size_t)bl::kBwdMaxBlocks * (size_t)K; }
 
-template <bool kBf16X, int VPT>
+// Persistent grid: as many blocks as are resident at once (queried once per device and
+// instantiation), at most kBwdMaxBlocks and at most one per row.
+template <bool kBf16X, int NT, int VPT, bool kGain>
 int launch_rmsnorm_bwd_v(const void* X, const float* rinv, const float* g, float* dX, int64_t T, int64_t K,
                          float* partial, int sms, cudaStream_t st) {
-    constexpr int R = VPT == 1 ? 4 : 1;   // 2 rows per iteration measured 15 % slower than 1 at VPT 2
-    int64_t grid = (T + R - 1) / R;
-    const int64_t cap = sms * 4 < bl::kBwdMaxBlocks ? sms * 4 : bl::kBwdMaxBlocks;
-    if (grid > cap) grid = cap;
-    pdl_launch(bl::rmsnorm_bwd_kernel<kBf16X, VPT, R>, dim3((unsigned)grid), dim3(bl::kBwdThreads), 0, st, X, rinv, g,
-               dX, (int)T, (int)K, partial);
+    auto kern = bl::rmsnorm_bwd_kernel<kBf16X, NT, VPT, kGain>;
+    static std::atomic<int> per_sm[64] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    int b = (dev_id >= 0 && dev_id < 64) ? per_sm[dev_id].load() : 0;
+    if (b == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, NT, 0) != cudaSuccess || b < 1) b = 1;
+        if (dev_id >= 0 && dev_id < 64) per_sm[dev_id].store(b);
+    }
+    int64_t grid = (int64_t)b * sms;
+    if (grid > bl::kBwdMaxBlocks) grid = bl::kBwdMaxBlocks;
+    if (grid > T) grid = T;
+    pdl_launch(kern, dim3((unsigned)grid), dim3(NT), 0, st, X, rinv, g, dX, (int)T, (int)K, partial);
     return (int)grid;
+}
+
+// Block size: the smallest of 128 / 256 / 512 / 1024 threads that covers a row with at most
+// four 16-byte column vectors per thread (K <= 16384).
+template <bool kBf16X, bool kGain>
+int launch_rmsnorm_bwd_g(const void* X, const float* rinv, const float* g, float* dX, int64_t T, int64_t K,
+                         float* partial, int sms, cudaStream_t st) {
+    const int64_t nvec = K / 4;
+#define BL_BWD(NT)                                                                                              \
+    if (nvec <= 4 * (NT)) {                                                                                     \
+        const int64_t vpt = (nvec + (NT) - 1) / (NT);                                                          \
+        if (vpt <= 1) return launch_rmsnorm_bwd_v<kBf16X, NT, 1, kGain>(X, rinv, g, dX, T, K, partial, sms, st); \
+        if (vpt <= 2) return launch_rmsnorm_bwd_v<kBf16X, NT, 2, kGain>(X, rinv, g, dX, T, K, partial, sms, st); \
+        if (vpt <= 3) return launch_rmsnorm_bwd_v<kBf16X, NT, 3, kGain>(X, rinv, g, dX, T, K, partial, sms, st); \
+        return launch_rmsnorm_bwd_v<kBf16X, NT, 4, kGain>(X, rinv, g, dX, T, K, partial, sms, st);               \
+    }
+    BL_BWD(128)
+    BL_BWD(256)
+    BL_BWD(512)
+    BL_BWD(1024)
+#undef BL_BWD
+    return 0;
 }
 
 template <bool kBf16X>
 int launch_rmsnorm_bwd(const void* X, const float* rinv, const float* g, float* dX, int64_t T, int64_t K,
                        float* partial, int sms, cudaStream_t st) {
-    const int64_t nvec = K / 4;
-    const int64_t vpt = (nvec + bl::kBwdThreads - 1) / bl::kBwdThreads;
-    if (vpt <= 1) return launch_rmsnorm_bwd_v<kBf16X, 1>(X, rinv, g, dX, T, K, partial, sms, st);
-    if (vpt <= 2) return launch_rmsnorm_bwd_v<kBf16X, 2>(X, rinv, g, dX, T, K, partial, sms, st);
-    if (vpt <= 4) return launch_rmsnorm_bwd_v<kBf16X, 4>(X, rinv, g, dX, T, K, partial, sms, st);
-    if (vpt <= 8) return launch_rmsnorm_bwd_v<kBf16X, 8>(X, rinv, g, dX, T, K, partial, sms, st);
-    if (vpt <= 12) return launch_rmsnorm_bwd_v<kBf16X, 12>(X, rinv, g, dX, T, K, partial, sms, st);
-    return launch_rmsnorm_bwd_v<kBf16X, 16>(X, rinv, g, dX, T, K, partial, sms, st);
+    if (g != nullptr) return launch_rmsnorm_bwd_g<kBf16X, true>(X, rinv, g, dX, T, K, partial, sms, st);
+    return launch_rmsnorm_bwd_g<kBf16X, false>(X, rinv, g, dX, T, K, partial, sms, st);
 }
 
 bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const float* g, float* dX, int64_t T,

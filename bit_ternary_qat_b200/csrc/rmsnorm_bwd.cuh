@@ -14,115 +14,130 @@
 //     are read from HBM exactly once, dX written once, in place, by the same thread);
 //   * dg accumulates in registers across all rows the block visits, and each block writes
 //     one partial dg row; dg_reduce_kernel sums the partials in a fixed order.
-// A block processes R rows per iteration (rows b, b + G, ...) with a single block
-// reduction for the R row sums, so R rows of loads are in flight per thread.
 #pragma once
 #include "common.cuh"
 
 namespace bl {
 
-constexpr int kBwdThreads = 256;
 constexpr int kBwdMaxBlocks = 592;   // partial dg rows; fixed so the workspace size is device-independent
-constexpr int kBwdMaxVpt = 16;       // K <= 16 * 4 * 256 = 16384
 
+// Persistent row kernel: grid = G blocks (<= kBwdMaxBlocks, all resident), block = NT
+// threads; thread i owns column vectors i + j*NT (4 columns each), j < VPT, of every row.
+// Block b visits rows b, b + G, b + 2G, ...; while it reduces and stores one row, the loads of
+// its next row are already in flight (two register buffers, the loop unrolled by two so the
+// buffers alternate without copies), so every SM keeps about two rows per block in flight.
+// One block barrier per row: the warp sums go to one of two shared arrays, alternating by row.
+// The arithmetic of a row is fixed (per thread over j and the 4 columns, then the warp
+// butterfly, then the warps in order), so results do not depend on the grid.
 template <bool kBf16X>
-__device__ __forceinline__ void load_x4(const void* X, int64_t idx_vec4, float (&x)[4]) {
-    if constexpr (kBf16X) {
-        const uint2 raw = __ldcs(reinterpret_cast<const uint2*>(X) + idx_vec4);
-        x[0] = __uint_as_float(raw.x << 16); x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-        x[2] = __uint_as_float(raw.y << 16); x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-    } else {
-        const float4 raw = __ldcs(reinterpret_cast<const float4*>(X) + idx_vec4);
-        x[0] = raw.x; x[1] = raw.y; x[2] = raw.z; x[3] = raw.w;
+struct BwdXRaw;
+template <>
+struct BwdXRaw<true> {
+    using T = uint2;   // 4 bf16
+    __device__ __forceinline__ static void widen(const uint2& r, float (&x)[4]) {
+        x[0] = __uint_as_float(r.x << 16); x[1] = __uint_as_float(r.x & 0xFFFF0000u);
+        x[2] = __uint_as_float(r.y << 16); x[3] = __uint_as_float(r.y & 0xFFFF0000u);
     }
-}
+};
+template <>
+struct BwdXRaw<false> {
+    using T = float4;
+    __device__ __forceinline__ static void widen(const float4& r, float (&x)[4]) {
+        x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+    }
+};
 
-// grid = G blocks (<= kBwdMaxBlocks), block = kBwdThreads; thread i owns vectors i + j*NT.
-template <bool kBf16X, int VPT, int R>
-__global__ void __launch_bounds__(kBwdThreads) rmsnorm_bwd_kernel(const void* __restrict__ X,
-                                                                  const float* __restrict__ rinv,
-                                                                  const float* __restrict__ g, float* dX, int T,
-                                                                  int K, float* __restrict__ dg_partial) {
-    constexpr int NT = kBwdThreads;
-    __shared__ float red[R][NT / 32];
+template <bool kBf16X, int NT, int VPT, bool kGain, bool kPf = (NT < 1024 || (kBf16X && VPT <= 3 && !kGain))>
+__global__ void __launch_bounds__(NT) rmsnorm_bwd_kernel(const void* __restrict__ X,
+                                                         const float* __restrict__ rinv,
+                                                         const float* __restrict__ g, float* dX, int T,
+                                                         int K, float* __restrict__ dg_partial) {
+    using XR = typename BwdXRaw<kBf16X>::T;
+    __shared__ float red[2][NT / 32];
     pdl_trigger_and_wait();
     const int nvec = K / 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x;
 
-    float gk[VPT][4];
     float dga[VPT][4];
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-        const int v = threadIdx.x + j * NT;
+    for (int j = 0; j < VPT; ++j)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            gk[j][e] = (g != nullptr && v < nvec) ? __ldg(g + 4 * v + e) : 1.0f;
-            dga[j][e] = 0.0f;
-        }
-    }
+        for (int e = 0; e < 4; ++e) dga[j][e] = 0.0f;
 
-    const int G = gridDim.x;
-    for (int t0 = blockIdx.x; t0 < T; t0 += G * R) {
-        float d[R][VPT][4], u[R][VPT][4], rr[R];
-        float part[R];
+    float4 dA[VPT], dB[kPf ? VPT : 1];
+    XR xA[VPT], xB[kPf ? VPT : 1];
+    auto load_row = [&](int t, float4 (&d)[VPT], XR (&x)[VPT]) {
 #pragma unroll
-        for (int q = 0; q < R; ++q) {
-            const int t = t0 + q * G;
-            part[q] = 0.0f;
-            rr[q] = t < T ? __ldg(rinv + t) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                const int v = threadIdx.x + j * NT;
-                if (t < T && v < nvec) {
-                    const float4 dv = reinterpret_cast<const float4*>(dX + static_cast<int64_t>(t) * K)[v];
-                    d[q][j][0] = dv.x; d[q][j][1] = dv.y; d[q][j][2] = dv.z; d[q][j][3] = dv.w;
-                    float x[4];
-                    load_x4<kBf16X>(X, static_cast<int64_t>(t) * nvec + v, x);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) u[q][j][e] = x[e] * rr[q];
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) { d[q][j][e] = 0.0f; u[q][j][e] = 0.0f; }
-                }
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+            if (v < nvec) {
+                d[j] = __ldcs(reinterpret_cast<const float4*>(dX + static_cast<int64_t>(t) * K) + v);
+                x[j] = __ldcs(reinterpret_cast<const XR*>(X) + static_cast<int64_t>(t) * nvec + v);
+            } else {
+                d[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                x[j] = XR{};
             }
         }
+    };
+    // one row: c_t = (1/K) sum_k g d u, dX = r (g d - u c_t), dg += d u
+    auto row = [&](int t, int par, const float4 (&d4)[VPT], const XR (&xr)[VPT]) {
+        const float rr = __ldg(rinv + t);
+        float d[VPT][4], u[VPT][4], gk[VPT][4];
+        float part = 0.0f;
 #pragma unroll
-        for (int q = 0; q < R; ++q)
-#pragma unroll
-            for (int j = 0; j < VPT; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    part[q] = fmaf(gk[j][e] * d[q][j][e], u[q][j][e], part[q]);
-                    dga[j][e] = fmaf(d[q][j][e], u[q][j][e], dga[j][e]);
-                }
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
-            const float w = warp_sum(part[q]);
-            if (lane == 0) red[q][warp] = w;
-        }
-        __syncthreads();
-        float c[R];
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
-            float tot = 0.0f;
-#pragma unroll
-            for (int w = 0; w < NT / 32; ++w) tot += red[q][w];
-            c[q] = tot / static_cast<float>(K);
-        }
-        __syncthreads();
-#pragma unroll
-        for (int q = 0; q < R; ++q) {
-            const int t = t0 + q * G;
-            if (t >= T) continue;
-#pragma unroll
-            for (int j = 0; j < VPT; ++j) {
-                const int v = threadIdx.x + j * NT;
-                if (v >= nvec) continue;
-                float o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[e] = rr[q] * (gk[j][e] * d[q][j][e] - u[q][j][e] * c[q]);
-                reinterpret_cast<float4*>(dX + static_cast<int64_t>(t) * K)[v] = make_float4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+            float x[4];
+            BwdXRaw<kBf16X>::widen(xr[j], x);
+            d[j][0] = d4[j].x; d[j][1] = d4[j].y; d[j][2] = d4[j].z; d[j][3] = d4[j].w;
+            float4 gv = make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            if constexpr (kGain) {
+                if (v < nvec) gv = __ldg(reinterpret_cast<const float4*>(g) + v);
             }
+            gk[j][0] = gv.x; gk[j][1] = gv.y; gk[j][2] = gv.z; gk[j][3] = gv.w;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                u[j][e] = x[e] * rr;
+                part = fmaf(gk[j][e] * d[j][e], u[j][e], part);
+                dga[j][e] = fmaf(d[j][e], u[j][e], dga[j][e]);
+            }
+        }
+        const float w = warp_sum(part);
+        if (lane == 0) red[par][warp] = w;
+        __syncthreads();
+        float tot = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NT / 32; ++i) tot += red[par][i];
+        const float c = tot / static_cast<float>(K);
+#pragma unroll
+        for (int j = 0; j < VPT; ++j) {
+            const int v = threadIdx.x + j * NT;
+            if (v >= nvec) continue;
+            float o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = rr * (gk[j][e] * d[j][e] - u[j][e] * c);
+            reinterpret_cast<float4*>(dX + static_cast<int64_t>(t) * K)[v] = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    };
+
+    int t = blockIdx.x;
+    if constexpr (kPf) {
+        if (t < T) load_row(t, dA, xA);
+        while (t < T) {
+            if (t + G < T) load_row(t + G, dB, xB);
+            row(t, 0, dA, xA);
+            t += G;
+            if (t >= T) break;
+            if (t + G < T) load_row(t + G, dA, xA);
+            row(t, 1, dB, xB);
+            t += G;
+        }
+    } else {
+        // 1024-thread blocks hold at most 64 registers per thread: one row buffer
+        for (int par = 0; t < T; t += G, par ^= 1) {
+            load_row(t, dA, xA);
+            row(t, par, dA, xA);
         }
     }
     if (dg_partial != nullptr) {
