@@ -869,10 +869,48 @@ def gemv_measure(bl, torch, dev, flush, pk, imma_peak=None):
             rec["imma_bound_us"] = mma_ops / (imma_peak * 1e12) * 1e6
             rec["frac_imma"] = rec["imma_bound_us"] / rec["us"]
         out[f"B{B}"] = rec
+    # per-launch fixed cost vs streaming rate: the same launches on a weight twice as tall
+    # (57344 x 8192, 117 MB; 2 copies cycled): marginal rate = the extra 58.7 MB / the extra time
+    W2, _ = synth.decode_inputs(1, 2 * N, K, seed=44)
+    q2 = bl.bitlinear_quant_weight(W2.to(dev), want_i8=False, want_bf16=False)
+    del W2
+    packs2 = [q2["packed"], q2["packed"].clone()]
+    for B in (1, 4, 16):
+        _, x = synth.decode_inputs(B, 16, K, seed=40 + B)
+        aq = bl.bitlinear_act_quant(x.to(dev), apply_rmsnorm=False, want_xdq=False)
+        y = torch.empty(B, 2 * N, dtype=torch.float32, device=dev)
+        for i in range(4):
+            bl.ternary_gemv(packs2[i % 2], q2["gamma"], K, aq["xq"], aq["sx"], y=y)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(reps):
+                bl.ternary_gemv(packs2[i % 2], q2["gamma"], K, aq["xq"], aq["sx"], y=y)
+        graph.replay()
+        samples = []
+        for _ in range(5):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            samples.append(a.elapsed_time(b) / reps)
+        del graph
+        us2 = statistics.median(samples) * 1e3
+        rec = out[f"B{B}"]
+        extra = us2 - rec["us"]
+        rec["us_2x_rows"] = us2
+        rec["marginal_GB/s"] = (N * K // 4) / (extra * 1e-6) / 1e9 if extra > 0 else None
+        rec["marginal_frac_hbm"] = rec["marginal_GB/s"] / pk["hbm"] if rec["marginal_GB/s"] else None
+        rec["fixed_us"] = rec["us"] - extra
+    del packs2, q2
     out["hbm_peak_GBs"] = pk["hbm"]
     out["imma_peak_T"] = imma_peak
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
-                       "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5")
+                       "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5; "
+                       "marginal rate and fixed cost from the same launches on a 57344x8192 weight (2 copies)")
     return out
 
 
