@@ -667,6 +667,7 @@ def main():
     sub = None
     if not args.no_sub:
         sub = {"decode_gemv": gemv_measure(bl, torch, dev, flush, pk, imma_peak=tpk["imma_sync"]),
+               "hbm_kernels_b2b": hbm_b2b_measure(bl, torch, dev, flush, pk),
                "configs": configs_measure(bl, torch, dev, flush)}
 
     cpu = None
@@ -700,6 +701,82 @@ def main():
     if world > 1:
         dist.destroy_process_group()
 
+
+
+def timed_b2b(bl, torch, flush, calls, reps):
+    """`reps` launches cycling over `calls`, captured in one CUDA graph between one pair of CUDA
+    events (median of 5 replays, L2 flushed before each): microseconds per launch."""
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(reps):
+            calls[i % len(calls)]()
+    graph.replay()
+    torch.cuda.synchronize()
+    samples = []
+    for _ in range(5):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        samples.append(a.elapsed_time(b) / reps)
+    del graph
+    assert bl.check_device_status() == 0
+    return statistics.median(samples) * 1e3
+
+
+def hbm_b2b_measure(bl, torch, dev, flush, pk):
+    """The HBM-bound kernels of the step at the 7B layer's sizes (16384 tokens; d_in 4096 and
+    11008; weights 4096 x 4096 and 11008 x 4096), each launched back to back over input copies
+    that together exceed L2, so every launch reads from HBM; bytes are algorithmic (each tensor
+    read once, each output written once)."""
+    from bit_ternary_qat_b200 import synth
+    gen = synth.generator(91)
+    T = 16384
+    out = {}
+
+    def row(us, nbytes, note):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": us, "GB/s": gbs, "frac_hbm": gbs / pk["hbm"], "bytes": nbytes, "note": note}
+
+    for K, copies in ((4096, 3), (11008, 2)):
+        Xs = [synth.normal((T, K), 1.0, gen).to(torch.bfloat16).to(dev) for _ in range(copies)]
+        a = dict(xq=torch.empty(T, K, dtype=torch.int8, device=dev), sx=torch.empty(T, device=dev),
+                 rinv=torch.empty(T, device=dev), xdq=torch.empty(T, K, dtype=torch.bfloat16, device=dev))
+        us = timed_b2b(bl, torch, flush, [lambda X=X: bl.bitlinear_act_quant(X, out=a) for X in Xs], 4 * copies)
+        out[f"act_quant_{T}x{K}"] = row(us, T * K * 5 + 8 * T, "RMSNorm + per-token int8 codes + bf16 X_dq")
+        ws = bl.workspace(T, 16, K, dev)
+        dg = torch.empty(K, device=dev)
+        dXs = [synth.normal((T, K), 1e-2, gen).to(dev) for _ in range(2 if K == 4096 else 1)]
+        Xb = Xs[:len(dXs)]
+        us = timed_b2b(bl, torch, flush, [lambda X=X, d=d: bl.bitlinear_rmsnorm_backward(X, a["rinv"], d, ws=ws, dg=dg)
+                                          for X, d in zip(Xb, dXs)], 4 * len(dXs))
+        out[f"rmsnorm_bwd_{T}x{K}"] = row(us, T * K * 10 + 4 * T, "reads fp32 dX_hat and bf16 X, writes fp32 dX "
+                                                                    "(plus the dg partial rows and their sum)")
+        del Xs, dXs, a, ws
+        torch.cuda.empty_cache()
+    for (N, K), copies in (((4096, 4096), 4), ((11008, 4096), 2)):
+        Ws = [synth.normal((N, K), 0.02, gen).to(dev) for _ in range(copies)]
+        ws = bl.workspace(1, N, K, dev)
+        q = dict(gamma=torch.empty(1, dtype=torch.float32, device=dev),
+                 wq_i8=torch.empty(N, K, dtype=torch.int8, device=dev),
+                 wq_bf16=torch.empty(N, K, dtype=torch.bfloat16, device=dev),
+                 packed=torch.empty(N, K // 4, dtype=torch.uint8, device=dev))
+        us = timed_b2b(bl, torch, flush, [lambda W=W: bl.bitlinear_quant_weight(W, ws=ws, out=q) for W in Ws],
+                       4 * copies)
+        rec = row(us, int(N * K * 7.25), "two launches: |W| partial sums, then codes (int8 + bf16 + 2-bit); "
+                                        "W is read twice (the second read hits L2 only when W fits there)")
+        rec["frac_hbm_both_reads"] = (N * K * 11.25) / (us * 1e-6) / 1e9 / pk["hbm"]
+        out[f"quant_weight_{N}x{K}"] = rec
+        del Ws, ws, q
+        torch.cuda.empty_cache()
+    out["hbm_peak_GBs"] = pk["hbm"]
+    return out
 
 def configs_measure(bl, torch, dev, flush, steps: int = 5):
     """The other training configurations' full steps (single, square, mlp7b): per layer weight

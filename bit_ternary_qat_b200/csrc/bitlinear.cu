@@ -553,9 +553,12 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     }
     a.splits = splits;
     const size_t budget = (size_t)dev.max_smem_optin;
-    // rings: 4 decoded and 4 activation stages; the packed ring (16 KB stages, 512 codes per
+    // rings: 8 decoded and 8 activation stages for token tiles of up to 32 (4 for wider
+    // tiles, whose activation stages are larger); the packed ring (16 KB stages, 512 codes per
     // row) takes the rest of shared memory (at most 12 stages)
-    int pstages = (int)((budget - bl::pk_smem_bytes((int)bt, 0)) / bl::kPkPBytes);
+    const int dstages = (bt <= 32 && bl::pk_smem_bytes((int)bt, 4, 2 * bl::kPkDecGroups) <= budget)
+                            ? 2 * bl::kPkDecGroups : bl::kPkDecGroups;
+    int pstages = (int)((budget - bl::pk_smem_bytes((int)bt, 0, dstages)) / bl::kPkPBytes);
     pstages = std::min(pstages, bl::kPkMaxPStages);
     BL_REQUIRE(pstages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
     a.pstages = pstages;
@@ -565,8 +568,9 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     CUtensorMap tp, tx;
     BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, bl::kPkBM));
     BL_TRY(make_tmap(&tx, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, (uint32_t)bt));
-    auto kern = bl::tc_gemm_packed_kernel<kBf16Out>;
-    const size_t smem = bl::pk_smem_bytes((int)bt, pstages);
+    auto kern = dstages == 2 * bl::kPkDecGroups ? bl::tc_gemm_packed_kernel<kBf16Out, 2 * bl::kPkDecGroups>
+                                                : bl::tc_gemm_packed_kernel<kBf16Out, bl::kPkDecGroups>;
+    const size_t smem = bl::pk_smem_bytes((int)bt, pstages, dstages);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     const int64_t units = base * splits;
@@ -587,9 +591,9 @@ constexpr int64_t kMaxRowK = 16384;
 
 // One block per SM (at most one per row group) of 16 warps (12 for two n-tiles, whose
 // accumulators need more registers).
-template <int NTILES>
+template <int NTILES, bool kBf16Out = false>
 bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int gamma_stride, int64_t N, int64_t K,
-                      const int8_t* xq, const float* sx, int64_t B, float* y, int32_t* acc, cudaStream_t st,
+                      const int8_t* xq, const float* sx, int64_t B, void* y, int32_t* acc, cudaStream_t st,
                       const DeviceInfo& dev) {
     constexpr int WB = NTILES == 1 ? 16 : 12;
     const int64_t n_rg = N / 16;
@@ -599,7 +603,7 @@ bl_status launch_gemv(const uint8_t* Wpacked, const float* gamma, int gamma_stri
     BL_REQUIRE(smem <= (size_t)dev.max_smem_optin, BL_ERR_UNSUPPORTED_SHAPE,
                "GEMV needs %zu bytes of shared memory for B = %lld, K = %lld; at most %d fit", smem, (long long)B,
                (long long)K, dev.max_smem_optin);
-    auto kern = bl::ternary_gemv_kernel<NTILES, WB>;
+    auto kern = bl::ternary_gemv_kernel<NTILES, WB, kBf16Out>;
     static std::atomic<uint64_t> attr_set{0};   // bit d: attribute set on device d
     int dev_id = 0;
     cudaGetDevice(&dev_id);
@@ -1081,6 +1085,21 @@ bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, 
     int32_t* scratch = static_cast<int32_t*>(ws);
     const size_t scratch_bytes = ws != nullptr ? ws_bytes : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // Up to 16 tokens whose activation rows fit a block's shared memory: the decode GEMV's
+    // kernel (codes decoded in registers, warp-level int8 MMA), which streams the packed
+    // weight faster than the tensor-core tile with 16-column MMAs.
+    if (T <= 16 && K <= 65536) {
+        const int64_t n_rg = N / 16;
+        const int64_t nb = n_rg < dev.sms ? n_rg : dev.sms;
+        const int max_rgs = (int)((n_rg + nb - 1) / nb);
+        if (bl::gemv_smem_bytes((int)T, (int)K, max_rgs) <= (size_t)dev.max_smem_optin) {
+            if (y_dt == BL_BF16)
+                return T <= 8 ? launch_gemv<1, true>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev)
+                              : launch_gemv<2, true>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev);
+            return T <= 8 ? launch_gemv<1, false>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev)
+                          : launch_gemv<2, false>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev);
+        }
+    }
     if (y_dt == BL_BF16)
         return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
     return launch_packed<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);

@@ -16,11 +16,11 @@
 //              the decoded ring): warp 0 keeps both full with TMA loads.  A packed box moves 128 bytes per
 //              weight row: with 32-byte rows the copy engine's per-row rate, not HBM, was the
 //              limit (measured);
-//   decoded ring (4 stages of 128 rows x 128 int8 codes, 128-byte-swizzled K-major):
-//              warps 6-21, four groups of four warps, group g owning decoded stage g, decode
-//              one k-block of a packed stage into the int8 layout the MMA reads (what TMA
-//              would have written for int8 codes), fence the writes to the async proxy and
-//              arrive;
+//   decoded ring (DS = 4 or 8 stages of 128 rows x 128 int8 codes, 128-byte-swizzled
+//              K-major): warps 6-21, four groups of four warps, group g decoding the k-blocks
+//              q = g mod 4 into stage q mod DS (stage g, or stages g and g + 4 in turn), one
+//              k-block of a packed stage into the int8 layout the MMA reads (what TMA would
+//              have written for int8 codes), fence the writes to the async proxy and arrive;
 //   warp 1     MMA issuer (tcgen05.mma kind::i8, one thread), accumulators in TMEM
 //              (two 256-column buffers: the epilogue of one unit overlaps the next);
 //   warps 2-5  epilogue: tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (warp-wide
@@ -29,10 +29,10 @@
 //              partial sums of split sp stored to slice sp of a workspace, which
 //              pk_finalize_kernel adds in split order (exact) before the same epilogue.
 // Every decoder warp waits on every packed stage and arrives on its empty barrier (16
-// arrivals), and the decoded ring's depth equals the number of groups, so each barrier's
-// phases are waited on strictly in order by each waiter (a parity wait cannot confuse a
-// phase with the one two phases earlier); the producer and the MMA issuer walk all rings in
-// order.
+// arrivals); each decoded stage is served by one group, which keeps one phase bit per stage
+// it serves, so each barrier's phases are waited on strictly in order by each waiter (a
+// parity wait cannot confuse a phase with the one two phases earlier); the producer and the
+// MMA issuer walk all rings in order.
 // Decode of one 32-bit word (16 codes): with a byte table TAB = {0, +1, -1, 0}, a byte
 // permute whose selector nibbles are the codes looks all of them up at once:
 //   even = prmt(TAB, sel = w & 0x33333333), odd = prmt(TAB, sel = (w >> 2) & 0x33333333)
@@ -47,9 +47,9 @@ constexpr int kPkDecGroups = 4;              // decoder groups of 4 warps
 constexpr int kPkThreads = 192 + kPkDecGroups * 128;
 constexpr int kPkBM = 128;                    // weight rows per tile (UMMA M)
 constexpr int kPkMaxBT = 256;                 // tokens per tile (UMMA N)
-constexpr int kPkDStages = kPkDecGroups;      // decoded ring depth (one stage per group)
-constexpr int kPkXStages = kPkDStages;       // activation ring depth: in step with the decoded
-                                              // ring, so one commit per k-block frees both
+constexpr int kPkMaxDStages = 2 * kPkDecGroups;   // decoded ring depth: 4 or 8 (one or two stages per group);
+                                                // the activation ring moves in step with it, so one
+                                                // commit per k-block frees both
 constexpr int kPkMaxPStages = 12;             // packed ring depth
 constexpr int kPkKbPerP = 4;                  // 128-code k-blocks per packed stage
 constexpr int kPkABytes = kPkBM * 128;        // decoded weight tile per stage (int8, SW128 K-major)
@@ -70,9 +70,9 @@ struct PkArgs {
     uint64_t wait_ns;
 };
 
-__host__ __device__ inline size_t pk_smem_bytes(int bt, int pstages) {
-    return 1024 + static_cast<size_t>(kPkDStages) * kPkABytes + static_cast<size_t>(kPkXStages) * bt * 128 +
-           static_cast<size_t>(pstages) * kPkPBytes + (2 * kPkMaxPStages + 3 * kPkDStages + 4) * sizeof(uint64_t) + 16;
+__host__ __device__ inline size_t pk_smem_bytes(int bt, int pstages, int dstages) {
+    return 1024 + static_cast<size_t>(dstages) * kPkABytes + static_cast<size_t>(dstages) * bt * 128 +
+           static_cast<size_t>(pstages) * kPkPBytes + (2 * kPkMaxPStages + 3 * kPkMaxDStages + 4) * sizeof(uint64_t) + 16;
 }
 
 // 16 codes of one packed word -> 16 int8 values (byte i = code i).
@@ -87,28 +87,29 @@ __device__ __forceinline__ uint4 pk_decode_word(uint32_t w) {
                       __byte_perm(e_hi, o_hi, 0x5140), __byte_perm(e_hi, o_hi, 0x7362));
 }
 
-template <bool kBf16Out>
+template <bool kBf16Out, int DS>
 __global__ void __launch_bounds__(kPkThreads, 1)
     tc_gemm_packed_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
                           const PkArgs args) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
-    constexpr int XS = kPkXStages;
+    static_assert(DS == kPkDecGroups || DS == 2 * kPkDecGroups, "decoded ring depth");
+    constexpr int XS = DS;
     const int PS = args.pstages;
     const int bt = args.bt;
     const uint32_t x_bytes = static_cast<uint32_t>(bt) * 128u;
     // [decoded A: 4 x 16 KB][packed: PS x 16 KB][activations: XS x bt x 128]; all 1024-aligned
     auto sA = [&](int d) { return smem + d * kPkABytes; };
-    uint8_t* sPbase = smem + kPkDStages * kPkABytes;
+    uint8_t* sPbase = smem + DS * kPkABytes;
     auto sP = [&](int p) { return sPbase + p * kPkPBytes; };
     uint8_t* sXbase = sPbase + PS * kPkPBytes;
     auto sX = [&](int x) { return sXbase + x * x_bytes; };
     uint64_t* pfull = reinterpret_cast<uint64_t*>(sXbase + XS * x_bytes);
     uint64_t* pempty = pfull + kPkMaxPStages;
     uint64_t* xfull = pempty + kPkMaxPStages;
-    uint64_t* dfull = xfull + kPkXStages;
-    uint64_t* dempty = dfull + kPkDStages;     // frees decoded stage d and activation stage d
-    uint64_t* tfull = dempty + kPkDStages;
+    uint64_t* dfull = xfull + XS;
+    uint64_t* dempty = dfull + DS;             // frees decoded stage d and activation stage d
+    uint64_t* tfull = dempty + DS;
     uint64_t* tempty = tfull + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(kPkThreads, 1)
         for (int x = 0; x < XS; ++x) {
             mbar_init(&xfull[x], 1);
         }
-        for (int d = 0; d < kPkDStages; ++d) {
+        for (int d = 0; d < DS; ++d) {
             mbar_init(&dfull[d], 4);     // the 4 decoder warps of the stage's group
             mbar_init(&dempty[d], 1);
         }
@@ -203,7 +204,8 @@ __global__ void __launch_bounds__(kPkThreads, 1)
         const int c = dt & 7;                      // word (16 codes) within a k-block's 32-byte row piece
         const int r0 = dt >> 3;                    // rows r0 + 16 i; r & 7 == r0 & 7 for all of them
         int p = 0;
-        uint32_t pph = 0, dph = 0;
+        uint32_t pph = 0;
+        uint32_t dph[DS / kPkDecGroups] = {};   // phase of each of the group's decoded stages
         int q = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -215,9 +217,11 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                 const int nkb = min(kPkKbPerP, kb1 - kb);
                 for (int j = 0; j < nkb; ++j, ++q) {
                     if ((q & (kPkDecGroups - 1)) != grp) continue;
-                    // the MMA has finished with this group's decoded stage (its previous use)
-                    if (!mbar_wait(&dempty[grp], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
-                    uint8_t* a = sA(grp);
+                    const int ds = q % DS;                      // grp, or grp + 4 on alternate turns
+                    const int li = ds / kPkDecGroups;
+                    // the MMA has finished with this decoded stage (its previous use)
+                    if (!mbar_wait(&dempty[ds], dph[li] ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    uint8_t* a = sA(ds);
                     // 16-byte chunk (2 j + c / 4) of row r sits at chunk (2 j + c / 4) ^ (r & 7)
                     const int src_off = ((((2 * j + (c >> 2)) ^ (r0 & 7)) << 4) | ((c & 3) << 2));
                     const int dst_off = (c ^ (r0 & 7)) << 4;
@@ -229,8 +233,8 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                     }
                     fence_proxy_async_shared();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&dfull[grp]);
-                    dph ^= 1u;
+                    if (lane == 0) mbar_arrive(&dfull[ds]);
+                    dph[li] ^= 1u;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pempty[p]);
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                                      umma_desc_sw128(x_base + kk * 32, 16, 1024), idesc,
                                      (kb != kb0 || kk != 0) ? 1u : 0u);
                     tc_commit(&dempty[d]);     // d == x: the rings move in step
-                    if (++d == kPkDStages) { d = 0; dph ^= 1u; }
+                    if (++d == DS) { d = 0; dph ^= 1u; }
                     if (++x == XS) { x = 0; xph ^= 1u; }
                 }
                 if (!ok) break;

@@ -70,10 +70,10 @@ __host__ __device__ inline size_t gemv_smem_bytes(int B, int K, int max_rgs) {
 // The activation rows reach shared memory by bulk copy (one bounded mbarrier wait) while
 // the first weight batch is already in flight, and are interleaved in place.
 // ------------------------------------------------------------------------------------
-template <int NTILES, int WB>
+template <int NTILES, int WB, bool kBf16Out = false>
 __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     const uint8_t* __restrict__ W, const float* __restrict__ gamma, int gamma_stride, int N, int K,
-    const int8_t* __restrict__ xq, const float* __restrict__ sx, int B, float* __restrict__ y,
+    const int8_t* __restrict__ xq, const float* __restrict__ sx, int B, void* __restrict__ y,
     int32_t* __restrict__ acc_out, uint64_t wait_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = smem_raw + ((16u - (smem_u32(smem_raw) & 15u)) & 15u);
@@ -247,7 +247,8 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
     __syncthreads();
 
     // y[b][n] = (acc - 2 sum x_b) * fl(gamma_n / s_b) for this block's rows, row-fastest
-    // (gamma_n = gamma[n * gamma_stride]: one scale, or one per weight row)
+    // (gamma_n = gamma[n * gamma_stride]: one scale, or one per weight row), stored as fp32
+    // or rounded to bf16
     const int rows = nrg * 16;
     for (int idx = threadIdx.x; idx < rows * B; idx += WB * 32) {
         const int b = idx / rows, r = idx - b * rows;
@@ -255,7 +256,11 @@ __global__ void __launch_bounds__(WB * 32, 1) ternary_gemv_kernel(
         const int n = rg0 * 16 + r;
         const int64_t o = static_cast<int64_t>(b) * N + n;
         const float gm = __ldg(gamma + static_cast<int64_t>(n) * gamma_stride);
-        y[o] = __fmul_rn(static_cast<float>(acc), __fdiv_rn(gm, __ldg(sx + b)));
+        const float yv = __fmul_rn(static_cast<float>(acc), __fdiv_rn(gm, __ldg(sx + b)));
+        if constexpr (kBf16Out)
+            static_cast<uint16_t*>(y)[o] = float_to_bf16_bits(yv);
+        else
+            static_cast<float*>(y)[o] = yv;
         if (acc_out != nullptr) acc_out[o] = acc;
     }
 }

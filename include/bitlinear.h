@@ -310,7 +310,9 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
  *   Y[t,n]   = fl32(acc[t,n] * fl32(gamma / sx[t]))     in y_dt
  * Xq int8 [T x K]; sx fp32 [T]; Wpacked uint8 [N x K/4]; gamma fp32 [1]; Y [T x N];
  * acc int32 [T x N] optional.  K % 64 == 0.  Meant for T up to a few hundred tokens
- * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).  When the
+ * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).  Up to 16
+ * tokens (when their activation rows fit one block's shared memory) the call runs the decode
+ * GEMV's kernel (codes decoded in registers, warp-level int8 MMA; ws unused).  When the
  * weight tiles alone cannot fill the GPU and at most 64 tokens are given, K may be split
  * across CTAs: split sp stores its exact int32 partial sums to slice sp of ws (int32
  * [splits x T x N]) and a second launch adds the slices in split order and applies the

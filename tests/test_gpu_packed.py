@@ -56,7 +56,7 @@ def _check(bl, xq, packed, s, gamma, out, split):
 
 @pytest.mark.parametrize("T,K,N", [(1, 64, 16), (7, 4096, 11008), (16, 8192, 28672), (64, 2048, 2048),
                                    (129, 1024, 400), (300, 512, 1040), (33, 192, 2064), (8, 2048, 400),
-                                   (3, 1024, 272)])
+                                   (3, 1024, 272), (32, 4096, 2048), (20, 1024, 400), (16, 65536, 64)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 @pytest.mark.parametrize("split", [False, True])
 def test_linear_packed_parity(bl, T, K, N, out, split):
