@@ -62,8 +62,9 @@ def parse():
     ap.add_argument("--only-packed", action="store_true",
                     help="run only the packed-weight linear at 16 tokens on the 28672 x 8192 weight (profiling)")
     ap.add_argument("--only-gemm", choices=["linear_i8", "grad_input", "grad_weight"], default=None,
-                    help="run three launches of one GEMM of the step on the gate projection's shape "
-                         "(16384 tokens, 4096 -> 11008; profiling)")
+                    help="run three launches of one GEMM of the step at 16384 tokens (profiling)")
+    ap.add_argument("--gemm-shape", choices=["q", "gate", "down"], default="gate",
+                    help="projection shape for --only-gemm: q 4096->4096, gate 4096->11008, down 11008->4096")
     ap.add_argument("--only-peak", action="store_true", help="run only the tensor-pipe peak probe")
     ap.add_argument("--next", action="store_true",
                     help="time the fused optimizer step and the quantiser variants back to back; one JSON object, "
@@ -339,7 +340,7 @@ def main():
             print(json.dumps({"tensor_peaks": probe_tensor_peaks(bl, torch, dev)}), flush=True)
             return
         if args.only_gemm:
-            print(json.dumps({"gemm": gemm_once(bl, torch, dev, args.only_gemm)}), flush=True)
+            print(json.dumps({"gemm": gemm_once(bl, torch, dev, args.only_gemm, args.gemm_shape)}), flush=True)
             return
         flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
         if args.only_mem:
@@ -859,10 +860,12 @@ def step_graph_ms(bl, torch, dev, flush, name, steps):
     return statistics.median(ms), T, layers
 
 
-def gemm_once(bl, torch, dev, which: str):
-    """Three launches of one GEMM of the step on the gate projection's shape (16384 tokens,
-    4096 -> 11008): a small case for a profiler capture (about 1 GB on the device)."""
-    T, K, N = 16384, 4096, 11008
+def gemm_once(bl, torch, dev, which: str, shape: str = "gate"):
+    """Three launches of one GEMM of the step on one projection's shape at 16384 tokens (q
+    4096 -> 4096, gate 4096 -> 11008, down 11008 -> 4096): a small case for a profiler capture
+    (at most about 1.5 GB on the device)."""
+    T = 16384
+    K, N = {"q": (4096, 4096), "gate": (4096, 11008), "down": (11008, 4096)}[shape]
     g = torch.Generator(device=dev).manual_seed(1)
     gamma = torch.full((1,), 0.02, device=dev)
     if which == "linear_i8":

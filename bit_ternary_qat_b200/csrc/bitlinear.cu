@@ -759,16 +759,15 @@ bl_status bitlinear_forward_qat(const void* X, bl_dtype x_dt, int64_t T, int64_t
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the |W| partial sums, the activation quantiser, then the ternary codes and the GEMM
-    // (a single launch for the first two measured no faster: the quantiser's occupancy
-    // limit throttled the partial-sum blocks)
+    // the |W| partial sums, the ternary codes (their second read of W follows the first
+    // directly, so it hits L2 when W fits there), the activation quantiser, then the GEMM
     const int64_t n = N * K;
     const int parts = bl::wq_num_partials(n);
     double* partials = static_cast<double*>(ws);
     pdl_launch(bl::absmean_partial_kernel, dim3(parts), dim3(bl::kWqThreads), 0, st, W, n, partials);
     BL_TRY(launched("absmean_partial"));
-    BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
     BL_TRY(run_ternary(W, n, partials, parts, Wq_i8, Wq_bf16, Wpacked, gamma, st, dev));
+    BL_TRY(run_act_quant(X, x_dt, T, K, 1, g, eps, Xq, sx, rinv, Xdq, st));
     return run_linear(Xq, sx, T, K, Wq_i8, gamma, N, Y, x_dt, acc, st, dev);
 }
 

@@ -353,6 +353,23 @@ __host__ __device__ constexpr size_t tc2_smem_bytes() {
     return 1024 + (size_t)kTc2Stages * 2 * kTc2HalfBytes + kEpiBytes + (2 * kTc2Stages + 4) * sizeof(uint64_t) + 16;
 }
 
+// Tile order of the 2-SM kernel (grouped raster): tiles are taken in groups of kTileGroupM
+// consecutive m-tiles; inside a group the m-tile varies fastest, then the n-tile.  The tiles
+// that run at the same time (one per cluster, consecutive indices) then cover a block about
+// kTileGroupM tall and (clusters / kTileGroupM) wide, so each operand panel they read is
+// shared by several of them and stays in L2 while the group moves along n, instead of every
+// wave touching almost every A panel once (m-fastest order).  The last group may be shorter.
+constexpr int kTileGroupM = 8;
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb) {
+    const int per_group = kTileGroupM * n_tiles;
+    const int grp = tile / per_group;
+    const int local = tile - grp * per_group;
+    const int m0 = grp * kTileGroupM;
+    const int gm = m_tiles - m0 < kTileGroupM ? m_tiles - m0 : kTileGroupM;
+    mb = m0 + local % gm;
+    nb = local / gm;
+}
+
 template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -421,8 +438,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             uint32_t ph = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-                const int mb = tile % args.m_tiles;
-                const int nb = tile / args.m_tiles;
+                int mb, nb;
+                tile_coords(tile, args.m_tiles, args.n_tiles, mb, nb);
                 const int arow = mb * 256 + static_cast<int>(rank) * 128;
                 const int brow = nb * kBN + static_cast<int>(rank) * 128;
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
@@ -508,8 +525,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             const uint32_t tph = (tcount >> 1) & 1;
             if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
-            const int mb = tile % args.m_tiles;
-            const int nb = tile / args.m_tiles;
+            int mb, nb;
+            tile_coords(tile, args.m_tiles, args.n_tiles, mb, nb);
             const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
             const int row = row0 + lane;
             const bool row_ok = row < args.M;

@@ -174,8 +174,8 @@ BL_API bl_status bitlinear_forward(const void* X, bl_dtype x_dt, int64_t T, int6
 /* ------------------------------------------------------------------------------
  * Quantisation-aware forward from the fp32 latent weight: what P3 §3.1's BitLinear.forward
  * computes (RMSNorm, activation_quant, weight_quant, then the linear), A1-A6 in one call:
- * the weight quantiser's fp64 partial sums of |W|, the activation quantiser, the ternary
- * codes, then the GEMM.
+ * the weight quantiser's fp64 partial sums of |W|, the ternary codes, the activation
+ * quantiser, then the GEMM.
  * Outputs: those of bitlinear_quant_weight (Wq_i8 required here -- the GEMM operand --,
  * Wq_bf16 and Wpacked optional, gamma) and of bitlinear_forward; all bit-identical to
  * bitlinear_quant_weight followed by bitlinear_forward.
