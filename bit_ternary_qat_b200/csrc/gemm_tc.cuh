@@ -370,6 +370,32 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
     nb = local / gm;
 }
 
+// Work units of the 2-SM kernel.  The tiles that would make up a last, partial wave -- when
+// there are at most half as many of them as clusters -- are each split into two 256 x 128
+// halves (N = 128 MMAs, half the time), so the tail takes half a wave instead of a whole one
+// while the other clusters idle.  Unit u < full_units is tile u; unit full_units + 2 j + h is
+// half h (output columns [128 h, 128 h + 128) of the tile) of tile full_units + j.
+struct Tc2Plan {
+    int full_units, num_units;
+};
+__device__ __forceinline__ Tc2Plan tc2_plan(int num_tiles, int npairs) {
+    const int tail = num_tiles % npairs;
+    const bool split = tail != 0 && 2 * tail <= npairs;
+    return Tc2Plan{split ? num_tiles - tail : num_tiles, split ? num_tiles + tail : num_tiles};
+}
+// unit -> tile coordinates and half (-1: the whole 256-column tile)
+__device__ __forceinline__ void tc2_unit(int u, const Tc2Plan& pl, int m_tiles, int n_tiles, int& mb, int& nb,
+                                         int& half) {
+    int tile = u;
+    half = -1;
+    if (u >= pl.full_units) {
+        const int v = u - pl.full_units;
+        tile = pl.full_units + (v >> 1);
+        half = v & 1;
+    }
+    tile_coords(tile, m_tiles, n_tiles, mb, nb);
+}
+
 template <bool kInt8, bool kAMN, bool kBMN, int kEpi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -430,6 +456,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     const int num_tiles = args.m_tiles * args.n_tiles;   // m_tiles counts 256-row pair tiles
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const uint64_t lim = args.wait_ns;
+    const Tc2Plan plan = tc2_plan(num_tiles, npairs);
+    constexpr uint32_t kIdescHalf = umma_idesc(kInt8, kAMN, kBMN, 256, kBN / 2);
 
     if (warp == 0) {
         // ----------------------------------------------------------------- producer (both CTAs)
@@ -437,11 +465,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-                int mb, nb;
-                tile_coords(tile, args.m_tiles, args.n_tiles, mb, nb);
+            for (int u = pair; u < plan.num_units && ok; u += npairs) {
+                int mb, nb, half;
+                tc2_unit(u, plan, args.m_tiles, args.n_tiles, mb, nb, half);
                 const int arow = mb * 256 + static_cast<int>(rank) * 128;
-                const int brow = nb * kBN + static_cast<int>(rank) * 128;
+                // CTA r supplies rows [128 r, 128 r + 128) of B for a whole tile, rows
+                // [128 h + 64 r, 128 h + 64 r + 64) of it for half h (the same boxes are
+                // loaded; the MMA reads their first 64 rows)
+                const int brow = half < 0 ? nb * kBN + static_cast<int>(rank) * 128
+                                          : nb * kBN + half * (kBN / 2) + static_cast<int>(rank) * 64;
                 for (int kb = 0; kb < args.k_blocks; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, lim, abort_flag)) { ok = false; break; }
                     if (leader) mbar_arrive_expect_tx(&full[s], kStageTxPair);
@@ -480,9 +512,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             uint32_t ph = 0;
             int tcount = 0;
             bool ok = true;
-            for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++tcount) {
+            for (int u = pair; u < plan.num_units && ok; u += npairs, ++tcount) {
                 const int b = tcount & 1;
                 const uint32_t tph = (tcount >> 1) & 1;
+                const uint32_t idesc = u < plan.full_units ? kIdesc : kIdescHalf;
                 if (!mbar_wait(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * kBN);
@@ -498,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
                         else adesc = umma_desc_sw128(a_base + kk * 2048, 8192, 1024);
                         if constexpr (!kBMN) bdesc = umma_desc_sw128(b_base + kk * 32, 16, 1024);
                         else bdesc = umma_desc_sw128(b_base + kk * 2048, 8192, 1024);
-                        tc_mma_pair<kInt8>(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_pair<kInt8>(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit_pair(&empty[s], 0x3);
                     if (++s == kTc2Stages) { s = 0; ph ^= 1u; }
@@ -520,13 +553,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         int tcount = 0;
         float gm = 1.0f;
         if constexpr (kEpi != kEpiF32 && !epi_is_col(kEpi)) gm = __ldg(args.gamma);
-        for (int tile = pair; tile < num_tiles; tile += npairs, ++tcount) {
+        for (int u = pair; u < plan.num_units; u += npairs, ++tcount) {
             const int b = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
             if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
-            int mb, nb;
-            tile_coords(tile, args.m_tiles, args.n_tiles, mb, nb);
+            int mb, nb, half;
+            tc2_unit(u, plan, args.m_tiles, args.n_tiles, mb, nb, half);
+            const int ucols = half < 0 ? kBN : kBN / 2;             // accumulator columns of the unit
+            const int col_base = nb * kBN + (half < 0 ? 0 : half * (kBN / 2));
             const int row0 = mb * 256 + static_cast<int>(rank) * 128 + quad * 32;
             const int row = row0 + lane;
             const bool row_ok = row < args.M;
@@ -540,8 +575,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(b * kBN);
 #pragma unroll 1
-            for (int c0 = 0; c0 < kBN; c0 += kChunkCols) {
-                const int col0 = nb * kBN + c0;
+            for (int c0 = 0; c0 < ucols; c0 += kChunkCols) {
+                const int col0 = col_base + c0;
                 if (col0 >= args.N) break;                     // warp-uniform
                 uint32_t ra[32], rb[32];
                 __syncwarp();

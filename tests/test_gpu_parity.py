@@ -212,6 +212,8 @@ def test_single_workload_seed0(bl):
 
 @pytest.mark.parametrize("T,K,N,dtype,gain", [
     (64, 256, 512, "f32", False),        # the single-layer fp32 shape on another seed
+    (3800, 1280, 3840, "bf16", False),   # 225 / 75 / 75 pair tiles: the 2-SM GEMMs' last partial
+                                         # wave runs as half tiles (ragged rows and columns too)
     (300, 160, 400, "bf16", True),
     (257, 512, 144, "f32", True),
     (130, 1024, 784, "bf16", False),
