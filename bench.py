@@ -579,15 +579,44 @@ def main():
         h2d = sum(h["W"].numel() * 4 + h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host)
         d2h = sum(d.numel() * 4 for d in dW_h) + 4 * len(layers)
 
+        # Copies run on their own streams so that PCIe traffic overlaps the compute: every
+        # projection's inputs go host -> device on one stream (each projection has its own
+        # device buffers), a projection's compute waits only for its own inputs, and its dW goes
+        # device -> host on a third stream as soon as it is final (PCIe is full duplex).
+        # gamma is copied to a per-projection device slot on the compute stream before the next
+        # projection overwrites it, and read back with the gradients.
+        h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        g_dev = torch.empty(len(layers), dtype=f32, device=dev)
+
         def e2e_step():
-            for li, (L, h) in enumerate(zip(layers, host)):
-                L["W"].copy_(h["W"], non_blocking=True)
-                L["X"].copy_(h["X"], non_blocking=True)
-                L["dY"].copy_(h["dY"], non_blocking=True)
+            main = torch.cuda.current_stream(dev)
+            start = torch.cuda.Event()
+            start.record(main)
+            h2d_s.wait_event(start)
+            d2h_s.wait_event(start)
+            ready = []
+            with torch.cuda.stream(h2d_s):
+                for L, h in zip(layers, host):
+                    L["W"].copy_(h["W"], non_blocking=True)
+                    L["X"].copy_(h["X"], non_blocking=True)
+                    L["dY"].copy_(h["dY"], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(h2d_s)
+                    ready.append(e)
+            for li, L in enumerate(layers):
+                main.wait_event(ready[li])
                 layer_step(L)
-                g_h[li:li + 1].copy_(L["fo"]["gamma"], non_blocking=True)
+                g_dev[li:li + 1].copy_(L["fo"]["gamma"])
                 dp.allreduce_weight_grad(L["dW"])
-                dW_h[li].copy_(L["dW"], non_blocking=True)
+                done = torch.cuda.Event()
+                done.record(main)
+                d2h_s.wait_event(done)
+                with torch.cuda.stream(d2h_s):
+                    dW_h[li].copy_(L["dW"], non_blocking=True)
+            d2h_s.wait_stream(main)
+            with torch.cuda.stream(d2h_s):
+                g_h.copy_(g_dev, non_blocking=True)
+            main.wait_stream(d2h_s)
 
         e2e_step()
         sync_all()
@@ -604,8 +633,10 @@ def main():
             dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         e2e = {"value": T * world * ke / (float(e2e_ms.item()) * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": ke,
-               "how": "per projection: pinned host -> device copies of W, X, dY, the eager library calls of the "
-                      "step, device -> host copies of dW and gamma; CUDA events around each step"}
+               "how": "pinned host -> device copies of every projection's W, X, dY on a copy stream, each "
+                      "projection's eager library calls as soon as its inputs have landed, device -> host copies "
+                      "of its dW on a second copy stream as soon as it is final, gamma read back at the end; "
+                      "CUDA events around each step on the compute stream, which joins both copy streams"}
         del host, dW_h
 
     if world > 1:
