@@ -407,29 +407,30 @@ def main():
     ovs = torch.cuda.Stream(device=dev)
 
     # One projection's step.  The forward is one call (bitlinear_forward_qat: the weight
-    # quantiser's |W| sums, the activation quantiser, the ternary codes, the int8 GEMM); after
+    # quantiser's |W| sums, the ternary codes, the activation quantiser, the int8 GEMM); after
     # the grad-input GEMM the RMSNorm backward and the decode GEMV go to a second stream and
-    # run beside the weight-gradient GEMM.  `dom` brackets one GEMM with two events.
+    # run beside the weight-gradient GEMM.  `dom` maps a GEMM's name to the two events that
+    # bracket it.
     def layer_step(L, dom=None, inputs=None):
         fo = L["fo"]
         Wi, Xi, dYi = inputs if inputs is not None else (L["W"], L["X"], L["dY"])
         main = torch.cuda.current_stream(dev)
         bl.bitlinear_forward_qat(Xi, Wi, ws=ws, out=fo)
-        if dom is not None and dom[0] == "grad_input":
-            dom[1].record()
+        if dom is not None and "grad_input" in dom:
+            dom["grad_input"][0].record()
         bl.bitlinear_grad_input(dYi, fo["wq_bf16"], fo["gamma"], dXhat=L["dX"])
-        if dom is not None and dom[0] == "grad_input":
-            dom[2].record()
+        if dom is not None and "grad_input" in dom:
+            dom["grad_input"][1].record()
         ovs.wait_stream(main)
         with torch.cuda.stream(ovs):
             bl.bitlinear_rmsnorm_backward(Xi, fo["rinv"], L["dX"], ws=ws, dg=L["dg"])
             bl.ternary_gemv(fo["packed"], fo["gamma"], L["K"], fo["xq"][:DECODE_B], fo["sx"][:DECODE_B],
                             y=L["ydec"])
-        if dom is not None and dom[0] == "grad_weight":
-            dom[1].record()
+        if dom is not None and "grad_weight" in dom:
+            dom["grad_weight"][0].record()
         bl.bitlinear_backward_weight(dYi, fo["xdq"], dW=L["dW"])
-        if dom is not None and dom[0] == "grad_weight":
-            dom[2].record()
+        if dom is not None and "grad_weight" in dom:
+            dom["grad_weight"][1].record()
         main.wait_stream(ovs)
 
     # The same work as separate sequential calls with an event before each (piece times).
@@ -549,24 +550,30 @@ def main():
     # ---------------------------------------------------------------- dominant kernel, live in the step
     ops_gemm = [2.0 * T * L["N"] * L["K"] for L in layers]
     dom = max(("grad_input", "grad_weight"), key=lambda p: sum(piece_ms[p]))
-    dev_ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-              for _ in layers]
+    # both backward GEMMs bracketed in the same replays: the dominant one gives the roofline,
+    # the other is reported beside it
+    gemm_names = ("grad_input", "grad_weight")
+    dev_ev = [{nm: (torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for nm in gemm_names} for _ in layers]
     g_dom = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(device=dev)
     side.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.graph(g_dom):
-        for L, (e0, e1) in zip(layers, dev_ev):
-            layer_step(L, dom=(dom, e0, e1))
+        for L, evs in zip(layers, dev_ev):
+            layer_step(L, dom=evs)
     g_dom.replay()
     torch.cuda.synchronize()
-    dom_ms = [[] for _ in layers]
+    inst_ms = {nm: [[] for _ in layers] for nm in gemm_names}
     for i in range(K):
         flush.zero_()
         g_dom.replay()
         torch.cuda.synchronize()
-        for li, (e0, e1) in enumerate(dev_ev):
-            dom_ms[li].append(e0.elapsed_time(e1))
+        for li, evs in enumerate(dev_ev):
+            for nm in gemm_names:
+                inst_ms[nm][li].append(evs[nm][0].elapsed_time(evs[nm][1]))
+    dom_ms = inst_ms[dom]
     dom_layer_ms = [statistics.mean(v) for v in dom_ms]
+    in_step = {nm: sum(statistics.mean(v) for v in inst_ms[nm]) for nm in gemm_names}
     assert bl.check_device_status() == 0
     del graphs, g_pc, g_dom
 
@@ -661,9 +668,13 @@ def main():
                 "flop_per_launch": sum(ops_gemm) / len(layers),
                 "per_layer_ms": {L["name"]: round(v, 5) for L, v in zip(layers, dom_layer_ms)},
                 "frac_of_probe_bf16": achieved / tpk["bf16"],
+                "in_step": {nm: {"ms_per_step": in_step[nm],
+                                 "achieved": sum(ops_gemm) / (in_step[nm] * 1e-3) / 1e12,
+                                 "frac": sum(ops_gemm) / (in_step[nm] * 1e-3) / 1e12 / bf16_peak}
+                            for nm in gemm_names},
                 "how": "two event nodes around this GEMM of every projection inside K further replays of the "
-                       "timed step's graph (L2 flushed before each); achieved = its FLOPs / its time, summed "
-                       "over the projections"}
+                       "timed step's graph (L2 flushed before each; the grad-input GEMM is bracketed in the same "
+                       "replays, `in_step`); achieved = its FLOPs / its time, summed over the projections"}
 
     # every kernel of the step against its roofline (sequential piece times)
     def bytes_of(p, L):
