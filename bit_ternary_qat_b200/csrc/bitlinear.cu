@@ -24,6 +24,7 @@
 #include "gemv.cuh"
 #include "optim.cuh"
 #include "gemm_packed.cuh"
+#include "gemm_packed2.cuh"
 #include "mma_peak.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
@@ -168,7 +169,7 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-enum TmType { kTmU8 = 0, kTmBf16 = 1, kTmF32 = 2 };
+enum TmType { kTmU8 = 0, kTmBf16 = 1, kTmF32 = 2, kTmI32 = 3 };
 
 // 2-D row-major tensor [outer x inner] with 128-byte swizzled boxes [box_outer x box_inner]
 // (box_inner * element size == 128 bytes).
@@ -177,8 +178,10 @@ bl_status make_tmap(CUtensorMap* tm, const void* base, TmType t, uint64_t inner,
     EncodeTiledFn fn = encode_fn();
     BL_REQUIRE(fn != nullptr, BL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const uint64_t esize = t == kTmU8 ? 1 : (t == kTmBf16 ? 2 : 4);
-    const CUtensorMapDataType dt = t == kTmU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                   : (t == kTmBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+    const CUtensorMapDataType dt = t == kTmU8    ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : t == kTmBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : t == kTmI32  ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {inner * esize};
     cuuint32_t box[2] = {box_inner, box_outer};
@@ -186,6 +189,23 @@ bl_status make_tmap(CUtensorMap* tm, const void* base, TmType t, uint64_t inner,
     CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    BL_REQUIRE(r == CUDA_SUCCESS, BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return BL_OK;
+}
+
+// 3-D map over int32 slices [outer][middle][inner] (no swizzle): the K-split partial sums,
+// one box of box_inner x box_middle elements in one slice.
+bl_status make_tmap3_i32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t middle, uint64_t outer,
+                         uint32_t box_inner, uint32_t box_middle) {
+    EncodeTiledFn fn = encode_fn();
+    BL_REQUIRE(fn != nullptr, BL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {inner, middle, outer};
+    cuuint64_t strides[2] = {inner * 4, inner * middle * 4};
+    cuuint32_t box[3] = {box_inner, box_middle, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_INT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     BL_REQUIRE(r == CUDA_SUCCESS, BL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return BL_OK;
 }
@@ -577,6 +597,94 @@ bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
     const unsigned grid = (unsigned)std::min<int64_t>(units, dev.sms);
     pdl_launch(kern, dim3(grid), dim3(bl::kPkThreads), smem, st, tp, tx, a);
     BL_TRY(launched("tc_gemm_packed"));
+    if (splits > 1) {
+        const int64_t nv = T * N / 4;
+        pdl_launch(bl::pk_finalize_kernel<kBf16Out>, dim3((unsigned)std::min<int64_t>((nv + 255) / 256, (int64_t)dev.sms * 8)),
+                   dim3(256), 0, st, static_cast<const int32_t*>(scratch), splits, sx, gamma, (int)T, (int)N, Y, acc);
+        BL_TRY(launched("pk_finalize"));
+    }
+    return BL_OK;
+}
+
+// Packed-weight GEMM on CTA pairs (17 or more tokens): 256-row weight tiles x bt tokens
+// (bt = T rounded up to 32, at most 256), the same K-split rule as the 1-SM kernel counted
+// in pairs, the activation ring, and the packed ring in the rest of shared memory.  The grid
+// is as many pairs as fit at once, at most one per unit.
+template <bool kBf16Out>
+bl_status launch_packed2(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
+                         const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch,
+                         size_t scratch_bytes, cudaStream_t st, const DeviceInfo& dev) {
+    bl::Pk2Args a2{};
+    bl::PkArgs& a = a2.pk;
+    a.T = (int)T; a.N = (int)N; a.K = (int)K;
+    int64_t bt = (T + 31) / 32 * 32;
+    if (bt > bl::kPkMaxBT) bt = bl::kPkMaxBT;
+    a.bt = (int)bt;
+    a.t_tiles = (int)((T + bt - 1) / bt);
+    a.n_tiles = (int)((N + 2 * bl::kPk2Rows - 1) / (2 * bl::kPk2Rows));
+    a.k_blocks = (int)((K + 127) / 128);
+    // activation stages of two k-blocks: at least 64 KB and at least as many as the decoded
+    // stages (the leader's decoders wait on an activation stage by its parity)
+    const int xstages = (int)std::min<int64_t>(bl::kPk2MaxXStages,
+                                               std::max<int64_t>(bl::kPk2DStages, 65536 / (bt * 128)));
+    a2.xstages = xstages;
+    const size_t budget = (size_t)dev.max_smem_optin;
+    int pstages = (int)((budget - bl::pk2_smem_bytes((int)bt, 0, xstages)) / bl::kPkPBytes);
+    pstages = std::min(pstages, bl::kPkMaxPStages);
+    BL_REQUIRE(pstages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
+    a.pstages = pstages;
+    auto kern = bl::tc_gemm_packed2_kernel<kBf16Out>;
+    const size_t smem = bl::pk2_smem_bytes((int)bt, pstages, xstages);
+    // pairs resident at once, per device and token-tile width (the shared memory differs)
+    static std::atomic<int> max_clusters[64][bl::kPkMaxBT / 32] = {};
+    int dev_id = 0;
+    cudaGetDevice(&dev_id);
+    if (dev_id < 0 || dev_id >= 64) return fail(BL_ERR_DEVICE, "device ordinal %d out of range", dev_id);
+    std::atomic<int>& mc_slot = max_clusters[dev_id][bt / 32 - 1];
+    int mc = mc_slot.load();
+    if (mc == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)(dev.sms / 2));
+        cfg.blockDim = dim3(bl::kPk2Threads);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaOccupancyMaxActiveClusters: %s", cudaGetErrorString(e));
+        if (n < 1) return fail(BL_ERR_DEVICE, "no 2-CTA cluster of the packed GEMM fits on the device");
+        mc = n;
+        mc_slot.store(mc);
+    }
+    const int64_t base = (int64_t)a.n_tiles * a.t_tiles;
+    int splits = 1;
+    if (bt <= 64) {
+        int smax = std::min<int64_t>(8, a.k_blocks / 2);
+        smax = (int)std::min<int64_t>(smax, K / (64 * T));
+        smax = (int)std::min<int64_t>(smax, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));
+        double best = wave_eff(base, mc);
+        for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, mc));
+        for (int sp = 1; sp <= std::max(1, smax); ++sp)
+            if (wave_eff(base * sp, mc) >= best - 0.03) { splits = sp; break; }
+    }
+    a.splits = splits;
+    a.sx = sx; a.gamma = gamma; a.y = Y;
+    a.acc = splits > 1 ? scratch : acc;
+    a.wait_ns = g_wait_ns.load();
+    CUtensorMap tp, tx, ty, tacc;
+    BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, bl::kPk2Rows));
+    BL_TRY(make_tmap(&tx, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, (uint32_t)(bt / 2)));
+    // the epilogue's TMA stores: 32 rows x 32 tokens per box, no swizzle
+    BL_TRY(make_tmap(&ty, Y, kBf16Out ? kTmBf16 : kTmF32, (uint64_t)N, (uint64_t)T, 32, 32, false));
+    std::memset(&tacc, 0, sizeof(tacc));
+    if (splits > 1)
+        BL_TRY(make_tmap3_i32(&tacc, scratch, (uint64_t)N, (uint64_t)T, (uint64_t)splits, 32, 32));
+    else if (acc != nullptr)
+        BL_TRY(make_tmap(&tacc, acc, kTmI32, (uint64_t)N, (uint64_t)T, 32, 32, false));
+    const int64_t units = base * splits;
+    const unsigned clusters = (unsigned)std::min<int64_t>(units, mc);
+    pdl_launch(kern, dim3(2 * clusters), dim3(bl::kPk2Threads), smem, st, tp, tx, ty, tacc, a2);
+    BL_TRY(launched("tc_gemm_packed2"));
     if (splits > 1) {
         const int64_t nv = T * N / 4;
         pdl_launch(bl::pk_finalize_kernel<kBf16Out>, dim3((unsigned)std::min<int64_t>((nv + 255) / 256, (int64_t)dev.sms * 8)),
@@ -1098,6 +1206,13 @@ bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, 
             return T <= 8 ? launch_gemv<1, false>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev)
                           : launch_gemv<2, false>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev);
         }
+    }
+    // 17 tokens or more: 2-SM tiles of 256 weight rows (M = 256 MMAs move about 1.6x more
+    // weight codes per SM per cycle than 1-SM tiles at these widths)
+    if (T > 16) {
+        if (y_dt == BL_BF16)
+            return launch_packed2<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
+        return launch_packed2<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
     }
     if (y_dt == BL_BF16)
         return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);

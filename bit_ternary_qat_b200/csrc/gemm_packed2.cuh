@@ -1,0 +1,479 @@
+// gemm_packed2.cuh -- int8 x packed-ternary linear on CTA pairs (tcgen05.mma.cta_group::2 with
+// the weight operand in tensor memory) for 17 or more tokens.
+//
+// The same contraction as gemm_packed.cuh (P3 §3.1's linear on P5 §4.1 / §5.1 2-bit codes):
+//   D[n, t] = sum_k W_q[n, k] x_q[t, k],   y[t, n] = fl(D * fl(gamma / s_t)),
+// with the weight rows as the MMA's M dimension.  A cluster of two CTAs computes a tile of 256
+// weight rows x bt tokens (bt = 32 ... 256) with one 2-SM instruction per 32 codes of K.
+//
+// The decoded weight never touches shared memory: each decoder thread owns one weight row,
+// decodes the row's 128 codes of a k-block in registers and writes them with tcgen05.st into
+// its CTA's tensor memory (lane = row, 4 codes per 32-bit column), where the MMA reads its A
+// operand.  Staging the decoded int8 tile in shared memory instead cost 1 byte written by the
+// decoders and 1 byte read by the tensor core per code, on top of the packed and activation
+// tiles; measured on B200, the decoders then ran at a fraction of their issue rate while the
+// MMAs streamed, and the kernel was slower than the int8-code GEMM from 32 tokens up.
+//
+// Per CTA r of a pair (rows [256 u + 128 r, +128) of weight tile u), 736 threads.  A "stage"
+// of the activation and decoded-weight rings is two k-blocks (256 codes of K); a packed stage
+// is four k-blocks.
+//   warp 0     packed producer: TMA loads of the CTA's 128 rows' packed codes (512 codes per
+//              row per stage, 128-byte swizzle) into its packed ring (its own barriers);
+//   warp 22    activation producer: TMA loads of the CTA's half of the token tile (bt / 2 rows x
+//              128 bytes per k-block) with the 2-SM TMA form, whose completion bytes count on the
+//              leader's barrier;
+//   warps 6-21 decoders, four groups of four warps (one per TMEM lane quarter): group g decodes
+//              the stages q = g mod 4 into its TMEM stage (64 columns): each thread owns one
+//              weight row, decodes the row's codes in registers and writes them with tcgen05.st;
+//              then tcgen05.wait::st, fence, and one arrival per warp on the LEADER's barrier of
+//              that stage (8 arrivals: the group in both CTAs).  The leader's warps first wait
+//              for the stage's activation tile, so the MMA issuer waits on one barrier;
+//   warp 1     leader only: one thread issues tcgen05.mma.cta_group::2.kind::i8 (eight per stage)
+//              with A from both CTAs' TMEM stage and B from both CTAs' activation halves; its
+//              commits arrive on both CTAs' stage-empty and activation-empty barriers, and after a
+//              unit's last stage on both CTAs' accumulator-full barriers;
+//   warps 2-5  epilogue (both CTAs): TMEM lanes are the CTA's 128 weight rows; the unit's token
+//              factors fl(gamma / s_t) are read before its accumulators are ready; per 32-token
+//              chunk tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (coalesced along n), or
+//              the exact int32 partial sums of K split sp into slice sp of a workspace
+//              (pk_finalize_kernel adds them in split order); one arrival per warp on the
+//              leader's accumulator-empty barrier.
+// The single-thread MMA loop's waits and commits cost about as much as the MMAs themselves at
+// these widths (measured); two k-blocks per stage halve them per MMA.
+// TMEM (512 columns per CTA): accumulators in columns [0, 256) -- two 128-column buffers when
+// bt <= 128 (a unit's epilogue overlaps the next unit's k-loop), one 256-column buffer
+// otherwise -- and the decoded-weight ring (4 stages x 64 columns) in [256, 512).  Work units
+// (weight tile, token tile, K split) are taken persistently, pair index + j * pairs.  Every wait
+// is bounded; on a timeout each role unwinds as in the 2-SM GEMM.  No TMA load uses multicast.
+#pragma once
+#include "common.cuh"
+#include "gemm_packed.cuh"
+
+namespace bl {
+
+constexpr int kPk2Rows = 128;          // weight rows per CTA (a pair tile: 256)
+constexpr int kPk2Threads = kPkThreads + 32;   // + the activation producer warp
+constexpr int kPk2MaxXStages = 16;     // activation ring depth (stages of 2 x bt / 2 x 128 bytes)
+constexpr int kPk2DStages = 4;         // decoded-weight stages in TMEM (one per decoder group)
+constexpr int kPk2KbPerStage = 2;      // k-blocks per activation / decoded stage
+constexpr uint32_t kPk2ACol = 256;     // first TMEM column of the decoded-weight ring
+constexpr uint32_t kPk2StageCols = 64; // 256 int8 codes per row = 64 columns
+
+constexpr uint32_t kPk2EpiBuf = 32 * 32 * 4;   // one 32-token x 32-row tile of 4-byte values
+constexpr uint32_t kPk2EpiBytes = 4 * 2 * kPk2EpiBuf;   // two staging tiles per epilogue warp
+
+__host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages, int xstages) {
+    return 1024 + static_cast<size_t>(pstages) * kPkPBytes + static_cast<size_t>(xstages) * static_cast<size_t>(bt) * 128 +
+           kPk2EpiBytes +
+           (2 * kPkMaxPStages + 2 * kPk2MaxXStages + 2 * kPk2DStages + 4) * sizeof(uint64_t) + 16;
+}
+
+// Bounded parity wait with cluster-scope acquire, for barriers that the other CTA of the pair
+// arrives on after writing its tensor memory or reading its accumulators.
+__device__ __forceinline__ bool pk2_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "n"(kWaitHintNs)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool pk2_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                 volatile int* abort) {
+    const uint32_t a = smem_u32(bar);
+    if (pk2_try_wait_cluster(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (pk2_try_wait_cluster(a, parity)) return true;
+        if ((i & 7u) == 0u) {
+            if (abort != nullptr && *abort) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                record_status(6 /* BL_ERR_TIMEOUT */);
+                if (abort != nullptr) *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Arrive on a barrier of either CTA of the pair (address in the cluster window) with the
+// default release at CTA scope.  The data the arrival publishes is ordered by tcgen05 fences
+// (decoded weights in TMEM, accumulators read from TMEM), not by this arrival.  Measured on
+// B200, an arrival with release at cluster scope cost 800-2500 cycles, on the path of every
+// k-block.
+__device__ __forceinline__ void pk2_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 32 consecutive TMEM columns of this warp's 32 lanes from 32 registers per thread.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// TMA store (shared -> global) of one 3-D box; completion tracked with bulk groups.
+__device__ __forceinline__ void tma_store_3d(const void* desc, const void* smem_src, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(desc)),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T on the CTA pair (A: each CTA's 128 rows in its own TMEM).
+__device__ __forceinline__ void tc_mma_pair_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "setp.ne.b32 P, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, P;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+struct Pk2Args {
+    PkArgs pk;        // shapes, outputs, pstages; pk.bt is the pair tile's token count
+    int xstages;      // activation ring depth
+};
+
+template <bool kBf16Out>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
+    tc_gemm_packed2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
+                           const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmAcc,
+                           const Pk2Args a2) {
+    const PkArgs& args = a2.pk;
+    constexpr int DS = kPk2DStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_align1024(smem_raw);
+    const int PS = args.pstages;
+    const int XS = a2.xstages;
+    const int bt = args.bt;                                            // multiple of 32
+    const int nacc = bt <= 128 ? 2 : 1;                                // accumulator buffers
+    const uint32_t xh_bytes = static_cast<uint32_t>(bt) * 64u;         // one k-block: bt / 2 rows x 128 bytes
+    // [packed: PS x 16 KB][activation halves: XS x 2 k-blocks x xh_bytes][epilogue staging]; 1024-aligned
+    auto sP = [&](int p) { return smem + p * kPkPBytes; };
+    uint8_t* sXbase = smem + PS * kPkPBytes;
+    auto sX = [&](int x) { return sXbase + static_cast<uint32_t>(x) * (kPk2KbPerStage * xh_bytes); };
+    uint8_t* sE = sXbase + static_cast<uint32_t>(XS) * (kPk2KbPerStage * xh_bytes);
+    uint64_t* pfull = reinterpret_cast<uint64_t*>(sE + kPk2EpiBytes);
+    uint64_t* pempty = pfull + kPkMaxPStages;    // this CTA's 16 decoder warps
+    uint64_t* xfull = pempty + kPkMaxPStages;    // leader's is used: both CTAs' activation bytes
+    uint64_t* xempty = xfull + kPk2MaxXStages;   // each CTA: the leader's commit
+    uint64_t* dfull = xempty + kPk2MaxXStages;   // leader's is used: the stage's group in both CTAs
+    uint64_t* dempty = dfull + DS;               // each CTA: the leader's commit
+    uint64_t* tfull = dempty + DS;               // each CTA: the leader's commit after a unit
+    uint64_t* tempty = tfull + 2;                // leader's is used: 4 epilogue warps per CTA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    if (threadIdx.x == 0) {
+        for (int p = 0; p < PS; ++p) {
+            mbar_init(&pfull[p], 1);
+            mbar_init(&pempty[p], 4 * kPkDecGroups);
+        }
+        for (int x = 0; x < XS; ++x) {
+            mbar_init(&xfull[x], 1);
+            mbar_init(&xempty[x], 1);
+        }
+        for (int d = 0; d < DS; ++d) {
+            mbar_init(&dfull[d], 8);
+            mbar_init(&dempty[d], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmP);
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger_and_wait();
+
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int units = args.n_tiles * args.t_tiles * args.splits;
+    const uint64_t lim = args.wait_ns;
+    // unit u -> (pair weight tile nt, token tile tt, K split sp) and its k-block range
+    auto unit_of = [&](int u, int& nt, int& tt, int& kb0, int& kb1) {
+        const int sp = u % args.splits;
+        const int rest = u / args.splits;
+        tt = rest % args.t_tiles;
+        nt = rest / args.t_tiles;
+        kb0 = static_cast<int>(static_cast<int64_t>(sp) * args.k_blocks / args.splits);
+        kb1 = static_cast<int>(static_cast<int64_t>(sp + 1) * args.k_blocks / args.splits);
+    };
+    // a bounded wait for the loads issued last, before the pair exits after a timeout
+    auto drain = [&](uint64_t* full, int n_stages, int next, uint32_t ph, int issued) {
+        for (int i = 0; i < n_stages && i < issued; ++i) {
+            const int s = (next - 1 - i + 2 * n_stages) % n_stages;
+            mbar_wait(&full[s], (next - 1 - i < 0) ? (ph ^ 1u) : ph, 100000000ull, nullptr);
+        }
+    };
+    if (warp == 0) {
+        // ----------------------------------------------------------------- packed producer (both CTAs)
+        if (elect_one()) {
+            int p = 0, issued = 0;
+            uint32_t pph = 0;
+            bool ok = true;
+            for (int u = pair; u < units && ok; u += npairs) {
+                int nt, tt, kb0, kb1;
+                unit_of(u, nt, tt, kb0, kb1);
+                const int prow = nt * 2 * kPk2Rows + static_cast<int>(rank) * kPk2Rows;
+                for (int kb = kb0; kb < kb1; kb += kPkKbPerP) {
+                    // the CTA's next packed stage: k-blocks kb .. kb + 3 of its 128 rows
+                    if (!mbar_wait(&pempty[p], pph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&pfull[p], static_cast<uint32_t>(kPkPBytes));
+                    tma_load_2d(sP(p), &tmP, &pfull[p], kb * 32, prow);
+                    ++issued;
+                    if (++p == PS) { p = 0; pph ^= 1u; }
+                }
+            }
+            if (!ok) drain(pfull, PS, p, pph, issued);
+        }
+        __syncwarp();
+    } else if (warp == kPk2Threads / 32 - 1) {
+        // ----------------------------------------------------------------- activation producer (both CTAs)
+        if (elect_one()) {
+            int x = 0, issued = 0;
+            uint32_t xph = 0;
+            bool ok = true;
+            for (int u = pair; u < units && ok; u += npairs) {
+                int nt, tt, kb0, kb1;
+                unit_of(u, nt, tt, kb0, kb1);
+                const int trow = tt * bt + static_cast<int>(rank) * (bt / 2);
+                for (int kb = kb0; kb < kb1; kb += kPk2KbPerStage) {
+                    const int nkb = min(kPk2KbPerStage, kb1 - kb);
+                    if (!mbar_wait(&xempty[x], xph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&xfull[x], 2u * static_cast<uint32_t>(nkb) * xh_bytes);
+                    const uint32_t bar = mapa_shared(smem_u32(&xfull[x]), 0);
+                    for (int j = 0; j < nkb; ++j)
+                        tma_load_2d_pair(sX(x) + j * xh_bytes, &tmX, bar, (kb + j) * 128, trow);
+                    ++issued;
+                    if (++x == XS) { x = 0; xph ^= 1u; }
+                }
+            }
+            // the leader's barriers count both CTAs' bytes
+            if (!ok && leader) drain(xfull, XS, x, xph, issued);
+        }
+        __syncwarp();
+    } else if (warp >= 6) {
+        // ----------------------------------------------------------------- decoders (both CTAs)
+        const int grp = (warp - 6) >> 2;                // decodes stage sequence numbers q = grp mod 4
+        const int row = 32 * (warp & 3) + lane;         // this thread's weight row = its TMEM lane
+        const int sw = row & 7;                         // 128-byte swizzle of the packed row
+        const uint32_t t_st = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + kPk2ACol +
+                              static_cast<uint32_t>(grp) * kPk2StageCols;
+        const uint32_t dfull_leader = mapa_shared(smem_u32(&dfull[grp]), 0);
+        int p = 0;
+        uint32_t pph = 0, dph = 0;
+        int q = 0;                                      // stage sequence number
+        bool ok = true;
+        for (int u = pair; u < units && ok; u += npairs) {
+            int nt, tt, kb0, kb1;
+            unit_of(u, nt, tt, kb0, kb1);
+            for (int kb = kb0; kb < kb1 && ok; kb += kPkKbPerP) {
+                if (!mbar_wait(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
+                const uint8_t* src = sP(p) + row * 128;
+                for (int h = 0; h < kPkKbPerP / kPk2KbPerStage; ++h) {
+                    const int ks = kb + h * kPk2KbPerStage;
+                    if (ks >= kb1) break;
+                    if ((q & (kPkDecGroups - 1)) == grp) {
+                        const int nkb = min(kPk2KbPerStage, kb1 - ks);
+                        // the MMA has finished reading this stage in both CTAs (its previous use)
+                        if (!mbar_wait(&dempty[grp], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int j = 0; j < nkb; ++j) {
+                            // k-block 2 h + j of the packed stage: the row's 16-byte chunks 2 jj, 2 jj + 1
+                            const int jj = h * kPk2KbPerStage + j;
+                            const uint4 w0 = *reinterpret_cast<const uint4*>(src + (((2 * jj) ^ sw) << 4));
+                            const uint4 w1 = *reinterpret_cast<const uint4*>(src + (((2 * jj + 1) ^ sw) << 4));
+                            const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                            uint32_t v[32];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const uint4 d = pk_decode_word(w[i]);   // codes 16 i .. 16 i + 15
+                                v[4 * i] = d.x;
+                                v[4 * i + 1] = d.y;
+                                v[4 * i + 2] = d.z;
+                                v[4 * i + 3] = d.w;
+                            }
+                            tmem_st_32x32b_x32(t_st + static_cast<uint32_t>(j) * 32u, v);
+                        }
+                        tmem_st_wait();
+                        // the leader's arrivals also vouch for the stage's activation tile (both halves)
+                        if (leader && lane == 0 &&
+                            !mbar_wait(&xfull[q % XS], static_cast<uint32_t>(q / XS) & 1u, lim, abort_flag))
+                            ok = false;
+                        tc_fence_before();
+                        __syncwarp();
+                        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                        if (lane == 0) pk2_arrive_remote(dfull_leader);
+                        dph ^= 1u;
+                    }
+                    ++q;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pempty[p]);
+                if (++p == PS) { p = 0; pph ^= 1u; }
+            }
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------------------- MMA issuer (leader)
+        if (leader && elect_one()) {
+            const uint32_t idesc = umma_idesc(true, false, false, 2 * kPk2Rows, bt);
+            int d = 0, x = 0;
+            uint32_t dph = 0;
+            int tcount = 0;
+            bool ok = true;
+            for (int u = pair; u < units && ok; u += npairs, ++tcount) {
+                int nt, tt, kb0, kb1;
+                unit_of(u, nt, tt, kb0, kb1);
+                const int b = tcount % nacc;
+                const uint32_t tph = (tcount / nacc) & 1;
+                if (!pk2_wait_cluster(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * 128);
+                for (int kb = kb0; kb < kb1; kb += kPk2KbPerStage) {
+                    const int nkb = min(kPk2KbPerStage, kb1 - kb);
+                    // decoded weights of both CTAs, and (through the leader's decoders) both
+                    // activation halves
+                    if (!pk2_wait_cluster(&dfull[d], dph, lim, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_tmem = tmem_base + kPk2ACol + static_cast<uint32_t>(d) * kPk2StageCols;
+                    const uint32_t x_base = smem_u32(sX(x));
+                    for (int j = 0; j < nkb; ++j) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_pair_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
+                                              umma_desc_sw128(x_base + j * xh_bytes + kk * 32, 16, 1024), idesc,
+                                              (kb != kb0 || j != 0 || kk != 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(&dempty[d], 0x3);
+                    tc_commit_pair(&xempty[x], 0x3);
+                    if (++d == DS) { d = 0; dph ^= 1u; }
+                    if (++x == XS) x = 0;
+                }
+                if (!ok) break;
+                tc_commit_pair(&tfull[b], 0x3);
+            }
+            if (!ok) {
+                tc_commit_pair(&tfull[tcount % nacc], 0x3);
+                mbar_wait(&tfull[tcount % nacc], (tcount / nacc) & 1, 100000000ull, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ----------------------------------------------------------------- epilogue (both CTAs)
+        const int quad = warp & 3;                 // TMEM lanes [32 quad, 32 quad + 32)
+        const float gm = __ldg(args.gamma);
+        uint8_t* ebuf = sE + (warp - 2) * 2 * kPk2EpiBuf;
+        int ebi = 0;
+        int tcount = 0;
+        for (int u = pair; u < units; u += npairs, ++tcount) {
+            int nt, tt, kb0, kb1;
+            unit_of(u, nt, tt, kb0, kb1);
+            const int b = tcount % nacc;
+            const uint32_t tph = (tcount / nacc) & 1;
+            const int t0 = tt * bt;
+            // lane l holds the factor of token t0 + 32 i + l, read before the accumulators are ready
+            float fac[kPkMaxBT / 32];
+#pragma unroll
+            for (int i = 0; i < kPkMaxBT / 32; ++i) {
+                const int t = t0 + 32 * i + lane;
+                fac[i] = (args.splits == 1 && 32 * i < bt && t < args.T) ? __fdiv_rn(gm, __ldg(args.sx + t)) : 0.0f;
+            }
+            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(b * 128);
+            // per 32-token chunk: the warp's 32 rows x 32 tokens are staged in shared memory as
+            // [token][row] and written with one TMA store (rows beyond N and tokens beyond T are
+            // clipped by the tensor map); two staging tiles per warp alternate
+            const int n0 = nt * 2 * kPk2Rows + static_cast<int>(rank) * kPk2Rows + quad * 32;
+#pragma unroll 1
+            for (int i = 0; i < kPkMaxBT / 32; ++i) {
+                const int c0 = 32 * i;
+                if (c0 >= bt || t0 + c0 >= args.T) break;      // warp-uniform
+                uint32_t r[32];
+                __syncwarp();
+                tmem_ld_32x32b_x32(t_row + c0, r);
+                tmem_ld_wait();
+                auto stage = [&]() -> uint8_t* {
+                    uint8_t* e = ebuf + ebi * kPk2EpiBuf;
+                    ebi ^= 1;
+                    if (lane == 0) bulk_wait_group_read<1>();   // the tile's previous store has read it
+                    __syncwarp();
+                    return e;
+                };
+                auto flush = [&](const CUtensorMap* tm, const uint8_t* e, bool three_d, int z) {
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (three_d) tma_store_3d(tm, e, n0, t0 + c0, z);
+                        else tma_store_2d(tm, e, n0, t0 + c0);
+                        bulk_commit_group();
+                    }
+                };
+                if (args.splits > 1 || args.acc != nullptr) {
+                    uint8_t* e = stage();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) reinterpret_cast<uint32_t*>(e + j * 128)[lane] = r[j];
+                    flush(&tmAcc, e, args.splits > 1, u % args.splits);
+                    if (args.splits > 1) continue;
+                }
+                float cl = fac[0];
+#pragma unroll
+                for (int k = 1; k < kPkMaxBT / 32; ++k)
+                    if (i == k) cl = fac[k];
+                uint8_t* e = stage();
+                if constexpr (kBf16Out) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        reinterpret_cast<uint16_t*>(e + j * 64)[lane] = float_to_bf16_bits(
+                            __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j)));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        reinterpret_cast<float*>(e + j * 128)[lane] =
+                            __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j));
+                }
+                flush(&tmY, e, false, 0);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) pk2_arrive_remote(mapa_shared(smem_u32(&tempty[b]), 0));
+        }
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();   // both CTAs done with TMEM, with their barriers and with remote arrivals
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, 512);
+    }
+}
+}  // namespace bl

@@ -1,4 +1,7 @@
-"""GPU parity of the int8 x packed-ternary tensor-core linear (few tokens) against the oracle.
+"""GPU parity of the int8 x packed-ternary linear (few tokens) against the oracle, on each of
+its three kernels: the decode GEMV's (up to 16 tokens), the 1-SM tensor-core tile (up to 16
+tokens when the GEMV's activation rows do not fit shared memory) and the 2-SM tile on CTA
+pairs (17 tokens or more; 256 weight rows x up to 256 tokens, ragged in rows, tokens and K).
 
 The accumulators are exact int32 and compared bit for bit with the oracle's contraction of
 the unpacked codes (reserved code 11 decodes to 0); Y = fl(acc * fl(gamma / s_t)) is
@@ -56,7 +59,9 @@ def _check(bl, xq, packed, s, gamma, out, split):
 
 @pytest.mark.parametrize("T,K,N", [(1, 64, 16), (7, 4096, 11008), (16, 8192, 28672), (64, 2048, 2048),
                                    (129, 1024, 400), (300, 512, 1040), (33, 192, 2064), (8, 2048, 400),
-                                   (3, 1024, 272), (32, 4096, 2048), (20, 1024, 400), (16, 65536, 64)])
+                                   (3, 1024, 272), (32, 4096, 2048), (20, 1024, 400), (16, 65536, 64),
+                                   (17, 1024, 272), (96, 640, 512), (200, 1088, 1008), (257, 512, 608),
+                                   (40, 256, 40000), (64, 4096, 11008), (256, 4096, 11008)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 @pytest.mark.parametrize("split", [False, True])
 def test_linear_packed_parity(bl, T, K, N, out, split):
