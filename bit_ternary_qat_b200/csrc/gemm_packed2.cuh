@@ -26,8 +26,7 @@
 //              the stages q = g mod 4 into its TMEM stage (64 columns): each thread owns one
 //              weight row, decodes the row's codes in registers and writes them with tcgen05.st;
 //              then tcgen05.wait::st, fence, and one arrival per warp on the LEADER's barrier of
-//              that stage (8 arrivals: the group in both CTAs).  The leader's warps first wait
-//              for the stage's activation tile, so the MMA issuer waits on one barrier;
+//              that stage (8 arrivals: the group in both CTAs);
 //   warp 1     leader only: one thread issues tcgen05.mma.cta_group::2.kind::i8 (eight per stage)
 //              with A from both CTAs' TMEM stage and B from both CTAs' activation halves; its
 //              commits arrive on both CTAs' stage-empty and activation-empty barriers, and after a
@@ -39,7 +38,9 @@
 //              (pk_finalize_kernel adds them in split order); one arrival per warp on the
 //              leader's accumulator-empty barrier.
 // The single-thread MMA loop's waits and commits cost about as much as the MMAs themselves at
-// these widths (measured); two k-blocks per stage halve them per MMA.
+// these widths (measured); two k-blocks per stage halve them per MMA.  (A wait for the
+// activation tile moved from the MMA issuer into the leader's decoders measured 300-400 cycles
+// there, on the decoders' path to the MMA, against 60-90 in the issuer.)
 // TMEM (512 columns per CTA): accumulators in columns [0, 256) -- two 128-column buffers when
 // bt <= 128 (a unit's epilogue overlaps the next unit's k-loop), one 256-column buffer
 // otherwise -- and the decoded-weight ring (4 stages x 64 columns) in [256, 512).  Work units
@@ -68,42 +69,26 @@ __host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages, int xstage
            (2 * kPkMaxPStages + 2 * kPk2MaxXStages + 2 * kPk2DStages + 4) * sizeof(uint64_t) + 16;
 }
 
-// Bounded parity wait with cluster-scope acquire, for barriers that the other CTA of the pair
-// arrives on after writing its tensor memory or reading its accumulators.
-__device__ __forceinline__ bool pk2_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
-    uint32_t ok;
+// TMA load of one 2-D box with an L2 evict-first policy: the packed weight is read once per
+// launch, and keeping it from evicting the activations and the kernel's own code from L2 shortens
+// the start of the next launch.
+__device__ __forceinline__ void tma_load_2d_evict_first(void* smem_dst, const void* desc, uint64_t* bar, int32_t x,
+                                                        int32_t y) {
     asm volatile(
-        "{\n\t.reg .pred P;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, P;\n\t}"
-        : "=r"(ok)
-        : "r"(bar_addr), "r"(parity), "n"(kWaitHintNs)
+        "{\n\t.reg .b64 pol;\n\t"
+        "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], pol;\n\t}" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool pk2_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                                 volatile int* abort) {
-    const uint32_t a = smem_u32(bar);
-    if (pk2_try_wait_cluster(a, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (pk2_try_wait_cluster(a, parity)) return true;
-        if ((i & 7u) == 0u) {
-            if (abort != nullptr && *abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                record_status(6 /* BL_ERR_TIMEOUT */);
-                if (abort != nullptr) *abort = 1;
-                return false;
-            }
-        }
-    }
 }
 
 // Arrive on a barrier of either CTA of the pair (address in the cluster window) with the
-// default release at CTA scope.  The data the arrival publishes is ordered by tcgen05 fences
-// (decoded weights in TMEM, accumulators read from TMEM), not by this arrival.  Measured on
-// B200, an arrival with release at cluster scope cost 800-2500 cycles, on the path of every
-// k-block.
+// default release at CTA scope; the waiter uses the default CTA-scope acquire.  The data the
+// arrival publishes is decoded weights in TMEM, ordered by tcgen05 fences, or the release of
+// accumulators read from TMEM -- not shared memory.  Measured on B200, an arrival with release at
+// cluster scope cost 800-2500 cycles and a wait with acquire at cluster scope about 100 cycles,
+// on the path of every stage.
 __device__ __forceinline__ void pk2_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -216,14 +201,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int units = args.n_tiles * args.t_tiles * args.splits;
     const uint64_t lim = args.wait_ns;
-    // unit u -> (pair weight tile nt, token tile tt, K split sp) and its k-block range
+    // unit u -> (pair weight tile nt, token tile tt, K split sp) and its k-block range (32-bit
+    // arithmetic: k_blocks < 2^24 and splits <= 8; a 64-bit division is a called routine whose
+    // first, cold fetch measured 0.7 us at the start of every role)
+    const int splits = args.splits, t_tiles = args.t_tiles, k_blocks = args.k_blocks;
     auto unit_of = [&](int u, int& nt, int& tt, int& kb0, int& kb1) {
-        const int sp = u % args.splits;
-        const int rest = u / args.splits;
-        tt = rest % args.t_tiles;
-        nt = rest / args.t_tiles;
-        kb0 = static_cast<int>(static_cast<int64_t>(sp) * args.k_blocks / args.splits);
-        kb1 = static_cast<int>(static_cast<int64_t>(sp + 1) * args.k_blocks / args.splits);
+        const int sp = splits == 1 ? 0 : u % splits;
+        const int rest = splits == 1 ? u : u / splits;
+        tt = t_tiles == 1 ? 0 : rest % t_tiles;
+        nt = t_tiles == 1 ? rest : rest / t_tiles;
+        kb0 = splits == 1 ? 0 : sp * k_blocks / splits;
+        kb1 = splits == 1 ? k_blocks : (sp + 1) * k_blocks / splits;
     };
     // a bounded wait for the loads issued last, before the pair exits after a timeout
     auto drain = [&](uint64_t* full, int n_stages, int next, uint32_t ph, int issued) {
@@ -246,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                     // the CTA's next packed stage: k-blocks kb .. kb + 3 of its 128 rows
                     if (!mbar_wait(&pempty[p], pph ^ 1u, lim, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&pfull[p], static_cast<uint32_t>(kPkPBytes));
-                    tma_load_2d(sP(p), &tmP, &pfull[p], kb * 32, prow);
+                    tma_load_2d_evict_first(sP(p), &tmP, &pfull[p], kb * 32, prow);
                     ++issued;
                     if (++p == PS) { p = 0; pph ^= 1u; }
                 }
@@ -323,13 +311,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                             tmem_st_32x32b_x32(t_st + static_cast<uint32_t>(j) * 32u, v);
                         }
                         tmem_st_wait();
-                        // the leader's arrivals also vouch for the stage's activation tile (both halves)
-                        if (leader && lane == 0 &&
-                            !mbar_wait(&xfull[q % XS], static_cast<uint32_t>(q / XS) & 1u, lim, abort_flag))
-                            ok = false;
                         tc_fence_before();
                         __syncwarp();
-                        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                         if (lane == 0) pk2_arrive_remote(dfull_leader);
                         dph ^= 1u;
                     }
@@ -345,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
         if (leader && elect_one()) {
             const uint32_t idesc = umma_idesc(true, false, false, 2 * kPk2Rows, bt);
             int d = 0, x = 0;
-            uint32_t dph = 0;
+            uint32_t dph = 0, xph = 0;
             int tcount = 0;
             bool ok = true;
             for (int u = pair; u < units && ok; u += npairs, ++tcount) {
@@ -353,14 +336,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 unit_of(u, nt, tt, kb0, kb1);
                 const int b = tcount % nacc;
                 const uint32_t tph = (tcount / nacc) & 1;
-                if (!pk2_wait_cluster(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&tempty[b], tph ^ 1u, lim, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * 128);
                 for (int kb = kb0; kb < kb1; kb += kPk2KbPerStage) {
                     const int nkb = min(kPk2KbPerStage, kb1 - kb);
-                    // decoded weights of both CTAs, and (through the leader's decoders) both
-                    // activation halves
-                    if (!pk2_wait_cluster(&dfull[d], dph, lim, abort_flag)) { ok = false; break; }
+                    // both CTAs' activation halves and decoded weights
+                    if (!mbar_wait(&xfull[x], xph, lim, abort_flag) || !mbar_wait(&dfull[d], dph, lim, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t a_tmem = tmem_base + kPk2ACol + static_cast<uint32_t>(d) * kPk2StageCols;
                     const uint32_t x_base = smem_u32(sX(x));
@@ -374,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                     tc_commit_pair(&dempty[d], 0x3);
                     tc_commit_pair(&xempty[x], 0x3);
                     if (++d == DS) { d = 0; dph ^= 1u; }
-                    if (++x == XS) x = 0;
+                    if (++x == XS) { x = 0; xph ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit_pair(&tfull[b], 0x3);
@@ -390,6 +375,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
         const int quad = warp & 3;                 // TMEM lanes [32 quad, 32 quad + 32)
         const float gm = __ldg(args.gamma);
         uint8_t* ebuf = sE + (warp - 2) * 2 * kPk2EpiBuf;
+        // staging slots: four 2-byte tiles (bf16 Y alone) or two 4-byte tiles (f32 Y, int32 sums)
+        const bool small_tiles = kBf16Out && args.splits == 1 && args.acc == nullptr;
+        const uint32_t slot_bytes = small_tiles ? kPk2EpiBuf / 2 : kPk2EpiBuf;
+        const int nslots = small_tiles ? 4 : 2;
         int ebi = 0;
         int tcount = 0;
         for (int u = pair; u < units; u += npairs, ++tcount) {
@@ -421,9 +410,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 tmem_ld_32x32b_x32(t_row + c0, r);
                 tmem_ld_wait();
                 auto stage = [&]() -> uint8_t* {
-                    uint8_t* e = ebuf + ebi * kPk2EpiBuf;
-                    ebi ^= 1;
-                    if (lane == 0) bulk_wait_group_read<1>();   // the tile's previous store has read it
+                    uint8_t* e = ebuf + ebi * slot_bytes;
+                    ebi = ebi + 1 == nslots ? 0 : ebi + 1;
+                    // the slot's previous store has read it
+                    if (lane == 0) {
+                        if (nslots == 4) bulk_wait_group_read<3>();
+                        else bulk_wait_group_read<1>();
+                    }
                     __syncwarp();
                     return e;
                 };
