@@ -623,18 +623,17 @@ bl_status launch_packed2(const int8_t* Xq, const float* sx, int64_t T, int64_t K
     a.t_tiles = (int)((T + bt - 1) / bt);
     a.n_tiles = (int)((N + 2 * bl::kPk2Rows - 1) / (2 * bl::kPk2Rows));
     a.k_blocks = (int)((K + 127) / 128);
-    // activation stages of two k-blocks: at least 64 KB and at least as many as the decoded
-    // stages (the leader's decoders wait on an activation stage by its parity)
-    const int xstages = (int)std::min<int64_t>(bl::kPk2MaxXStages,
-                                               std::max<int64_t>(bl::kPk2DStages, 65536 / (bt * 128)));
-    a2.xstages = xstages;
     const size_t budget = (size_t)dev.max_smem_optin;
-    int pstages = (int)((budget - bl::pk2_smem_bytes((int)bt, 0, xstages)) / bl::kPkPBytes);
+    int pstages = (int)((budget - bl::pk2_smem_bytes((int)bt, 0)) / bl::kPkPBytes);
     pstages = std::min(pstages, bl::kPkMaxPStages);
-    BL_REQUIRE(pstages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
+    // the decoder warps stage their share of the last epilogue (16 x 8 KB) in the packed and
+    // activation rings
+    BL_REQUIRE(pstages >= 2 && (size_t)pstages * bl::kPkPBytes + (size_t)bl::kPk2DStages * bt * 128 >=
+                                   16 * 2 * (size_t)bl::kPk2EpiBuf,
+               BL_ERR_DEVICE, "packed GEMM: shared memory too small");
     a.pstages = pstages;
     auto kern = bl::tc_gemm_packed2_kernel<kBf16Out>;
-    const size_t smem = bl::pk2_smem_bytes((int)bt, pstages, xstages);
+    const size_t smem = bl::pk2_smem_bytes((int)bt, pstages);
     // pairs resident at once, per device and token-tile width (the shared memory differs)
     static std::atomic<int> max_clusters[64][bl::kPkMaxBT / 32] = {};
     int dev_id = 0;

@@ -21,7 +21,8 @@
 //              row per stage, 128-byte swizzle) into its packed ring (its own barriers);
 //   warp 22    activation producer: TMA loads of the CTA's half of the token tile (bt / 2 rows x
 //              128 bytes per k-block) with the 2-SM TMA form, whose completion bytes count on the
-//              leader's barrier;
+//              leader's barrier of the stage -- the same barrier the decoders arrive on, so the
+//              MMA issuer waits once and commits once per stage;
 //   warps 6-21 decoders, four groups of four warps (one per TMEM lane quarter): group g decodes
 //              the stages q = g mod 4 into its TMEM stage (64 columns): each thread owns one
 //              weight row, decodes the row's codes in registers and writes them with tcgen05.st;
@@ -29,18 +30,17 @@
 //              that stage (8 arrivals: the group in both CTAs);
 //   warp 1     leader only: one thread issues tcgen05.mma.cta_group::2.kind::i8 (eight per stage)
 //              with A from both CTAs' TMEM stage and B from both CTAs' activation halves; its
-//              commits arrive on both CTAs' stage-empty and activation-empty barriers, and after a
-//              unit's last stage on both CTAs' accumulator-full barriers;
+//              commit frees the stage in both CTAs (TMEM and activation tile), and after a unit's
+//              last stage another arrives on both CTAs' accumulator-full barriers;
 //   warps 2-5  epilogue (both CTAs): TMEM lanes are the CTA's 128 weight rows; the unit's token
 //              factors fl(gamma / s_t) are read before its accumulators are ready; per 32-token
 //              chunk tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (coalesced along n), or
 //              the exact int32 partial sums of K split sp into slice sp of a workspace
 //              (pk_finalize_kernel adds them in split order); one arrival per warp on the
 //              leader's accumulator-empty barrier.
-// The single-thread MMA loop's waits and commits cost about as much as the MMAs themselves at
-// these widths (measured); two k-blocks per stage halve them per MMA.  (A wait for the
-// activation tile moved from the MMA issuer into the leader's decoders measured 300-400 cycles
-// there, on the decoders' path to the MMA, against 60-90 in the issuer.)
+// The single-thread MMA loop's barrier waits (about 130 cycles each, measured, even on a completed
+// phase) and commits cost about as much as the MMAs themselves at these widths: two k-blocks per
+// stage and one barrier per stage keep them to one wait and one commit per 8 MMAs.
 // TMEM (512 columns per CTA): accumulators in columns [0, 256) -- two 128-column buffers when
 // bt <= 128 (a unit's epilogue overlaps the next unit's k-loop), one 256-column buffer
 // otherwise -- and the decoded-weight ring (4 stages x 64 columns) in [256, 512).  Work units
@@ -54,19 +54,20 @@ namespace bl {
 
 constexpr int kPk2Rows = 128;          // weight rows per CTA (a pair tile: 256)
 constexpr int kPk2Threads = kPkThreads + 32;   // + the activation producer warp
-constexpr int kPk2MaxXStages = 16;     // activation ring depth (stages of 2 x bt / 2 x 128 bytes)
-constexpr int kPk2DStages = 4;         // decoded-weight stages in TMEM (one per decoder group)
+constexpr int kPk2DStages = 4;         // stages in flight: decoded weights in TMEM (one per decoder
+                                       // group) and activation tiles in shared memory
 constexpr int kPk2KbPerStage = 2;      // k-blocks per activation / decoded stage
 constexpr uint32_t kPk2ACol = 256;     // first TMEM column of the decoded-weight ring
 constexpr uint32_t kPk2StageCols = 64; // 256 int8 codes per row = 64 columns
 
 constexpr uint32_t kPk2EpiBuf = 32 * 32 * 4;   // one 32-token x 32-row tile of 4-byte values
 constexpr uint32_t kPk2EpiBytes = 4 * 2 * kPk2EpiBuf;   // two staging tiles per epilogue warp
+constexpr int kPk2EpiHelpers = 5;      // warps per TMEM quarter sharing a pair's last epilogue:
+                                       // its epilogue warp and its four decoder warps
 
-__host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages, int xstages) {
-    return 1024 + static_cast<size_t>(pstages) * kPkPBytes + static_cast<size_t>(xstages) * static_cast<size_t>(bt) * 128 +
-           kPk2EpiBytes +
-           (2 * kPkMaxPStages + 2 * kPk2MaxXStages + 2 * kPk2DStages + 4) * sizeof(uint64_t) + 16;
+__host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages) {
+    return 1024 + static_cast<size_t>(pstages) * kPkPBytes + static_cast<size_t>(kPk2DStages) * static_cast<size_t>(bt) * 128 +
+           kPk2EpiBytes + (2 * kPkMaxPStages + 2 * kPk2DStages + 4) * sizeof(uint64_t) + 16;
 }
 
 // TMA load of one 2-D box with an L2 evict-first policy: the packed weight is read once per
@@ -127,7 +128,6 @@ __device__ __forceinline__ void tc_mma_pair_i8_ts(uint32_t d_tmem, uint32_t a_tm
 
 struct Pk2Args {
     PkArgs pk;        // shapes, outputs, pstages; pk.bt is the pair tile's token count
-    int xstages;      // activation ring depth
 };
 
 template <bool kBf16Out>
@@ -140,21 +140,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_align1024(smem_raw);
     const int PS = args.pstages;
-    const int XS = a2.xstages;
     const int bt = args.bt;                                            // multiple of 32
     const int nacc = bt <= 128 ? 2 : 1;                                // accumulator buffers
     const uint32_t xh_bytes = static_cast<uint32_t>(bt) * 64u;         // one k-block: bt / 2 rows x 128 bytes
-    // [packed: PS x 16 KB][activation halves: XS x 2 k-blocks x xh_bytes][epilogue staging]; 1024-aligned
+    // [packed: PS x 16 KB][activation halves: DS x 2 k-blocks x xh_bytes][epilogue staging]; 1024-aligned
     auto sP = [&](int p) { return smem + p * kPkPBytes; };
     uint8_t* sXbase = smem + PS * kPkPBytes;
     auto sX = [&](int x) { return sXbase + static_cast<uint32_t>(x) * (kPk2KbPerStage * xh_bytes); };
-    uint8_t* sE = sXbase + static_cast<uint32_t>(XS) * (kPk2KbPerStage * xh_bytes);
+    uint8_t* sE = sXbase + static_cast<uint32_t>(DS) * (kPk2KbPerStage * xh_bytes);
     uint64_t* pfull = reinterpret_cast<uint64_t*>(sE + kPk2EpiBytes);
     uint64_t* pempty = pfull + kPkMaxPStages;    // this CTA's 16 decoder warps
-    uint64_t* xfull = pempty + kPkMaxPStages;    // leader's is used: both CTAs' activation bytes
-    uint64_t* xempty = xfull + kPk2MaxXStages;   // each CTA: the leader's commit
-    uint64_t* dfull = xempty + kPk2MaxXStages;   // leader's is used: the stage's group in both CTAs
-    uint64_t* dempty = dfull + DS;               // each CTA: the leader's commit
+    // stage d: dfull[d] (the leader's is used) completes when the group of d in both CTAs has
+    // arrived (8 warps), the leader's activation producer has arrived with the stage's byte
+    // count, and both CTAs' activation halves have landed; dempty[d] (each CTA) is the leader's
+    // commit after the stage's MMAs (frees the TMEM stage and the activation stage)
+    uint64_t* dfull = pempty + kPkMaxPStages;
+    uint64_t* dempty = dfull + DS;
     uint64_t* tfull = dempty + DS;               // each CTA: the leader's commit after a unit
     uint64_t* tempty = tfull + 2;                // leader's is used: 4 epilogue warps per CTA
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
@@ -169,12 +170,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
             mbar_init(&pfull[p], 1);
             mbar_init(&pempty[p], 4 * kPkDecGroups);
         }
-        for (int x = 0; x < XS; ++x) {
-            mbar_init(&xfull[x], 1);
-            mbar_init(&xempty[x], 1);
-        }
         for (int d = 0; d < DS; ++d) {
-            mbar_init(&dfull[d], 8);
+            mbar_init(&dfull[d], 9);
             mbar_init(&dempty[d], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -220,6 +217,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
             mbar_wait(&full[s], (next - 1 - i < 0) ? (ph ^ 1u) : ph, 100000000ull, nullptr);
         }
     };
+    // ---- epilogue pieces: the epilogue warps run them for every unit; for the pair's last unit
+    // the decoder warps take a share of the chunks (see the decoder role)
+    // staging slots: four 2-byte tiles (bf16 Y alone) or two 4-byte tiles (f32 Y, int32 sums)
+    const bool small_tiles = kBf16Out && args.splits == 1 && args.acc == nullptr;
+    const uint32_t slot_bytes = small_tiles ? kPk2EpiBuf / 2 : kPk2EpiBuf;
+    const int nslots = small_tiles ? 4 : 2;
+    // fl(gamma / s_t) of token t (0 for the K-split partial sums, which are scaled later)
+    auto token_factor = [&](float gm, int t) -> float {
+        return (args.splits == 1 && t < args.T) ? __fdiv_rn(gm, __ldg(args.sx + t)) : 0.0f;
+    };
+    // chunk i of unit u: this warp's 32 TMEM lanes (weight rows) x 32 tokens, staged in shared
+    // memory as [token][row] and written with one TMA store (rows beyond N and tokens beyond T are
+    // clipped by the tensor map); cl = the factor of token t0 + 32 i + lane
+    auto epi_chunk = [&](int u, int nt, int t0, uint32_t t_row, int i, float cl, uint8_t* ebuf, int& ebi) {
+        const int c0 = 32 * i;
+        const int n0 = nt * 2 * kPk2Rows + static_cast<int>(rank) * kPk2Rows + (warp & 3) * 32;
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row + c0, r);
+        tmem_ld_wait();
+        auto stage = [&]() -> uint8_t* {
+            uint8_t* e = ebuf + ebi * slot_bytes;
+            ebi = ebi + 1 == nslots ? 0 : ebi + 1;
+            // the slot's previous store has read it
+            if (lane == 0) {
+                if (nslots == 4) bulk_wait_group_read<3>();
+                else bulk_wait_group_read<1>();
+            }
+            __syncwarp();
+            return e;
+        };
+        auto flush = [&](const CUtensorMap* tm, const uint8_t* e, bool three_d, int z) {
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                if (three_d) tma_store_3d(tm, e, n0, t0 + c0, z);
+                else tma_store_2d(tm, e, n0, t0 + c0);
+                bulk_commit_group();
+            }
+        };
+        if (args.splits > 1 || args.acc != nullptr) {
+            uint8_t* e = stage();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) reinterpret_cast<uint32_t*>(e + j * 128)[lane] = r[j];
+            flush(&tmAcc, e, args.splits > 1, u % args.splits);
+            if (args.splits > 1) return;
+        }
+        uint8_t* e = stage();
+        if constexpr (kBf16Out) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                reinterpret_cast<uint16_t*>(e + j * 64)[lane] = float_to_bf16_bits(
+                    __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j)));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                reinterpret_cast<float*>(e + j * 128)[lane] =
+                    __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j));
+        }
+        flush(&tmY, e, false, 0);
+    };
+
     if (warp == 0) {
         // ----------------------------------------------------------------- packed producer (both CTAs)
         if (elect_one()) {
@@ -245,8 +304,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
     } else if (warp == kPk2Threads / 32 - 1) {
         // ----------------------------------------------------------------- activation producer (both CTAs)
         if (elect_one()) {
-            int x = 0, issued = 0;
-            uint32_t xph = 0;
+            int d = 0;
+            uint32_t dph = 0;
             bool ok = true;
             for (int u = pair; u < units && ok; u += npairs) {
                 int nt, tt, kb0, kb1;
@@ -254,17 +313,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 const int trow = tt * bt + static_cast<int>(rank) * (bt / 2);
                 for (int kb = kb0; kb < kb1; kb += kPk2KbPerStage) {
                     const int nkb = min(kPk2KbPerStage, kb1 - kb);
-                    if (!mbar_wait(&xempty[x], xph ^ 1u, lim, abort_flag)) { ok = false; break; }
-                    if (leader) mbar_arrive_expect_tx(&xfull[x], 2u * static_cast<uint32_t>(nkb) * xh_bytes);
-                    const uint32_t bar = mapa_shared(smem_u32(&xfull[x]), 0);
+                    // the stage's previous MMAs are done in both CTAs; the leader's barrier is in
+                    // this stage's phase
+                    if (!mbar_wait(&dempty[d], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    if (leader) mbar_arrive_expect_tx(&dfull[d], 2u * static_cast<uint32_t>(nkb) * xh_bytes);
+                    const uint32_t bar = mapa_shared(smem_u32(&dfull[d]), 0);
                     for (int j = 0; j < nkb; ++j)
-                        tma_load_2d_pair(sX(x) + j * xh_bytes, &tmX, bar, (kb + j) * 128, trow);
-                    ++issued;
-                    if (++x == XS) { x = 0; xph ^= 1u; }
+                        tma_load_2d_pair(sX(d) + j * xh_bytes, &tmX, bar, (kb + j) * 128, trow);
+                    if (++d == DS) { d = 0; dph ^= 1u; }
                 }
             }
-            // the leader's barriers count both CTAs' bytes
-            if (!ok && leader) drain(xfull, XS, x, xph, issued);
+            // the loads issued last complete on a barrier that also waits for decoder arrivals:
+            // after a timeout, give them time to land before the pair exits
+            if (!ok) {
+                const uint64_t t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 50000ull) __nanosleep(1000);
+            }
         }
         __syncwarp();
     } else if (warp >= 6) {
@@ -323,12 +387,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 if (++p == PS) { p = 0; pph ^= 1u; }
             }
         }
+        // the pair's last unit: this warp takes epilogue chunks 1 + grp and 1 + grp + 5 of its TMEM
+        // quarter (the quarter's epilogue warp takes chunks 0 and 5).  Its staging tiles lie in the
+        // packed and activation rings, whose last loads have been consumed once the unit's
+        // accumulators are complete.
+        if (ok && pair < units) {
+            const int last = (units - 1 - pair) / npairs;       // the unit's index among the pair's
+            const int u = pair + last * npairs;
+            int nt, tt, kb0, kb1;
+            unit_of(u, nt, tt, kb0, kb1);
+            const int t0 = tt * bt;
+            const int i0 = 1 + grp, i1 = 1 + grp + kPk2EpiHelpers;
+            if (32 * i0 < bt && t0 + 32 * i0 < args.T) {
+                const float gm = __ldg(args.gamma);
+                const float cl0 = token_factor(gm, t0 + 32 * i0 + lane);
+                const float cl1 = 32 * i1 < bt ? token_factor(gm, t0 + 32 * i1 + lane) : 0.0f;
+                const int b = last % nacc;
+                if (mbar_wait(&tfull[b], (last / nacc) & 1, lim, abort_flag)) {
+                    tc_fence_after();
+                    uint8_t* hbuf = smem + (warp - 6) * 2 * kPk2EpiBuf;
+                    int hbi = 0;
+                    const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                                           static_cast<uint32_t>(b * 128);
+                    epi_chunk(u, nt, t0, t_row, i0, cl0, hbuf, hbi);
+                    if (32 * i1 < bt && t0 + 32 * i1 < args.T) epi_chunk(u, nt, t0, t_row, i1, cl1, hbuf, hbi);
+                    if (lane == 0) bulk_wait_group<0>();
+                    __syncwarp();
+                }
+            }
+        }
     } else if (warp == 1) {
         // ----------------------------------------------------------------- MMA issuer (leader)
         if (leader && elect_one()) {
             const uint32_t idesc = umma_idesc(true, false, false, 2 * kPk2Rows, bt);
-            int d = 0, x = 0;
-            uint32_t dph = 0, xph = 0;
+            int d = 0;
+            uint32_t dph = 0;
             int tcount = 0;
             bool ok = true;
             for (int u = pair; u < units && ok; u += npairs, ++tcount) {
@@ -341,14 +434,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(b * 128);
                 for (int kb = kb0; kb < kb1; kb += kPk2KbPerStage) {
                     const int nkb = min(kPk2KbPerStage, kb1 - kb);
-                    // both CTAs' activation halves and decoded weights
-                    if (!mbar_wait(&xfull[x], xph, lim, abort_flag) || !mbar_wait(&dfull[d], dph, lim, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+                    // both CTAs' decoded weights and activation halves
+                    if (!mbar_wait(&dfull[d], dph, lim, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_tmem = tmem_base + kPk2ACol + static_cast<uint32_t>(d) * kPk2StageCols;
-                    const uint32_t x_base = smem_u32(sX(x));
+                    const uint32_t x_base = smem_u32(sX(d));
                     for (int j = 0; j < nkb; ++j) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
@@ -357,9 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                                               (kb != kb0 || j != 0 || kk != 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&dempty[d], 0x3);
-                    tc_commit_pair(&xempty[x], 0x3);
                     if (++d == DS) { d = 0; dph ^= 1u; }
-                    if (++x == XS) { x = 0; xph ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit_pair(&tfull[b], 0x3);
@@ -375,10 +463,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
         const int quad = warp & 3;                 // TMEM lanes [32 quad, 32 quad + 32)
         const float gm = __ldg(args.gamma);
         uint8_t* ebuf = sE + (warp - 2) * 2 * kPk2EpiBuf;
-        // staging slots: four 2-byte tiles (bf16 Y alone) or two 4-byte tiles (f32 Y, int32 sums)
-        const bool small_tiles = kBf16Out && args.splits == 1 && args.acc == nullptr;
-        const uint32_t slot_bytes = small_tiles ? kPk2EpiBuf / 2 : kPk2EpiBuf;
-        const int nslots = small_tiles ? 4 : 2;
         int ebi = 0;
         int tcount = 0;
         for (int u = pair; u < units; u += npairs, ++tcount) {
@@ -387,72 +471,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
             const int b = tcount % nacc;
             const uint32_t tph = (tcount / nacc) & 1;
             const int t0 = tt * bt;
+            // the pair's last unit: chunks i = 0 mod kPk2EpiHelpers here, the rest in the decoders
+            const int step = u + npairs >= units ? kPk2EpiHelpers : 1;
             // lane l holds the factor of token t0 + 32 i + l, read before the accumulators are ready
             float fac[kPkMaxBT / 32];
 #pragma unroll
-            for (int i = 0; i < kPkMaxBT / 32; ++i) {
-                const int t = t0 + 32 * i + lane;
-                fac[i] = (args.splits == 1 && 32 * i < bt && t < args.T) ? __fdiv_rn(gm, __ldg(args.sx + t)) : 0.0f;
-            }
+            for (int i = 0; i < kPkMaxBT / 32; ++i)
+                fac[i] = (32 * i < bt && i % step == 0) ? token_factor(gm, t0 + 32 * i + lane) : 0.0f;
             if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(b * 128);
-            // per 32-token chunk: the warp's 32 rows x 32 tokens are staged in shared memory as
-            // [token][row] and written with one TMA store (rows beyond N and tokens beyond T are
-            // clipped by the tensor map); two staging tiles per warp alternate
-            const int n0 = nt * 2 * kPk2Rows + static_cast<int>(rank) * kPk2Rows + quad * 32;
 #pragma unroll 1
-            for (int i = 0; i < kPkMaxBT / 32; ++i) {
-                const int c0 = 32 * i;
-                if (c0 >= bt || t0 + c0 >= args.T) break;      // warp-uniform
-                uint32_t r[32];
-                __syncwarp();
-                tmem_ld_32x32b_x32(t_row + c0, r);
-                tmem_ld_wait();
-                auto stage = [&]() -> uint8_t* {
-                    uint8_t* e = ebuf + ebi * slot_bytes;
-                    ebi = ebi + 1 == nslots ? 0 : ebi + 1;
-                    // the slot's previous store has read it
-                    if (lane == 0) {
-                        if (nslots == 4) bulk_wait_group_read<3>();
-                        else bulk_wait_group_read<1>();
-                    }
-                    __syncwarp();
-                    return e;
-                };
-                auto flush = [&](const CUtensorMap* tm, const uint8_t* e, bool three_d, int z) {
-                    fence_proxy_async_shared();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (three_d) tma_store_3d(tm, e, n0, t0 + c0, z);
-                        else tma_store_2d(tm, e, n0, t0 + c0);
-                        bulk_commit_group();
-                    }
-                };
-                if (args.splits > 1 || args.acc != nullptr) {
-                    uint8_t* e = stage();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) reinterpret_cast<uint32_t*>(e + j * 128)[lane] = r[j];
-                    flush(&tmAcc, e, args.splits > 1, u % args.splits);
-                    if (args.splits > 1) continue;
-                }
+            for (int i = 0; i < kPkMaxBT / 32; i += step) {
+                if (32 * i >= bt || t0 + 32 * i >= args.T) break;      // warp-uniform
                 float cl = fac[0];
 #pragma unroll
                 for (int k = 1; k < kPkMaxBT / 32; ++k)
                     if (i == k) cl = fac[k];
-                uint8_t* e = stage();
-                if constexpr (kBf16Out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        reinterpret_cast<uint16_t*>(e + j * 64)[lane] = float_to_bf16_bits(
-                            __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j)));
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        reinterpret_cast<float*>(e + j * 128)[lane] =
-                            __fmul_rn(static_cast<float>(static_cast<int32_t>(r[j])), __shfl_sync(0xffffffffu, cl, j));
-                }
-                flush(&tmY, e, false, 0);
+                epi_chunk(u, nt, t0, t_row, i, cl, ebuf, ebi);
             }
             tc_fence_before();
             __syncwarp();
