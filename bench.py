@@ -60,7 +60,9 @@ def parse():
                     help="run each HBM-bound kernel of the step (and the optimizer step) once on 7B-MLP-sized "
                          "inputs larger than L2 (profiling)")
     ap.add_argument("--only-packed", action="store_true",
-                    help="run only the packed-weight linear at 16 tokens on the 28672 x 8192 weight (profiling)")
+                    help="run three launches of the packed-weight linear only (profiling); see --packed-case")
+    ap.add_argument("--packed-case", default="16,28672,8192",
+                    help="tokens,d_out,d_in of --only-packed (default: 16 tokens on the 28672 x 8192 weight)")
     ap.add_argument("--only-gemm", choices=["linear_i8", "grad_input", "grad_weight"], default=None,
                     help="run three launches of one GEMM of the step at 16384 tokens (profiling)")
     ap.add_argument("--gemm-shape", choices=["q", "gate", "down"], default="gate",
@@ -346,7 +348,8 @@ def main():
         if args.only_mem:
             print(json.dumps({"memory_kernels": mem_once(bl, torch, dev)}), flush=True)
         elif args.only_packed:
-            print(json.dumps({"linear_packed": packed_once(bl, torch, dev)}), flush=True)
+            T_, N_, K_ = (int(v) for v in args.packed_case.split(","))
+            print(json.dumps({"linear_packed": packed_once(bl, torch, dev, T_, N_, K_)}), flush=True)
         elif args.next:
             print(json.dumps({"next": next_measure(bl, torch, dev, flush, peaks())}), flush=True)
         elif args.table:
@@ -1062,11 +1065,10 @@ def mem_once(bl, torch, dev):
             "optimizer_step": f"{K}x{N} with re-quantisation"}
 
 
-def packed_once(bl, torch, dev):
-    """Three launches of the packed-weight linear, 16 tokens x the 28672 x 8192 decode weight
-    (a small case for a profiler capture); returns the last launch's event time."""
+def packed_once(bl, torch, dev, T=16, N=28672, K=8192):
+    """Three launches of the packed-weight linear, T tokens x an N x K weight (a small case for a
+    profiler capture); returns the last launch's event time."""
     from bit_ternary_qat_b200 import synth
-    N, K, T = 28672, 8192, 16
     W, _ = synth.decode_inputs(1, N, K)
     q = bl.bitlinear_quant_weight(W.to(dev), want_i8=False, want_bf16=False)
     del W
@@ -1194,7 +1196,9 @@ def next_measure(bl, torch, dev, flush, pk):
                                           "note": "fl(gamma_n / s_t) per element epilogue"}
     del xq, y
     # packed-weight tensor-core linear vs the int8-code linear and the decode GEMV, few tokens
-    for (T, N, K) in ((16, 28672, 8192), (64, 11008, 4096), (256, 11008, 4096)):
+    for (T, N, K) in ((16, 28672, 8192), (64, 28672, 8192), (256, 28672, 8192), (32, 11008, 4096),
+                      (64, 11008, 4096), (128, 11008, 4096), (256, 11008, 4096), (64, 4096, 4096),
+                      (256, 4096, 4096)):
         Wd = synth.normal((N, K), 0.02, gen).to(dev)
         qd = bl.bitlinear_quant_weight(Wd)
         del Wd
@@ -1214,6 +1218,8 @@ def next_measure(bl, torch, dev, flush, pk):
                "packed_weight_GBs": N * K / 4 / (us_p * 1e-6) / 1e9,
                "packed_frac_hbm": (N * K / 4 + T * K + 2 * T * N) / (us_p * 1e-6) / 1e9 / pk["hbm"],
                "int8_frac_hbm": (N * K + T * K + 2 * T * N) / (us_8 * 1e-6) / 1e9 / pk["hbm"],
+               "speedup_vs_int8": us_8 / us_p,
+               "kernel": "ternary_gemv" if T <= 16 else "tc_gemm_packed2 (CTA pairs)",
                "weight_copies": {"int8": c8, "packed": cp}}
         if T <= 16:
             y32 = torch.empty(T, N, dtype=torch.float32, device=dev)

@@ -304,17 +304,21 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
 /* ==============================================================================
  * int8 x packed-ternary linear for few tokens (prefill chunks, batched decode): the
  * linear of bitlinear_linear computed from the 2-bit packed weight (P5 §4.1 codes, §5.1
- * packing; a quarter of the int8 weight bytes cross HBM), decoded to int8 in shared
- * memory and multiplied on the tensor cores (P3 §3.1):
+ * packing; a quarter of the int8 weight bytes cross HBM), decoded to int8 on chip and
+ * multiplied on the tensor cores (P3 §3.1):
  *   acc[t,n] = sum_k decode(Wpacked[n,k]) * Xq[t,k]     exact int32 (reserved 11 -> 0)
  *   Y[t,n]   = fl32(acc[t,n] * fl32(gamma / sx[t]))     in y_dt
  * Xq int8 [T x K]; sx fp32 [T]; Wpacked uint8 [N x K/4]; gamma fp32 [1]; Y [T x N];
  * acc int32 [T x N] optional.  K % 64 == 0.  Meant for T up to a few hundred tokens
- * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).  Up to 16
- * tokens (when their activation rows fit one block's shared memory) the call runs the decode
- * GEMV's kernel (codes decoded in registers, warp-level int8 MMA; ws unused).  When the
- * weight tiles alone cannot fill the GPU and at most 64 tokens are given, K may be split
- * across CTAs: split sp stores its exact int32 partial sums to slice sp of ws (int32
+ * (beyond that bitlinear_linear on the int8 codes is compute-bound and faster).
+ * Kernels by token count:
+ *   up to 16 tokens, when their activation rows fit one block's shared memory: the decode
+ *     GEMV's kernel (codes decoded in registers, warp-level int8 MMA; ws unused);
+ *   17 tokens or more: CTA pairs with 256 weight rows x up to 256 tokens per tile (codes
+ *     decoded into tensor memory, 2-SM tcgen05 MMAs, TMA-stored output);
+ *   other cases of up to 16 tokens: a 1-SM tensor-core tile.
+ * When the weight tiles alone cannot fill the GPU and at most 64 tokens are given, K may be
+ * split: split sp stores its exact int32 partial sums to slice sp of ws (int32
  * [splits x T x N]) and a second launch adds the slices in split order and applies the
  * scale.  The split count is limited by ws_bytes / (4 T N) (ws NULL: no split), by 8 and by
  * K / (64 T).  One or two launches. */
