@@ -9,10 +9,10 @@
 // The decoded weight never touches shared memory: each decoder thread owns one weight row,
 // decodes the row's 128 codes of a k-block in registers and writes them with tcgen05.st into
 // its CTA's tensor memory (lane = row, 4 codes per 32-bit column), where the MMA reads its A
-// operand.  Staging the decoded int8 tile in shared memory instead cost 1 byte written by the
-// decoders and 1 byte read by the tensor core per code, on top of the packed and activation
-// tiles; measured on B200, the decoders then ran at a fraction of their issue rate while the
-// MMAs streamed, and the kernel was slower than the int8-code GEMM from 32 tokens up.
+// operand.  That saves the 2 bytes of shared-memory traffic per code of a staged int8 tile,
+// and an M = 256 instruction with A in TMEM measured faster than with A in shared memory in
+// the same issue loop (26.8 / 41 / 73 / 137 against 58.5 / 72.9 / 103.6 / 167.6 cycles at
+// N = 32 / 64 / 128 / 256).
 //
 // Per CTA r of a pair (rows [256 u + 128 r, +128) of weight tile u), 736 threads.  A "stage"
 // of the activation and decoded-weight rings is two k-blocks (256 codes of K); a packed stage
@@ -27,17 +27,19 @@
 //              the stages q = g mod 4 into its TMEM stage (64 columns): each thread owns one
 //              weight row, decodes the row's codes in registers and writes them with tcgen05.st;
 //              then tcgen05.wait::st, fence, and one arrival per warp on the LEADER's barrier of
-//              that stage (8 arrivals: the group in both CTAs);
+//              that stage (9 arrivals: the group in both CTAs and the leader's activation
+//              producer);
 //   warp 1     leader only: one thread issues tcgen05.mma.cta_group::2.kind::i8 (eight per stage)
 //              with A from both CTAs' TMEM stage and B from both CTAs' activation halves; its
 //              commit frees the stage in both CTAs (TMEM and activation tile), and after a unit's
 //              last stage another arrives on both CTAs' accumulator-full barriers;
 //   warps 2-5  epilogue (both CTAs): TMEM lanes are the CTA's 128 weight rows; the unit's token
 //              factors fl(gamma / s_t) are read before its accumulators are ready; per 32-token
-//              chunk tcgen05.ld, then y[t, n] = fl(acc * fl(gamma / s_t)) (coalesced along n), or
-//              the exact int32 partial sums of K split sp into slice sp of a workspace
-//              (pk_finalize_kernel adds them in split order); one arrival per warp on the
-//              leader's accumulator-empty barrier.
+//              chunk tcgen05.ld, y[t, n] = fl(acc * fl(gamma / s_t)) staged in shared memory as a
+//              [token][row] tile and written with one TMA store (or the exact int32 partial sums
+//              of K split sp into slice sp of a workspace, which pk_finalize_kernel adds in split
+//              order); one arrival per warp on the leader's accumulator-empty barrier.  For the
+//              pair's last unit the decoder warps, idle by then, take four of every five chunks.
 // The single-thread MMA loop's barrier waits (about 130 cycles each, measured, even on a completed
 // phase) and commits cost about as much as the MMAs themselves at these widths: two k-blocks per
 // stage and one barrier per stage keep them to one wait and one commit per 8 MMAs.
