@@ -86,6 +86,15 @@ __device__ __forceinline__ void tma_load_2d_evict_first(void* smem_dst, const vo
         : "memory");
 }
 
+// L2 prefetch of one 2-D box of a tensor map (no data returns to the SM, so it may run before
+// the launch's dependency wait: L2 is the point of coherence for the previous kernel's writes).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* desc, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(desc)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Arrive on a barrier of either CTA of the pair (address in the cluster window) with the
 // default release at CTA scope; the waiter uses the default CTA-scope acquire.  The data the
 // arrival publishes is decoded weights in TMEM, ordered by tcgen05 fences, or the release of
@@ -195,9 +204,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
     cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    if (warp == 0 && lane == 0) {
+        // the first unit's first packed stages into L2 while the previous kernel finishes
+        // (its k-blocks [0, k_blocks / splits): the split index is 0 or the unit's own)
+        const int nt = (pair / args.splits) / args.t_tiles;
+        const int sp = pair % args.splits;
+        const int kb0 = sp * args.k_blocks / args.splits;
+        const int kb1 = (sp + 1) * args.k_blocks / args.splits;
+        const int prow = nt * 2 * kPk2Rows + static_cast<int>(rank) * kPk2Rows;
+        for (int i = 0, kb = kb0; i < PS && kb < kb1; ++i, kb += kPkKbPerP) tma_prefetch_l2_2d(&tmP, kb * 32, prow);
+    }
     pdl_trigger_and_wait();
 
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int units = args.n_tiles * args.t_tiles * args.splits;
     const uint64_t lim = args.wait_ns;
     // unit u -> (pair weight tile nt, token tile tt, K split sp) and its k-block range (32-bit
