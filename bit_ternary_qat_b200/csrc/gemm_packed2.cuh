@@ -137,6 +137,35 @@ __device__ __forceinline__ void tc_mma_pair_i8_ts(uint32_t d_tmem, uint32_t a_tm
         : "memory");
 }
 
+// The eight MMAs of a full stage (two k-blocks x four 32-code steps) in one asm block.  A: 8
+// TMEM columns per step from `a`.  B: the shared-memory descriptors b0 and b1 of the stage's
+// two activation k-blocks, 32 bytes (2 in the descriptor's start-address field, which cannot
+// carry: addresses stay below 256 KB) per step.  The first MMA accumulates iff `accumulate`,
+// the other seven always.  One predicate set-up per stage instead of per MMA: measured on B200,
+// a single thread issuing MMAs one C++ call at a time needed ~50 cycles per N = 64 instruction,
+// which the tensor pipe runs in 32.
+__device__ __forceinline__ void pk2_mma_stage(uint32_t d_tmem, uint32_t a, uint64_t b0, uint64_t b1, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred P, Q;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t.reg .b64 c1, c2, c3, c5, c6, c7;\n\t"
+        "setp.ne.b32 P, %5, 0;\n\t"
+        "setp.eq.b32 Q, %5, %5;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\tadd.u32 a4, %1, 32;\n\t"
+        "add.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+        "add.s64 c1, %2, 2;\n\tadd.s64 c2, %2, 4;\n\tadd.s64 c3, %2, 6;\n\t"
+        "add.s64 c5, %3, 2;\n\tadd.s64 c6, %3, 4;\n\tadd.s64 c7, %3, 6;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %4, P;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a1], c1, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a2], c2, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a3], c3, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a4], %3, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a5], c5, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a6], c6, %4, Q;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [a7], c7, %4, Q;\n\t}" ::"r"(d_tmem),
+        "r"(a), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 struct Pk2Args {
     PkArgs pk;        // shapes, outputs, pstages; pk.bt is the pair tile's token count
 };
@@ -441,6 +470,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
         // ----------------------------------------------------------------- MMA issuer (leader)
         if (leader && elect_one()) {
             const uint32_t idesc = umma_idesc(true, false, false, 2 * kPk2Rows, bt);
+            // B descriptors: stage d's first k-block at x_desc0 + d * x_stage16, its second
+            // xh16 further (descriptor start addresses count 16-byte units)
+            const uint64_t x_desc0 = umma_desc_sw128(smem_u32(sXbase), 16, 1024);
+            const uint64_t x_stage16 = static_cast<uint64_t>((kPk2KbPerStage * xh_bytes) >> 4);
+            const uint64_t xh16 = static_cast<uint64_t>(xh_bytes >> 4);
             int d = 0;
             uint32_t dph = 0;
             int tcount = 0;
@@ -459,13 +493,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                     if (!mbar_wait(&dfull[d], dph, lim, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_tmem = tmem_base + kPk2ACol + static_cast<uint32_t>(d) * kPk2StageCols;
-                    const uint32_t x_base = smem_u32(sX(d));
-                    for (int j = 0; j < nkb; ++j) {
+                    const uint64_t b0 = x_desc0 + static_cast<uint64_t>(d) * x_stage16;
+                    if (nkb == kPk2KbPerStage) {
+                        pk2_mma_stage(d_tmem, a_tmem, b0, b0 + xh16, idesc, kb != kb0 ? 1u : 0u);
+                    } else {   // a unit's last, single k-block
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_pair_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
-                                              umma_desc_sw128(x_base + j * xh_bytes + kk * 32, 16, 1024), idesc,
-                                              (kb != kb0 || j != 0 || kk != 0) ? 1u : 0u);
+                            tc_mma_pair_i8_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>(2 * kk), idesc,
+                                              (kb != kb0 || kk != 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&dempty[d], 0x3);
                     if (++d == DS) { d = 0; dph ^= 1u; }
