@@ -12,7 +12,8 @@
 // operand.  That saves the 2 bytes of shared-memory traffic per code of a staged int8 tile,
 // and an M = 256 instruction with A in TMEM measured faster than with A in shared memory in
 // the same issue loop (26.8 / 41 / 73 / 137 against 58.5 / 72.9 / 103.6 / 167.6 cycles at
-// N = 32 / 64 / 128 / 256).
+// N = 32 / 64 / 128 / 256); issued without per-instruction overhead it runs at the full int8
+// rate (16 / 32 cycles at N = 32 / 64).
 //
 // Per CTA r of a pair (rows [256 u + 128 r, +128) of weight tile u), 736 threads.  A "stage"
 // of the activation and decoded-weight rings is two k-blocks (256 codes of K); a packed stage
