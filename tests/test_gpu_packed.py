@@ -86,3 +86,35 @@ def test_linear_packed_matches_int8_linear(bl):
     torch.cuda.synchronize()
     assert torch.equal(acc8, accp)
     assert torch.equal(y8.view(torch.int16), yp.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,K,N", [(17, 1024, 272), (64, 4096, 11008), (100, 640, 4112), (256, 512, 1040),
+                                   (40, 256, 40000)])
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_linear_packed_without_accumulators(bl, T, K, N, out):
+    """Y alone (no int32 copy requested): the CTA-pair epilogue stages bf16 output in four 2 KB
+    tiles per warp instead of two 4 KB ones; Y must equal the path with the copy bit for bit."""
+    xq, packed, s = _case(T, K, N, seed=3 * T + K)
+    args = (_gpu(xq), _gpu(s), _gpu(packed), _gpu(torch.tensor([0.0173])), K)
+    dt = torch.bfloat16 if out == "bf16" else torch.float32
+    y_only, none = bl.bitlinear_linear_packed(*args, out_dtype=dt)
+    assert none is None
+    y, acc = bl.bitlinear_linear_packed(*args, out_dtype=dt, want_acc=True)
+    torch.cuda.synchronize()
+    assert bl.check_device_status() == 0
+    assert torch.equal(y_only.view(torch.int16 if out == "bf16" else torch.int32),
+                       y.view(torch.int16 if out == "bf16" else torch.int32))
+    rows = sample_rows(T, 6, seed=T)
+    acc_o = oracle.int_gemm(xq, oracle.unpack(packed, K), rows=rows)
+    y_o = oracle.linear_epilogue(acc_o, 0.0173, s[rows])
+    assert np.array_equal(np_(y_only)[rows], oracle.round_bf16(y_o) if out == "bf16" else y_o)
+
+
+def test_linear_packed_split_with_single_k_block_stages(bl):
+    """K = 5440 (42.5 k-blocks) at 20 tokens on 512 rows: two pair tiles, so K is split -- three
+    ways by the launcher's rule (14 / 14 / 15 k-blocks); the last split ends in a one-k-block
+    stage, the half k-block of the K tail."""
+    xq, packed, s = _case(20, 5440, 512, seed=11)
+    for out in ("bf16", "f32"):
+        _check(bl, xq, packed, s, 0.0173, out, True)
+        _check(bl, xq, packed, s, 0.0173, out, False)
