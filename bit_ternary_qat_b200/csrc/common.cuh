@@ -123,6 +123,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// The same wait by every lane of a warp, decided for the whole warp: after a timeout no lane
+// goes on alone into the warp-wide (.sync.aligned) instructions that follow.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                               volatile int* abort) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns, abort));
+}
+
 // ------------------------------------------------------------------------------------
 // TMA (bulk tensor copies, global -> shared), no multicast.
 // ------------------------------------------------------------------------------------

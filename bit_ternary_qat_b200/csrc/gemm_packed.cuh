@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kPkThreads, 1)
             int nt, tt, kb0, kb1;
             unit_of(u, nt, tt, kb0, kb1);
             for (int kb = kb0; kb < kb1 && ok; kb += kPkKbPerP) {
-                if (!mbar_wait(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
                 const uint8_t* src = sP(p);
                 const int nkb = min(kPkKbPerP, kb1 - kb);
                 for (int j = 0; j < nkb; ++j, ++q) {
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kPkThreads, 1)
                     const int ds = q % DS;                      // grp, or grp + 4 on alternate turns
                     const int li = ds / kPkDecGroups;
                     // the MMA has finished with this decoded stage (its previous use)
-                    if (!mbar_wait(&dempty[ds], dph[li] ^ 1u, lim, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_warp(&dempty[ds], dph[li] ^ 1u, lim, abort_flag)) { ok = false; break; }
                     uint8_t* a = sA(ds);
                     // 16-byte chunk (2 j + c / 4) of row r sits at chunk (2 j + c / 4) ^ (r & 7)
                     const int src_off = ((((2 * j + (c >> 2)) ^ (r0 & 7)) << 4) | ((c & 3) << 2));
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kPkThreads, 1)
             unit_of(u, nt, tt, kb0, kb1);
             const int b = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
-            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            if (!mbar_wait_warp(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
             const int n = nt * kPkBM + quad * 32 + lane;
             const bool n_ok = n < args.N;

@@ -398,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
             int nt, tt, kb0, kb1;
             unit_of(u, nt, tt, kb0, kb1);
             for (int kb = kb0; kb < kb1 && ok; kb += kPkKbPerP) {
-                if (!mbar_wait(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(&pfull[p], pph, lim, abort_flag)) { ok = false; break; }
                 const uint8_t* src = sP(p) + row * 128;
                 for (int h = 0; h < kPkKbPerP / kPk2KbPerStage; ++h) {
                     const int ks = kb + h * kPk2KbPerStage;
@@ -406,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                     if ((q & (kPkDecGroups - 1)) == grp) {
                         const int nkb = min(kPk2KbPerStage, kb1 - ks);
                         // the MMA has finished reading this stage in both CTAs (its previous use)
-                        if (!mbar_wait(&dempty[grp], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait_warp(&dempty[grp], dph ^ 1u, lim, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         for (int j = 0; j < nkb; ++j) {
                             // k-block 2 h + j of the packed stage: the row's 16-byte chunks 2 jj, 2 jj + 1
@@ -454,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 const float cl0 = token_factor(gm, t0 + 32 * i0 + lane);
                 const float cl1 = 32 * i1 < bt ? token_factor(gm, t0 + 32 * i1 + lane) : 0.0f;
                 const int b = last % nacc;
-                if (mbar_wait(&tfull[b], (last / nacc) & 1, lim, abort_flag)) {
+                if (mbar_wait_warp(&tfull[b], (last / nacc) & 1, lim, abort_flag)) {
                     tc_fence_after();
                     uint8_t* hbuf = smem + (warp - 6) * 2 * kPk2EpiBuf;
                     int hbi = 0;
@@ -535,7 +535,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
 #pragma unroll
             for (int i = 0; i < kPkMaxBT / 32; ++i)
                 fac[i] = (32 * i < bt && i % step == 0) ? token_factor(gm, t0 + 32 * i + lane) : 0.0f;
-            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            if (!mbar_wait_warp(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(b * 128);
 #pragma unroll 1

@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
             const int b = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
-            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            if (!mbar_wait_warp(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
             const int mb = tile % args.m_tiles;
             const int nb = tile / args.m_tiles;
@@ -556,7 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
         for (int u = pair; u < plan.num_units; u += npairs, ++tcount) {
             const int b = tcount & 1;
             const uint32_t tph = (tcount >> 1) & 1;
-            if (!mbar_wait(&tfull[b], tph, lim, abort_flag)) break;
+            if (!mbar_wait_warp(&tfull[b], tph, lim, abort_flag)) break;
             tc_fence_after();
             int mb, nb, half;
             tc2_unit(u, plan, args.m_tiles, args.n_tiles, mb, nb, half);
