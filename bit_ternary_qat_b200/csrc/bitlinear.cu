@@ -544,69 +544,8 @@ inline double wave_eff(int64_t units, int sms) {
     return static_cast<double>(units) / static_cast<double>(waves * sms);
 }
 
-template <bool kBf16Out>
-bl_status launch_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
-                        const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch, size_t scratch_bytes,
-                        cudaStream_t st, const DeviceInfo& dev) {
-    bl::PkArgs a{};
-    a.T = (int)T; a.N = (int)N; a.K = (int)K;
-    int64_t bt = (T + 15) / 16 * 16;
-    if (bt > bl::kPkMaxBT) bt = bl::kPkMaxBT;
-    a.bt = (int)bt;
-    a.t_tiles = (int)((T + bt - 1) / bt);
-    a.n_tiles = (int)((N + bl::kPkBM - 1) / bl::kPkBM);
-    a.k_blocks = (int)((K + 127) / 128);
-    // K split: only for a narrow token tile (bt <= 64), with a workspace for the int32 partial
-    // sums (splits x T x N), at least two k-blocks per unit, and partial-sum bytes at most a
-    // quarter of the packed weight bytes (splits <= K / (64 T)); the smallest split whose last
-    // wave is within 3 % of the best
-    const int64_t base = (int64_t)a.n_tiles * a.t_tiles;
-    int splits = 1;
-    if (bt <= 64) {
-        int smax = std::min<int64_t>(8, a.k_blocks / 2);
-        smax = (int)std::min<int64_t>(smax, K / (64 * T));
-        smax = (int)std::min<int64_t>(smax, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));
-        double best = wave_eff(base, dev.sms);
-        for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, dev.sms));
-        for (int sp = 1; sp <= std::max(1, smax); ++sp)
-            if (wave_eff(base * sp, dev.sms) >= best - 0.03) { splits = sp; break; }
-    }
-    a.splits = splits;
-    const size_t budget = (size_t)dev.max_smem_optin;
-    // rings: 8 decoded and 8 activation stages for token tiles of up to 32 (4 for wider
-    // tiles, whose activation stages are larger); the packed ring (16 KB stages, 512 codes per
-    // row) takes the rest of shared memory (at most 12 stages)
-    const int dstages = (bt <= 32 && bl::pk_smem_bytes((int)bt, 4, 2 * bl::kPkDecGroups) <= budget)
-                            ? 2 * bl::kPkDecGroups : bl::kPkDecGroups;
-    int pstages = (int)((budget - bl::pk_smem_bytes((int)bt, 0, dstages)) / bl::kPkPBytes);
-    pstages = std::min(pstages, bl::kPkMaxPStages);
-    BL_REQUIRE(pstages >= 2, BL_ERR_DEVICE, "packed GEMM: shared memory too small");
-    a.pstages = pstages;
-    a.sx = sx; a.gamma = gamma; a.y = Y;
-    a.acc = splits > 1 ? scratch : acc;
-    a.wait_ns = g_wait_ns.load();
-    CUtensorMap tp, tx;
-    BL_TRY(make_tmap(&tp, Wpacked, kTmU8, (uint64_t)(K / 4), (uint64_t)N, 128, bl::kPkBM));
-    BL_TRY(make_tmap(&tx, Xq, kTmU8, (uint64_t)K, (uint64_t)T, 128, (uint32_t)bt));
-    auto kern = dstages == 2 * bl::kPkDecGroups ? bl::tc_gemm_packed_kernel<kBf16Out, 2 * bl::kPkDecGroups>
-                                                : bl::tc_gemm_packed_kernel<kBf16Out, bl::kPkDecGroups>;
-    const size_t smem = bl::pk_smem_bytes((int)bt, pstages, dstages);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(BL_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-    const int64_t units = base * splits;
-    const unsigned grid = (unsigned)std::min<int64_t>(units, dev.sms);
-    pdl_launch(kern, dim3(grid), dim3(bl::kPkThreads), smem, st, tp, tx, a);
-    BL_TRY(launched("tc_gemm_packed"));
-    if (splits > 1) {
-        const int64_t nv = T * N / 4;
-        pdl_launch(bl::pk_finalize_kernel<kBf16Out>, dim3((unsigned)std::min<int64_t>((nv + 255) / 256, (int64_t)dev.sms * 8)),
-                   dim3(256), 0, st, static_cast<const int32_t*>(scratch), splits, sx, gamma, (int)T, (int)N, Y, acc);
-        BL_TRY(launched("pk_finalize"));
-    }
-    return BL_OK;
-}
 
-// Packed-weight GEMM on CTA pairs (17 or more tokens): 256-row weight tiles x bt tokens
+// Packed-weight GEMM on CTA pairs: 256-row weight tiles x bt tokens
 // (bt = T rounded up to 32, at most 256), the same K-split rule as the 1-SM kernel counted
 // in pairs, the activation ring, and the packed ring in the rest of shared memory.  The grid
 // is as many pairs as fit at once, at most one per unit.
@@ -1206,16 +1145,11 @@ bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, 
                           : launch_gemv<2, false>(Wpacked, gamma, 0, N, K, Xq, sx, T, Y, acc, st, dev);
         }
     }
-    // 17 tokens or more: 2-SM tiles of 256 weight rows (M = 256 MMAs move about 1.6x more
-    // weight codes per SM per cycle than 1-SM tiles at these widths)
-    if (T > 16) {
-        if (y_dt == BL_BF16)
-            return launch_packed2<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
-        return launch_packed2<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
-    }
+    // Otherwise (17 tokens or more, or rows too long for the GEMV): 2-SM tiles of 256 weight
+    // rows with the decoded codes in tensor memory
     if (y_dt == BL_BF16)
-        return launch_packed<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
-    return launch_packed<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
+        return launch_packed2<true>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
+    return launch_packed2<false>(Xq, sx, T, K, Wpacked, gamma, N, Y, acc, scratch, scratch_bytes, st, dev);
 }
 
 // ------------------------------------------------------------------------------------

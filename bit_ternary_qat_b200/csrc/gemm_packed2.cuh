@@ -1,7 +1,8 @@
 // gemm_packed2.cuh -- int8 x packed-ternary linear on CTA pairs (tcgen05.mma.cta_group::2 with
-// the weight operand in tensor memory) for 17 or more tokens.
+// the weight operand in tensor memory): 17 or more tokens, or fewer when their activation rows
+// do not fit the decode GEMV's shared memory.
 //
-// The same contraction as gemm_packed.cuh (P3 §3.1's linear on P5 §4.1 / §5.1 2-bit codes):
+// P3 §3.1's linear on the 2-bit codes of P5 §4.1 / §5.1:
 //   D[n, t] = sum_k W_q[n, k] x_q[t, k],   y[t, n] = fl(D * fl(gamma / s_t)),
 // with the weight rows as the MMA's M dimension.  A cluster of two CTAs computes a tile of 256
 // weight rows x bt tokens (bt = 32 ... 256) with one 2-SM instruction per 32 codes of K.

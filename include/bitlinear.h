@@ -314,9 +314,8 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
  * Kernels by token count:
  *   up to 16 tokens, when their activation rows fit one block's shared memory: the decode
  *     GEMV's kernel (codes decoded in registers, warp-level int8 MMA; ws unused);
- *   17 tokens or more: CTA pairs with 256 weight rows x up to 256 tokens per tile (codes
- *     decoded into tensor memory, 2-SM tcgen05 MMAs, TMA-stored output);
- *   other cases of up to 16 tokens: a 1-SM tensor-core tile.
+ *   otherwise: CTA pairs with 256 weight rows x up to 256 tokens per tile (codes decoded
+ *     into tensor memory, 2-SM tcgen05 MMAs, TMA-stored output).
  * When the weight tiles alone cannot fill the GPU and at most 64 tokens are given, K may be
  * split: split sp stores its exact int32 partial sums to slice sp of ws (int32
  * [splits x T x N]) and a second launch adds the slices in split order and applies the

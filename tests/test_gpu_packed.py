@@ -1,7 +1,7 @@
-"""GPU parity of the int8 x packed-ternary linear (few tokens) against the oracle, on each of
-its three kernels: the decode GEMV's (up to 16 tokens), the 1-SM tensor-core tile (up to 16
-tokens when the GEMV's activation rows do not fit shared memory) and the 2-SM tile on CTA
-pairs (17 tokens or more; 256 weight rows x up to 256 tokens, ragged in rows, tokens and K).
+"""GPU parity of the int8 x packed-ternary linear (few tokens) against the oracle, on both of
+its kernels: the decode GEMV's (up to 16 tokens) and the 2-SM tile on CTA pairs (17 tokens or
+more, and up to 16 tokens whose activation rows do not fit the GEMV's shared memory, such as
+16 x 65536; 256 weight rows x up to 256 tokens, ragged in rows, tokens and K).
 
 The accumulators are exact int32 and compared bit for bit with the oracle's contraction of
 the unpacked codes (reserved code 11 decodes to 0); Y = fl(acc * fl(gamma / s_t)) is

@@ -234,25 +234,29 @@ def test_packed_gemm_decoder_matches_code_table():
 
 
 def test_packed_gemm_decoder_addresses():
-    """The packed linear's decoder (4 groups x 128 threads; thread dt owns word c = dt % 8 of
-    rows dt / 8 + 16 i) reads each 32-bit word of k-block j of a 128-byte-swizzled packed
-    stage exactly once and writes each 16-byte chunk of the int8 tile exactly once, at the
-    position the 128-byte swizzle gives it (chunk c of row r at chunk c ^ (r % 8))."""
-    for j in range(4):
-        reads, writes = {}, {}
-        for dt in range(128):
-            c, r0 = dt & 7, dt >> 3
-            src_off = ((((2 * j + (c >> 2)) ^ (r0 & 7)) << 4) | ((c & 3) << 2))
-            dst_off = (c ^ (r0 & 7)) << 4
-            for i in range(8):
-                r = r0 + 16 * i
-                assert r & 7 == r0 & 7
-                # logical word c of k-block j of row r: bytes 32 j + 4 c of the 128-byte row,
-                # i.e. chunk 2 j + c // 4, stored at chunk (2 j + c // 4) ^ (r % 8)
-                logical_chunk = 2 * j + (c >> 2)
-                assert src_off == ((logical_chunk ^ (r % 8)) << 4) | ((c & 3) << 2)
-                reads[(r, c)] = reads.get((r, c), 0) + 1
-                assert dst_off == ((c ^ (r % 8)) << 4)
-                writes[(r, dst_off)] = writes.get((r, dst_off), 0) + 1
-        assert len(reads) == 128 * 8 and set(reads.values()) == {1}
-        assert len(writes) == 128 * 8 and set(writes.values()) == {1}
+    """The pair kernel's decoders: a group of four warps (warps 6 + 4 g .. 9 + 4 g) covers the
+    four TMEM lane quarters (warp % 4), so thread (warp, lane) owns weight row
+    32 (warp % 4) + lane.  For k-block jj of a 128-byte-swizzled packed stage it reads the row's
+    logical 16-byte chunks 2 jj and 2 jj + 1 at chunk (c ^ (row % 8)); over the stage's four
+    k-blocks every physical chunk of every row is read exactly once, and word i of a k-block
+    (codes 16 i .. 16 i + 15) lands in TMEM columns 4 i .. 4 i + 3 of that k-block's 32."""
+    for g in range(4):
+        rows = sorted(32 * (w % 4) + lane for w in range(6 + 4 * g, 10 + 4 * g) for lane in range(32))
+        assert rows == list(range(128))
+    reads = {}
+    for row in range(128):
+        sw = row & 7
+        for jj in range(4):
+            for half in range(2):
+                logical = 2 * jj + half
+                phys = logical ^ sw
+                assert 0 <= phys < 8
+                reads[(row, phys)] = reads.get((row, phys), 0) + 1
+                # the 16 bytes of this chunk are words 4 half .. 4 half + 3 of k-block jj; word
+                # q covers codes 16 q .. 16 q + 15 and goes to columns 4 q .. 4 q + 3
+                for q in range(4 * half, 4 * half + 4):
+                    byte0 = 32 * jj + 4 * q                  # byte of the logical packed row
+                    assert byte0 // 16 == logical
+                    assert [4 * q + e for e in range(4)] == list(range(4 * q, 4 * q + 4))
+    assert len(reads) == 128 * 8 and set(reads.values()) == {1}
+
