@@ -75,8 +75,7 @@ __host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages) {
 }
 
 // TMA load of one 2-D box with an L2 evict-first policy: the packed weight is read once per
-// launch, and keeping it from evicting the activations and the kernel's own code from L2 shortens
-// the start of the next launch.
+// launch, so it should not displace the activations (read by every weight tile) from L2.
 __device__ __forceinline__ void tma_load_2d_evict_first(void* smem_dst, const void* desc, uint64_t* bar, int32_t x,
                                                         int32_t y) {
     asm volatile(
