@@ -33,15 +33,18 @@
 //              producer);
 //   warp 1     leader only: one thread issues tcgen05.mma.cta_group::2.kind::i8 (eight per stage)
 //              with A from both CTAs' TMEM stage and B from both CTAs' activation halves; its
-//              commit frees the stage in both CTAs (TMEM and activation tile), and after a unit's
-//              last stage another arrives on both CTAs' accumulator-full barriers;
+//              commit frees the stage in both CTAs (TMEM and activation tile), after a unit's
+//              last stage another arrives on both CTAs' accumulator-full barriers, and after
+//              the pair's last unit a third arrives on a barrier used once;
 //   warps 2-5  epilogue (both CTAs): TMEM lanes are the CTA's 128 weight rows; the unit's token
 //              factors fl(gamma / s_t) are read before its accumulators are ready; per 32-token
 //              chunk tcgen05.ld, y[t, n] = fl(acc * fl(gamma / s_t)) staged in shared memory as a
 //              [token][row] tile and written with one TMA store (or the exact int32 partial sums
 //              of K split sp into slice sp of a workspace, which pk_finalize_kernel adds in split
 //              order); one arrival per warp on the leader's accumulator-empty barrier.  For the
-//              pair's last unit the decoder warps, idle by then, take four of every five chunks.
+//              pair's last unit the decoder warps, idle by then, take four of every five chunks;
+//              they wait on the once-used barrier (they can run ahead of the accumulator-full
+//              phases, where a parity wait would take an earlier unit's phase for the last's).
 // The single-thread MMA loop's barrier waits (about 130 cycles each, measured, even on a completed
 // phase) and commits cost about as much as the MMAs themselves at these widths: two k-blocks per
 // stage and one barrier per stage keep them to one wait and one commit per 8 MMAs.
@@ -71,7 +74,7 @@ constexpr int kPk2EpiHelpers = 5;      // warps per TMEM quarter sharing a pair'
 
 __host__ __device__ inline size_t pk2_smem_bytes(int bt, int pstages) {
     return 1024 + static_cast<size_t>(pstages) * kPkPBytes + static_cast<size_t>(kPk2DStages) * static_cast<size_t>(bt) * 128 +
-           kPk2EpiBytes + (2 * kPkMaxPStages + 2 * kPk2DStages + 4) * sizeof(uint64_t) + 16;
+           kPk2EpiBytes + (2 * kPkMaxPStages + 2 * kPk2DStages + 5) * sizeof(uint64_t) + 16;
 }
 
 // TMA load of one 2-D box with an L2 evict-first policy: the packed weight is read once per
@@ -199,7 +202,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
     uint64_t* dempty = dfull + DS;
     uint64_t* tfull = dempty + DS;               // each CTA: the leader's commit after a unit
     uint64_t* tempty = tfull + 2;                // leader's is used: 4 epilogue warps per CTA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    // each CTA, used once: the leader's commit after the pair's last unit.  The decoder warps
+    // wait on it, not on tfull: they may reach the last unit while a unit two or more commits
+    // earlier is still open, and a parity wait cannot tell that phase from the one it wants.
+    uint64_t* tlast = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tlast + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -219,6 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
             mbar_init(&tfull[b], 1);
             mbar_init(&tempty[b], 8);
         }
+        mbar_init(tlast, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -454,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 const float cl0 = token_factor(gm, t0 + 32 * i0 + lane);
                 const float cl1 = 32 * i1 < bt ? token_factor(gm, t0 + 32 * i1 + lane) : 0.0f;
                 const int b = last % nacc;
-                if (mbar_wait_warp(&tfull[b], (last / nacc) & 1, lim, abort_flag)) {
+                if (mbar_wait_warp(tlast, 0, lim, abort_flag)) {
                     tc_fence_after();
                     uint8_t* hbuf = smem + (warp - 6) * 2 * kPk2EpiBuf;
                     int hbi = 0;
@@ -509,9 +517,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPk2Threads, 1)
                 if (!ok) break;
                 tc_commit_pair(&tfull[b], 0x3);
             }
+            // completes when every MMA of the pair is done (after a timeout too, so that the
+            // bounded wait below outlasts the MMAs in flight before TMEM is freed)
+            tc_commit_pair(tlast, 0x3);
             if (!ok) {
-                tc_commit_pair(&tfull[tcount % nacc], 0x3);
-                mbar_wait(&tfull[tcount % nacc], (tcount / nacc) & 1, 100000000ull, nullptr);
+                tc_commit_pair(&tfull[tcount % nacc], 0x3);   // releases the epilogue warps
+                mbar_wait(tlast, 0, 100000000ull, nullptr);
             }
         }
         __syncwarp();

@@ -110,6 +110,25 @@ def test_linear_packed_without_accumulators(bl, T, K, N, out):
     assert np.array_equal(np_(y_only)[rows], oracle.round_bf16(y_o) if out == "bf16" else y_o)
 
 
+@pytest.mark.parametrize("T,K,N", [(256, 512, 20480), (200, 1024, 40000), (64, 256, 40000)])
+def test_linear_packed_short_last_units(bl, T, K, N):
+    """More weight tiles than CTA pairs, with short units (one, two or four stages of two
+    k-blocks): a pair's decoder warps finish decoding its last unit while an earlier unit's
+    accumulators are still open, and then take part in the last unit's epilogue.  One 256-column
+    accumulator (200 and 256 tokens) or two (64 tokens).  Every token is checked on the first
+    weight tile and on the last 4096 rows, which hold the pairs' second and third units."""
+    xq, packed, s = _case(T, K, N, seed=T + K + N)
+    gamma = 0.0173
+    y, acc = bl.bitlinear_linear_packed(_gpu(xq), _gpu(s), _gpu(packed), _gpu(torch.tensor([gamma])), K,
+                                        want_acc=True)
+    torch.cuda.synchronize()
+    assert bl.check_device_status() == 0
+    sel = np.r_[0:256, N - 4096:N]
+    acc_o = oracle.int_gemm(xq, oracle.unpack(packed[sel], K))
+    assert np.array_equal(np_(acc)[:, sel], acc_o)
+    assert np.array_equal(np_(y)[:, sel], oracle.round_bf16(oracle.linear_epilogue(acc_o, gamma, s)))
+
+
 def test_linear_packed_split_with_single_k_block_stages(bl):
     """K = 5440 (42.5 k-blocks) at 20 tokens on 512 rows: two pair tiles, so K is split -- three
     ways by the launcher's rule (14 / 14 / 15 k-blocks); the last split ends in a one-k-block
