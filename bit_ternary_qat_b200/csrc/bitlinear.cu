@@ -604,6 +604,14 @@ bl_status launch_packed2(const int8_t* Xq, const float* sx, int64_t T, int64_t K
         for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, mc));
         for (int sp = 1; sp <= std::max(1, smax); ++sp)
             if (wave_eff(base * sp, mc) >= best - 0.03) { splits = sp; break; }
+    } else if (2 * base <= mc) {
+        // wider token tiles: the partial sums cost more than a second wave returns, so split only
+        // when the tiles fill at most half the pairs, into as many units as one wave holds, each
+        // at least 8 k-blocks (4 stages) long
+        int64_t sp = std::min<int64_t>(8, (int64_t)mc / base);
+        sp = std::min<int64_t>(sp, a.k_blocks / 8);
+        sp = std::min<int64_t>(sp, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));
+        splits = (int)std::max<int64_t>(1, sp);
     }
     a.splits = splits;
     a.sx = sx; a.gamma = gamma; a.y = Y;

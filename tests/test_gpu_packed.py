@@ -61,7 +61,8 @@ def _check(bl, xq, packed, s, gamma, out, split):
                                    (129, 1024, 400), (300, 512, 1040), (33, 192, 2064), (8, 2048, 400),
                                    (3, 1024, 272), (32, 4096, 2048), (20, 1024, 400), (16, 65536, 64),
                                    (17, 1024, 272), (96, 640, 512), (200, 1088, 1008), (257, 512, 608),
-                                   (40, 256, 40000), (64, 4096, 11008), (256, 4096, 11008)])
+                                   (40, 256, 40000), (64, 4096, 11008), (256, 4096, 11008),
+                                   (256, 4096, 4096), (192, 4096, 4096), (100, 2048, 1024)])
 @pytest.mark.parametrize("out", ["bf16", "f32"])
 @pytest.mark.parametrize("split", [False, True])
 def test_linear_packed_parity(bl, T, K, N, out, split):
