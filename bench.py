@@ -1030,12 +1030,75 @@ def gemv_measure(bl, torch, dev, flush, pk, imma_peak=None):
         rec["marginal_GB/s"] = (N * K // 4) / (extra * 1e-6) / 1e9 if extra > 0 else None
         rec["marginal_frac_hbm"] = rec["marginal_GB/s"] / pk["hbm"] if rec["marginal_GB/s"] else None
         rec["fixed_us"] = rec["us"] - extra
+
+    def graph_us(call, flush_first=True):
+        """us per launch of `reps` launches call(0..reps-1) in one CUDA graph, median of 5."""
+        for i in range(8):
+            call(i)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(reps):
+                call(i)
+        graph.replay()
+        samples = []
+        for _ in range(5):
+            if flush_first:
+                flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            samples.append(a.elapsed_time(b) / reps)
+        del graph
+        return statistics.median(samples) * 1e3
+
+    # the read-only ceiling of the same bytes, read the same way and chained the same way (the
+    # library's read probe: no arithmetic), on the same weight copies and the 2x-tall ones
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    wbytes = N * K // 4
+    ceiling = {}
+    for pat in ("gemv", "coalesced"):
+        u1 = graph_us(lambda i: bl.read_peak_probe(packs[i % copies], pat, sink))
+        u2 = graph_us(lambda i: bl.read_peak_probe(packs2[i % 2], pat, sink))
+        ceiling[pat] = {"us": u1, "GB/s": wbytes / (u1 * 1e-6) / 1e9, "frac_hbm": wbytes / (u1 * 1e-6) / 1e9 / pk["hbm"],
+                        "marginal_GB/s": wbytes / ((u2 - u1) * 1e-6) / 1e9 if u2 > u1 else None,
+                        "fixed_us": 2 * u1 - u2}
+    assert bl.check_device_status() == 0
+    out["read_ceiling"] = ceiling
+    for B in (1, 4, 16):
+        out[f"B{B}"]["frac_of_read_ceiling"] = ceiling["gemv"]["us"] / out[f"B{B}"]["us"]
     del packs2, q2
+
+    # the GEMV's loop with the weight resident in L2 (one 4736- or 14208-row weight, 9.7 or
+    # 29.1 MB, reused by every launch): the marginal time per 28672 rows is its
+    # instruction-bound rate, to set beside the streaming rate above
+    small = {}
+    for n in (4736, 14208):
+        Wn, _ = synth.decode_inputs(1, n, K, seed=45)
+        small[n] = bl.bitlinear_quant_weight(Wn.to(dev), want_i8=False, want_bf16=False)
+        del Wn
+    for B in (1, 4, 16):
+        _, x = synth.decode_inputs(B, 16, K, seed=40 + B)
+        aq = bl.bitlinear_act_quant(x.to(dev), apply_rmsnorm=False, want_xdq=False)
+        t = {}
+        for n in (4736, 14208):
+            y = torch.empty(B, n, dtype=torch.float32, device=dev)
+            qn = small[n]
+            t[n] = graph_us(lambda i: bl.ternary_gemv(qn["packed"], qn["gamma"], K, aq["xq"], aq["sx"], y=y),
+                            flush_first=False)
+        out[f"B{B}"]["l2_resident_us_per_28672_rows"] = (t[14208] - t[4736]) / (14208 - 4736) * N
+    del small
     out["hbm_peak_GBs"] = pk["hbm"]
     out["imma_peak_T"] = imma_peak
     out["workload"] = ("decode: packed W 28672x8192 (58.7 MB), int8 x [B x 8192]; 4 weight copies cycled "
                        "(inputs larger than L2), 40 launches in one CUDA graph per event pair, median of 5; "
-                       "marginal rate and fixed cost from the same launches on a 57344x8192 weight (2 copies)")
+                       "marginal rate and fixed cost from the same launches on a 57344x8192 weight (2 copies); "
+                       "read_ceiling: the library's read probe on the same copies (the GEMV's partition and a "
+                       "coalesced one, no arithmetic); l2_resident: the GEMV on 4736- and 14208-row weights "
+                       "reused by every launch")
     return out
 
 

@@ -14,7 +14,7 @@ from .ops import (  # noqa: F401
     bitlinear_quant_weight_noalloc, check_device_status, launch_count,
     selftest_bounded_wait, set_wait_limit_ns, ternary_gemv, ternary_pack, workspace, workspace_bytes,
     bitlinear_act_quant_tensor, bitlinear_linear_rows, bitlinear_quant_weight_rows, bitlinear_quant_weight_tau,
-    ternary_gemv_rows, bitlinear_optimizer_step, bitlinear_linear_packed, mma_peak_probe,
+    ternary_gemv_rows, bitlinear_optimizer_step, bitlinear_linear_packed, mma_peak_probe, read_peak_probe,
 )
 
 

@@ -51,6 +51,7 @@ SIGNATURES = {
     "ternary_gemv": (INT, [P, P, I64, I64, P, P, I64, P, P, P]),
     "bl_selftest_bounded_wait": (INT, [U64, P]),
     "bl_mma_peak_probe": (INT, [INT, INT, INT, P, P]),
+    "bl_read_peak_probe": (INT, [P, I64, I64, INT, P, P]),
     "bitlinear_quant_weight_rows": (INT, [P, I64, I64, P, P, P, P, P]),
     "bitlinear_quant_weight_tau": (INT, [P, I64, I64, F, P, P, P, P, P, SZ, P]),
     "bitlinear_act_quant_tensor": (INT, [P, INT, I64, I64, INT, P, F, P, P, P, P, P, SZ, P]),

@@ -26,6 +26,7 @@
 #include "gemm_packed.cuh"
 #include "gemm_packed2.cuh"
 #include "mma_peak.cuh"
+#include "read_peak.cuh"
 
 // Scratch of bitlinear_quant_weight_noalloc: the pass-1 partial sums of |W| live in this
 // file-scope device array instead of a caller workspace.  Every device that loads the
@@ -1263,6 +1264,32 @@ bl_status bl_mma_peak_probe(int kind, int pair, int iters, double* ops_out, void
     if (ops_out) *ops_out = units * 4.0 * (double)iters * per_instr;
     pdl_launch(kern, dim3((unsigned)ctas), dim3(bl::kPeakThreads), (size_t)bl::kPeakSmemBytes, st, iters, wait_ns);
     return launched("mma_peak");
+}
+
+bl_status bl_read_peak_probe(const uint8_t* buf, int64_t rows, int64_t row_bytes, int pattern, uint32_t* sink,
+                             void* stream) {
+    BL_TRY(check_ptr(buf, "buf", true));
+    BL_TRY(check_ptr(sink, "sink", true));
+    BL_REQUIRE(pattern == 0 || pattern == 1, BL_ERR_INVALID_ARG, "pattern must be 0 (GEMV) or 1 (coalesced), got %d",
+               pattern);
+    BL_REQUIRE(rows >= 16 && rows % 16 == 0 && rows <= (1 << 30), BL_ERR_UNSUPPORTED_SHAPE,
+               "rows must be a positive multiple of 16 (at most 2^30), got %lld", (long long)rows);
+    BL_REQUIRE(row_bytes >= 64 && row_bytes % 64 == 0 && row_bytes <= (1 << 24), BL_ERR_UNSUPPORTED_SHAPE,
+               "row_bytes must be a positive multiple of 64 (at most 2^24), got %lld", (long long)row_bytes);
+    DeviceInfo dev;
+    BL_TRY(current_device(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n_rg = rows / 16;
+    if (pattern == 0) {
+        // as the GEMV: one block per SM, at most one per row group
+        const unsigned nb = (unsigned)std::min<int64_t>(n_rg, dev.sms);
+        pdl_launch(bl::read_peak_gemv_kernel, dim3(nb), dim3(bl::kReadWarps * 32), 0, st, buf, (int)rows,
+                   (int)row_bytes, sink);
+    } else {
+        pdl_launch(bl::read_peak_coalesced_kernel, dim3((unsigned)dev.sms), dim3(bl::kReadWarps * 32), 0, st,
+                   reinterpret_cast<const uint4*>(buf), rows * row_bytes / 16, sink);
+    }
+    return launched("read_peak");
 }
 
 bl_status bl_selftest_bounded_wait(uint64_t limit_ns, void* stream) {

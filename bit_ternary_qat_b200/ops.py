@@ -457,6 +457,19 @@ def selftest_bounded_wait(limit_ns: int, device=None) -> None:
     _lib.call("bl_selftest_bounded_wait", int(limit_ns), _stream(dev))
 
 
+def read_peak_probe(buf: torch.Tensor, pattern: str = "gemv", sink: Optional[torch.Tensor] = None) -> int:
+    """Launch the read-bandwidth probe on buf (uint8 [rows x row_bytes], rows a multiple of 16,
+    row_bytes of 64) on the current stream; returns the bytes the launch reads.  Time it with
+    CUDA events for the rate."""
+    _cuda(buf, "buf", torch.uint8)
+    rows, row_bytes = buf.shape
+    if sink is None:
+        sink = torch.zeros(4, dtype=torch.int32, device=buf.device)
+    _lib.call("bl_read_peak_probe", buf.data_ptr(), rows, row_bytes, {"gemv": 0, "coalesced": 1}[pattern],
+              sink.data_ptr(), _stream(buf.device))
+    return rows * row_bytes
+
+
 def mma_peak_probe(kind: str = "int8", pair: bool = True, iters: int = 20000, device=None) -> float:
     """Launch the tensor-pipe peak probe on the current stream (tcgen05.mma from fixed
     shared-memory operands, no global traffic).  Returns 2 x the multiply-adds of the

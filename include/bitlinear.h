@@ -367,6 +367,20 @@ BL_API bl_status bitlinear_optimizer_step(float* W, const float* dW, float* m, f
 BL_API bl_status bl_mma_peak_probe(int kind, int pair, int iters, double* ops_out, void* stream);
 
 /* ------------------------------------------------------------------------------
+ * Read-bandwidth probe (a measurement kernel with no counterpart on the pages): one launch
+ * that reads every byte of buf, a [rows x row_bytes] uint8 device array, once and does no
+ * arithmetic with it, giving the read-only ceiling against which the decode GEMV's weight
+ * stream is judged.  pattern 0 reads it as the decode GEMV reads a packed weight (one block
+ * per SM, balanced 16-row groups, 64-byte column steps, 8 rows x 64 bytes per warp load);
+ * pattern 1 reads contiguous equal spans per block, 512 bytes per warp load.  rows: a
+ * positive multiple of 16 (at most 2^30); row_bytes: a positive multiple of 64 (at most
+ * 2^24); buf 16-byte aligned.  sink: one device uint32 that the kernel writes only if the
+ * XOR of all loads equals a fixed constant (the buffer's owner may ignore it).  Launched with
+ * programmatic dependent launch like the GEMV; time it with CUDA events on `stream`. */
+BL_API bl_status bl_read_peak_probe(const uint8_t* buf, int64_t rows, int64_t row_bytes, int pattern, uint32_t* sink,
+                                    void* stream);
+
+/* ------------------------------------------------------------------------------
  * Self-test of the bounded-wait machinery: launches one block that waits on an
  * mbarrier nothing arrives on, with the given limit (ns), and returns.  Afterwards
  * bl_check_device_status() must report BL_ERR_TIMEOUT.  No counterpart on the pages. */

@@ -181,6 +181,21 @@ def test_status_values_match_header():
     assert {v: k for k, v in vals.items()} == _lib.STATUS_NAMES
 
 
+@pytest.mark.parametrize("rows,row_bytes,pattern,status", [(16, 64, 2, 1), (16, 64, -1, 1), (8, 64, 0, 2), (24, 64, 1, 2),
+                                                         (16, 32, 0, 2), (16, 96, 0, 2), (0, 64, 0, 2)])
+def test_read_probe_validation(L, rows, row_bytes, pattern, status):
+    """The read probe rejects a bad pattern or shape before touching the (fake, aligned) pointers."""
+    fake = 1 << 20
+    assert _lib.status("bl_read_peak_probe", fake, rows, row_bytes, pattern, fake, None) == status
+    assert len(_lib.last_error()) > 0
+
+
+def test_read_probe_null_and_misaligned(L):
+    assert _lib.status("bl_read_peak_probe", None, 16, 64, 0, 1 << 20, None) == 1
+    assert _lib.status("bl_read_peak_probe", 1 << 20, 16, 64, 0, None, None) == 1
+    assert _lib.status("bl_read_peak_probe", (1 << 20) + 8, 16, 64, 0, 1 << 20, None) == 3
+
+
 @pytest.mark.parametrize("kind,pair,iters", [(3, 0, 10), (-1, 0, 10), (0, 2, 10), (0, 0, 0), (1, 1, (1 << 20) + 1)])
 def test_peak_probe_validation(L, kind, pair, iters):
     assert _lib.status("bl_mma_peak_probe", kind, pair, iters, None, None) == 1
