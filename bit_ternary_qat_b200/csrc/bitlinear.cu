@@ -1276,6 +1276,8 @@ bl_status bl_read_peak_probe(const uint8_t* buf, int64_t rows, int64_t row_bytes
                "rows must be a positive multiple of 16 (at most 2^30), got %lld", (long long)rows);
     BL_REQUIRE(row_bytes >= 64 && row_bytes % 64 == 0 && row_bytes <= (1 << 24), BL_ERR_UNSUPPORTED_SHAPE,
                "row_bytes must be a positive multiple of 64 (at most 2^24), got %lld", (long long)row_bytes);
+    // keeps a block's step count (32-bit in the kernel) in range
+    BL_REQUIRE(rows * row_bytes <= (int64_t(1) << 40), BL_ERR_UNSUPPORTED_SHAPE, "buffer larger than 2^40 bytes");
     DeviceInfo dev;
     BL_TRY(current_device(&dev));
     cudaStream_t st = static_cast<cudaStream_t>(stream);

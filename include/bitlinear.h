@@ -374,7 +374,7 @@ BL_API bl_status bl_mma_peak_probe(int kind, int pair, int iters, double* ops_ou
  * per SM, balanced 16-row groups, 64-byte column steps, 8 rows x 64 bytes per warp load);
  * pattern 1 reads contiguous equal spans per block, 512 bytes per warp load.  rows: a
  * positive multiple of 16 (at most 2^30); row_bytes: a positive multiple of 64 (at most
- * 2^24); buf 16-byte aligned.  sink: one device uint32 that the kernel writes only if the
+ * 2^24); rows x row_bytes at most 2^40; buf 16-byte aligned.  sink: one device uint32 that the kernel writes only if the
  * XOR of all loads equals a fixed constant (the buffer's owner may ignore it).  Launched with
  * programmatic dependent launch like the GEMV; time it with CUDA events on `stream`. */
 BL_API bl_status bl_read_peak_probe(const uint8_t* buf, int64_t rows, int64_t row_bytes, int pattern, uint32_t* sink,

@@ -182,7 +182,8 @@ def test_status_values_match_header():
 
 
 @pytest.mark.parametrize("rows,row_bytes,pattern,status", [(16, 64, 2, 1), (16, 64, -1, 1), (8, 64, 0, 2), (24, 64, 1, 2),
-                                                         (16, 32, 0, 2), (16, 96, 0, 2), (0, 64, 0, 2)])
+                                                         (16, 32, 0, 2), (16, 96, 0, 2), (0, 64, 0, 2),
+                                                         (1 << 30, 1 << 14, 0, 2)])
 def test_read_probe_validation(L, rows, row_bytes, pattern, status):
     """The read probe rejects a bad pattern or shape before touching the (fake, aligned) pointers."""
     fake = 1 << 20
