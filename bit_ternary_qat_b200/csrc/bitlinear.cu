@@ -539,17 +539,10 @@ bl_status run_rmsnorm_bwd(const void* X, bl_dtype dt, const float* rinv, const f
 // ------------------------------------------------------------------------------------
 // packed-weight GEMM: tile shape, K split and launch
 // ------------------------------------------------------------------------------------
-// Work units per wave: the fraction of the last wave's SMs that have work.
-inline double wave_eff(int64_t units, int sms) {
-    const int64_t waves = (units + sms - 1) / sms;
-    return static_cast<double>(units) / static_cast<double>(waves * sms);
-}
-
-
 // Packed-weight GEMM on CTA pairs: 256-row weight tiles x bt tokens
-// (bt = T rounded up to 32, at most 256), the same K-split rule as the 1-SM kernel counted
-// in pairs, the activation ring, and the packed ring in the rest of shared memory.  The grid
-// is as many pairs as fit at once, at most one per unit.
+// (bt = T rounded up to 32, at most 256), a K split when the tiles fill at most half the
+// pairs, the activation ring, and the packed ring in the rest of shared memory.  The grid is
+// as many pairs as fit at once, at most one per unit.
 template <bool kBf16Out>
 bl_status launch_packed2(const int8_t* Xq, const float* sx, int64_t T, int64_t K, const uint8_t* Wpacked,
                          const float* gamma, int64_t N, void* Y, int32_t* acc, int32_t* scratch,
@@ -597,18 +590,10 @@ bl_status launch_packed2(const int8_t* Xq, const float* sx, int64_t T, int64_t K
     }
     const int64_t base = (int64_t)a.n_tiles * a.t_tiles;
     int splits = 1;
-    if (bt <= 64) {
-        int smax = std::min<int64_t>(8, a.k_blocks / 2);
-        smax = (int)std::min<int64_t>(smax, K / (64 * T));
-        smax = (int)std::min<int64_t>(smax, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));
-        double best = wave_eff(base, mc);
-        for (int sp = 2; sp <= smax; ++sp) best = std::max(best, wave_eff(base * sp, mc));
-        for (int sp = 1; sp <= std::max(1, smax); ++sp)
-            if (wave_eff(base * sp, mc) >= best - 0.03) { splits = sp; break; }
-    } else if (2 * base <= mc) {
-        // wider token tiles: the partial sums cost more than a second wave returns, so split only
-        // when the tiles fill at most half the pairs, into as many units as one wave holds, each
-        // at least 8 k-blocks (4 stages) long
+    if (2 * base <= mc) {
+        // the partial sums and their second launch cost more than a second wave of units
+        // returns, so K is split only when the tiles fill at most half the pairs, into as many
+        // units as one wave holds, each at least 8 k-blocks (4 stages) long
         int64_t sp = std::min<int64_t>(8, (int64_t)mc / base);
         sp = std::min<int64_t>(sp, a.k_blocks / 8);
         sp = std::min<int64_t>(sp, (int64_t)(scratch_bytes / ((size_t)T * N * sizeof(int32_t))));

@@ -316,11 +316,10 @@ BL_API bl_status ternary_gemv_rows(const uint8_t* Wpacked, const float* gamma_ro
  *     GEMV's kernel (codes decoded in registers, warp-level int8 MMA; ws unused);
  *   otherwise: CTA pairs with 256 weight rows x up to 256 tokens per tile (codes decoded
  *     into tensor memory, 2-SM tcgen05 MMAs, TMA-stored output).
- * When the weight tiles alone cannot fill the GPU, K may be split: split sp stores its exact
- * int32 partial sums to slice sp of ws (int32 [splits x T x N]) and a second launch adds the
- * slices in split order and applies the scale.  The split count is limited by
- * ws_bytes / (4 T N) (ws NULL: no split) and by 8; up to 64 tokens also by K / (64 T), above
- * that to tiles that fill at most half the CTA pairs, by K / 1024 and by one wave of pairs.
+ * When the weight tiles fill at most half of the CTA pairs, K may be split: split sp stores
+ * its exact int32 partial sums to slice sp of ws (int32 [splits x T x N]) and a second launch
+ * adds the slices in split order and applies the scale.  The split count is limited by
+ * ws_bytes / (4 T N) (ws NULL: no split), by 8, by K / 1024 and by one wave of pairs.
  * One or two launches. */
 BL_API bl_status bitlinear_linear_packed(const int8_t* Xq, const float* sx, int64_t T, int64_t K,
                                   const uint8_t* Wpacked, const float* gamma, int64_t N,

@@ -131,9 +131,9 @@ def test_linear_packed_short_last_units(bl, T, K, N):
 
 
 def test_linear_packed_split_with_single_k_block_stages(bl):
-    """K = 5440 (42.5 k-blocks) at 20 tokens on 512 rows: two pair tiles, so K is split -- three
-    ways by the launcher's rule (14 / 14 / 15 k-blocks); the last split ends in a one-k-block
-    stage, the half k-block of the K tail."""
+    """K = 5440 (42.5 k-blocks) at 20 tokens on 512 rows: two pair tiles, so K is split -- five
+    ways by the launcher's rule (8 / 9 / 8 / 9 / 9 k-blocks); the splits of 9 k-blocks end in a
+    one-k-block stage, the last of them on the half k-block of the K tail."""
     xq, packed, s = _case(20, 5440, 512, seed=11)
     for out in ("bf16", "f32"):
         _check(bl, xq, packed, s, 0.0173, out, True)
